@@ -1,0 +1,263 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+Each test names what it pins and the mistake it is there to catch. Nothing here calls the
+CUDA library.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------- generator
+
+def test_splitmix64_published_vector(golden_dir):
+    """Published SplitMix64 sequence for seed 1234567 (catches a wrong constant or shift)."""
+    kat = _load(golden_dir, "splitmix64_kat.json")
+    got = [int(O.splitmix64_draws(np.uint64(kat["seed"]), t)) for t in range(5)]
+    assert got == [int(v) for v in kat["outputs"]]
+
+
+def test_draws_are_counter_based():
+    """draw(key, t) equals the t-th output of the sequential generator for every t."""
+    key = np.uint64(0xDEADBEEFCAFEF00D)
+    state = int(key)
+    for t in range(50):
+        state = (state + O.GAMMA) % (1 << 64)
+        assert int(O.splitmix64_draws(key, t)) == int(O.mix64(np.uint64(state)))
+
+
+def test_fisher_yates_is_uniform():
+    """All 24 permutations of 4 items appear equally often over many independent blocks.
+
+    A Sattolo-style off-by-one (j in [0, i)) yields only the 6 cyclic permutations, and a
+    naive 'swap with any position' shuffle is biased; both fail the chi-square bound.
+    """
+    n = 48000
+    keys = O.block_key(12345, np.arange(n))
+    perm = O.block_permutation(keys, 4)
+    counts = {}
+    for p in map(tuple, perm):
+        counts[p] = counts.get(p, 0) + 1
+    assert len(counts) == 24
+    exp = n / 24
+    chi2 = sum((v - exp) ** 2 / exp for v in counts.values())
+    assert chi2 < 60.0  # 23 dof: P(chi2 > 60) ~ 4e-5
+
+
+def test_fisher_yates_positions_uniform_bk128():
+    """Each value lands in each position with probability 1/BK (BK = 128)."""
+    BK, n = 128, 4000
+    perm = O.block_permutation(O.block_key(7, np.arange(n)), BK)
+    for row in perm[:50]:
+        assert sorted(row.tolist()) == list(range(BK))
+    # position of value 0 and of value BK-1: uniform over [0, BK)
+    for v in (0, BK - 1):
+        pos = np.argmax(perm == v, axis=1)
+        hist = np.bincount(pos // 16, minlength=8)
+        exp = n / 8
+        chi2 = float(((hist - exp) ** 2 / exp).sum())
+        assert chi2 < 30.0  # 7 dof
+
+
+def test_signs_balanced_and_independent_of_perm():
+    g = O.block_signs(O.block_key(99, np.arange(2000)), 64).astype(np.int64)
+    frac = (g == 1).mean()
+    assert abs(frac - 0.5) < 0.01
+    assert set(np.unique(g).tolist()) == {-1, 1}
+
+
+# ---------------------------------------------------------------------------- tables
+
+@pytest.mark.parametrize("K,N,c,BK,BN,seed", [
+    (768, 768, 2, 64, 64, 0),
+    (1280, 512, 4, 128, 128, 2),
+    (1024, 256, 8, 256, 128, 3),
+    (512, 256, 8, 128, 128, 4),
+    (512, 256, 1, 128, 128, 4),
+])
+def test_table_invariants(K, N, c, BK, BN, seed):
+    """Every chunk maps onto its own S columns, exactly c inputs per column, signs +-1."""
+    h, g = O.ss1_tables(K, N, c, BK, BN, seed)
+    NB, KC, S = N // BN, K // BK, BK // c
+    assert h.shape == (NB, K) and g.shape == (NB, K)
+    assert set(np.unique(g).tolist()) <= {-1, 1}
+    for nb in range(NB):
+        for kc in range(KC):
+            hh = h[nb, kc * BK:(kc + 1) * BK]
+            assert hh.min() >= kc * S and hh.max() < (kc + 1) * S
+            assert np.all(np.bincount(hh - kc * S, minlength=S) == c)
+    if c == 1:
+        assert np.array_equal(h, np.broadcast_to(np.arange(K), (NB, K)))
+        assert np.all(g == 1)
+
+
+def test_tables_independent_per_block_and_seed():
+    h, g = O.ss1_tables(1024, 512, 2, 128, 128, 5)
+    blocks = [(h[nb, kc * 128:(kc + 1) * 128] - kc * 64).tobytes() for nb in range(4) for kc in range(8)]
+    assert len(set(blocks)) == len(blocks)
+    h2, _ = O.ss1_tables(1024, 512, 2, 128, 128, 6)
+    assert not np.array_equal(h, h2)
+    h3, g3 = O.ss1_tables(1024, 512, 2, 128, 128, 5)
+    assert np.array_equal(h, h3) and np.array_equal(g, g3)
+
+
+def test_fold_is_mod_S():
+    """hl(k) = perm[k] mod S: recomputed from the permutation of one block."""
+    K, N, c, BK, BN, seed = 256, 128, 4, 128, 128, 11
+    h, _ = O.ss1_tables(K, N, c, BK, BN, seed)
+    S = BK // c
+    perm = O.block_permutation(O.block_key(seed, [1]), BK)[0]   # block id 1 = (nb 0, kc 1)
+    assert np.array_equal(h[0, BK:2 * BK] - S, perm % S)
+
+
+def test_tables_regression(golden_dir):
+    ref = _load(golden_dir, "tables_regression.json")
+    for case in ref["cases"]:
+        K, N, c, BK, BN, seed = (case[k] for k in ("K", "N", "c", "BK", "BN", "seed"))
+        h, g = O.ss1_tables(K, N, c, BK, BN, seed)
+        assert h[0, :BK].tolist() == case["h_nb0_kc0"]
+        assert g[0, :BK].tolist() == case["g_nb0_kc0"]
+        assert h[-1, K - BK:K - BK + 16].tolist() == case["h_last16"]
+        assert g[-1, K - BK:K - BK + 16].tolist() == case["g_last16"]
+
+
+@pytest.mark.parametrize("c", [1, 2, 4, 8])
+def test_sketch_gram_identity(c):
+    """S^T S = c I for every block's sketch operator (count-sketch with balanced buckets)."""
+    K, N, BK, BN = 512, 256, 128, 128
+    h, g = O.ss1_tables(K, N, c, BK, BN, 3)
+    for nb in range(N // BN):
+        Sk = O.sketch_matrix(h, g, nb, K, K // c)
+        assert np.array_equal(Sk.T @ Sk, c * np.eye(K // c))
+
+
+# ---------------------------------------------------------------------------- forward
+
+def test_handworked_examples(golden_dir):
+    ref = _load(golden_dir, "handworked_forward.json")
+    for case in ref["cases"]:
+        h = np.array(case["h"], dtype=np.int32)
+        g = np.array(case["g"], dtype=np.int8)
+        X = np.array(case["X"], dtype=np.float64)
+        Wc = np.array(case["Wc"], dtype=np.float64)
+        want = np.array(case["Y"], dtype=np.float64)
+        assert np.array_equal(O.ss1_forward(X, Wc, h, g, case["BN"]), want), case["name"]
+        assert np.array_equal(O.ss1_forward_sketch(X, Wc, h, g, case["BN"]), want), case["name"]
+
+
+def test_c1_is_dense_gemm():
+    """With c = 1 (identity hash) the layer is X Wc^T (catches a transposed operand)."""
+    rng = np.random.default_rng(0)
+    M, K, N = 7, 256, 384
+    X = rng.standard_normal((M, K))
+    Wc = rng.standard_normal((N, K))
+    h, g = O.ss1_tables(K, N, 1, 128, 128, 4)
+    np.testing.assert_allclose(O.ss1_forward(X, Wc, h, g, 128), X @ Wc.T, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("K,N,c,BK,BN", [(64, 32, 2, 16, 8), (256, 256, 4, 64, 64), (512, 256, 8, 256, 128),
+                                         (768, 768, 2, 64, 64)])
+def test_two_routes_agree(K, N, c, BK, BN):
+    """Definition (expanded tied weight) and sketch-then-multiply agree to fp64 rounding."""
+    rng = np.random.default_rng(K + N + c)
+    X = rng.standard_normal((9, K))
+    Wc = rng.standard_normal((N, K // c))
+    h, g = O.ss1_tables(K, N, c, BK, BN, 1)
+    a = O.ss1_forward(X, Wc, h, g, BN)
+    b = O.ss1_forward_sketch(X, Wc, h, g, BN)
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-11 * np.abs(a).max())
+
+
+@pytest.mark.parametrize("c", [1, 2, 4, 8])
+def test_frobenius_identity(c):
+    """Each row of the tied weight holds every Wc entry of its row exactly c times, +-1:
+    ||W_full[n,:]||^2 = c ||Wc[n,:]||^2 (catches a dropped or duplicated term)."""
+    K, N, BK, BN = 512, 256, 128, 128
+    rng = np.random.default_rng(c)
+    Wc = rng.standard_normal((N, K // c))
+    h, g = O.ss1_tables(K, N, c, BK, BN, 8)
+    W = np.concatenate([O.expand_weight(Wc, h, g, BN, nb) for nb in range(N // BN)])
+    np.testing.assert_allclose((W ** 2).sum(1), c * (Wc ** 2).sum(1), rtol=1e-12)
+
+
+def test_one_hot_probe_structure():
+    """Probing the forward with the identity (X = I_K) returns the tied weight. With all Wc
+    entries distinct, each probed value decodes to one (n, j): j must lie in the chunk's
+    column range, every j of a chunk must appear exactly c times per neuron, the map must be
+    the same for the neurons of one block and differ between blocks."""
+    K, N, c, BK, BN = 256, 64, 4, 64, 16
+    Kc = K // c
+    Wc = (np.arange(N)[:, None] * 1000 + np.arange(Kc)[None, :] + 1).astype(np.float64)
+    h, g = O.ss1_tables(K, N, c, BK, BN, 21)
+    Wt = O.ss1_forward(np.eye(K), Wc, h, g, BN)            # [K, N] = W_full^T
+    mag = np.abs(Wt)
+    nrow = (mag // 1000).astype(np.int64)
+    j = (mag - nrow * 1000 - 1).astype(np.int64)
+    assert np.all(nrow == np.arange(N)[None, :])
+    S = BK // c
+    maps = []
+    for n in range(N):
+        col = j[:, n]
+        for kc in range(K // BK):
+            seg = col[kc * BK:(kc + 1) * BK]
+            assert seg.min() >= kc * S and seg.max() < (kc + 1) * S
+            assert np.all(np.bincount(seg - kc * S, minlength=S) == c)
+        maps.append((col.tobytes(), np.sign(Wt[:, n]).tobytes()))
+    for nb in range(N // BN):
+        assert len(set(maps[nb * BN:(nb + 1) * BN])) == 1
+    assert len(set(maps[::BN])) == N // BN
+
+
+def test_linearity_and_sign_symmetry():
+    rng = np.random.default_rng(5)
+    K, N, c, BK, BN = 256, 128, 2, 128, 64
+    h, g = O.ss1_tables(K, N, c, BK, BN, 2)
+    Wc = rng.standard_normal((N, K // c))
+    X1, X2 = rng.standard_normal((4, K)), rng.standard_normal((4, K))
+    f = lambda X: O.ss1_forward(X, Wc, h, g, BN)  # noqa: E731
+    np.testing.assert_allclose(f(2.5 * X1 - 1.5 * X2), 2.5 * f(X1) - 1.5 * f(X2), rtol=1e-10, atol=1e-10)
+    assert np.array_equal(f(np.zeros((3, K))), np.zeros((3, N)))
+    assert np.array_equal(f(-X1), -f(X1))
+
+
+def test_rows_sample_matches_full():
+    rng = np.random.default_rng(6)
+    K, N, c, BK, BN = 256, 256, 4, 128, 128
+    h, g = O.ss1_tables(K, N, c, BK, BN, 2)
+    X = rng.standard_normal((33, K))
+    Wc = rng.standard_normal((N, K // c))
+    full = O.ss1_forward(X, Wc, h, g, BN)
+    rows = [0, 5, 32]
+    assert np.array_equal(O.ss1_forward_rows(X, Wc, h, g, BN, rows), full[rows])
+
+
+# ---------------------------------------------------------------------------- projection
+
+def test_projection_recovers_tied_weights():
+    """Projecting an SS1 tied weight returns its Wc; the residual of a dense W is
+    orthogonal to the SS1 subspace (least squares, from S^T S = c I)."""
+    rng = np.random.default_rng(7)
+    K, N, c, BK, BN = 256, 128, 4, 64, 32
+    h, g = O.ss1_tables(K, N, c, BK, BN, 9)
+    Wc = rng.standard_normal((N, K // c))
+    Wfull = np.concatenate([O.expand_weight(Wc, h, g, BN, nb) for nb in range(N // BN)])
+    np.testing.assert_allclose(O.project_dense(Wfull, h, g, BN, c), Wc, rtol=1e-12, atol=1e-12)
+    W = rng.standard_normal((N, K))
+    P = O.project_dense(W, h, g, BN, c)
+    Wp = np.concatenate([O.expand_weight(P, h, g, BN, nb) for nb in range(N // BN)])
+    R = W - Wp
+    # residual is orthogonal to every tied direction: projecting it gives zero
+    np.testing.assert_allclose(O.project_dense(R, h, g, BN, c), 0.0, atol=1e-12)
+    assert math.isclose((W * W).sum(), (Wp * Wp).sum() + (R * R).sum(), rel_tol=1e-12)

@@ -1,0 +1,43 @@
+"""Host-side checks of the seeded workloads and of the parity metric (no GPU)."""
+
+import numpy as np
+import torch
+
+from structured_compressed_linear_b200.workloads import WORKLOADS, make_inputs, instance_seed
+from tests._parity import row_normalised_max_err
+
+
+def test_workload_shapes_are_valid_ss1_layers():
+    for wid, layers in WORKLOADS.items():
+        for L in layers:
+            assert L.K % L.BK == 0 and L.N % L.BN == 0 and L.BK % L.c == 0, L
+            assert L.BK <= 256
+    assert len(WORKLOADS[4]) == 24 and len(WORKLOADS[5]) == 19
+
+
+def test_inputs_deterministic_and_distinct():
+    L = WORKLOADS[2][1].with_M(64)
+    X1, W1 = make_inputs(L)
+    X2, W2 = make_inputs(L)
+    assert torch.equal(X1, X2) and torch.equal(W1, W2)
+    assert X1.dtype == torch.bfloat16 and X1.shape == (64, 768) and W1.shape == (768, 384)
+    seeds = {instance_seed(L) for ws in WORKLOADS.values() for L in ws}
+    assert len(seeds) == sum(len(ws) for ws in WORKLOADS.values())
+
+
+def test_outlier_rows():
+    L = WORKLOADS[3][1].with_M(1000)
+    X, Wc = make_inputs(L)
+    rn = X.float().abs().amax(dim=1)
+    assert int((rn > 12).sum()) >= 9          # ~1% of rows scaled x20
+    bound = 1.0 / np.sqrt(L.K)
+    assert float(Wc.float().abs().max()) <= bound * 1.01
+
+
+def test_parity_metric():
+    ref = np.array([[1.0, -2.0, 0.5], [100.0, 0.0, 1.0]])
+    y = ref.copy()
+    y[0, 1] += 0.02
+    y[1, 2] += 1.0
+    assert abs(row_normalised_max_err(y, ref) - 0.01) < 1e-12
+    assert row_normalised_max_err(ref, ref) == 0.0
