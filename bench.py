@@ -1,0 +1,423 @@
+"""Benchmark of the SS1 layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID]
+
+One step = the forward of every layer of the workload (default: the four GPT-2 Small shaped
+SS1 layers, M = 8192 tokens, c = 2, BK = BN = 128, bf16 with fp32 accumulation) on seeded
+synthetic inputs already resident in HBM. L2 is flushed (a 256 MiB write, outside the event
+brackets) before every timed step. Each layer launch is bracketed by CUDA events on the
+launching stream; ms_per_step is the mean over the K timed steps of the summed layer times,
+max over ranks. Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun): the rows of X are independent, so every rank runs its own batch of M
+rows with replicated weights and tables and no data-path collective (weak scaling); the value
+is the whole-job dense-equivalent throughput, all ranks' work over the slowest rank's time.
+
+--impl reference times the CPU oracle (the plain float64 definition) on the host cores on a
+bounded row sample of the same workload and prints the same line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SS1 layer ms & dense-equiv TFLOP/s on 1 B200; achieved fraction of roofline"
+UNIT = "TFLOP/s (dense-equivalent 2*M*N*K per layer)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_work(L):
+    """Algorithmic work of one layer: dense-equivalent flops, actual flops, bytes moved."""
+    e = 2 if L.dtype == "bf16" else 4
+    dense = 2.0 * L.M * L.N * L.K
+    adds = float(L.M) * (L.N // L.BN) * L.K * (1.0 - 1.0 / L.c)
+    actual = 2.0 * L.M * L.N * L.K / L.c + adds
+    byts = float(e) * (L.M * L.K + L.N * L.K // L.c + L.M * L.N)
+    return dense, actual, byts
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "structured_compressed_linear_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel_name):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(kernel_name)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index):
+        self.ok = False
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def prepare_oracle(layers, max_rows=None):
+    """Inputs and tables for the CPU oracle's row sample (prepared once, not timed)."""
+    import oracle as O
+    from structured_compressed_linear_b200.workloads import make_inputs
+    prepared = []
+    for L in layers:
+        X, Wc = make_inputs(L if max_rows is None else L.with_M(min(L.M, max_rows)))
+        h, g = O.ss1_tables(L.K, L.N, L.c, L.BK, L.BN, L.seed)
+        prepared.append((L, X.double().numpy(), Wc.double().numpy(), h, g))
+    return prepared
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max(i.get("num_threads", 0) for i in threadpool_info())
+        if n:
+            return n
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_pass(prepared, rows):
+    import oracle as O
+    t0 = time.perf_counter()
+    dense = 0.0
+    for L, X, Wc, h, g in prepared:
+        r = min(rows, X.shape[0])
+        O.ss1_forward(X[:r], Wc, h, g, L.BN)
+        dense += 2.0 * r * L.N * L.K
+    return dense, time.perf_counter() - t0
+
+
+def oracle_sample_rate(prepared, budget_s, rows_per_layer=None):
+    """Times the CPU oracle (float64 definition) on a row sample of every layer.
+
+    Without a given sample size, the sample grows until one pass takes about budget_s
+    (or covers every prepared row). Returns (dense-equivalent TFLOP/s, seconds, rows)."""
+    max_rows = max(p[1].shape[0] for p in prepared)
+    if rows_per_layer is None:
+        rows = 64
+        while True:
+            _, dt = _oracle_pass(prepared, rows)
+            if dt >= budget_s / 2 or rows >= max_rows:
+                break
+            rows = int(min(max_rows, rows * max(2.0, 0.8 * budget_s / max(dt, 1e-6))))
+        rows_per_layer = rows
+    dense, dt = 0.0, 0.0
+    while dt < min(budget_s, 3.0) or dense == 0.0:      # repeat short samples for a stable time
+        d, t = _oracle_pass(prepared, rows_per_layer)
+        dense, dt = dense + d, dt + t
+    return dense / dt / 1e12, dt, rows_per_layer
+
+
+def run_reference(args, layers, wid, rank, world):
+    if rank != 0:
+        return
+    cfg = workload_config(layers, wid, world)
+    prepared = prepare_oracle(layers, max_rows=2048)
+    threads = oracle_threads()
+    rows = None
+    for _ in range(args.warmup):
+        _, _, rows = oracle_sample_rate(prepared, 2.0, rows)
+    times = []
+    for _ in range(args.steps):
+        _, dt, rows = oracle_sample_rate(prepared, 2.0, rows)
+        times.append(dt)
+    mean_t = statistics.mean(times)
+    dense_sample = sum(2.0 * min(rows, L.M) * L.N * L.K for L in layers)
+    value = dense_sample / mean_t / 1e12
+    full_ms = sum(2.0 * L.M * L.N * L.K for L in layers) / (value * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"first {rows} rows of each layer per step (float64 definition, numpy BLAS); "
+                                   f"ms_per_step extrapolated to all rows (rows are independent)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(layers, wid, world):
+    L0 = layers[0]
+    return {
+        "workload": f"{L0.workload} (workload {wid}): " + ", ".join(f"{L.K}x{L.N}" for L in layers)
+                    + f" at M={L0.M} per GPU, c={L0.c}, BK={L0.BK}, BN={L0.BN}",
+        "layers": [{"M": L.M, "K": L.K, "N": L.N, "c": L.c, "BK": L.BK, "BN": L.BN} for L in layers],
+        "dtype_in": L0.dtype, "accumulate": "fp32", "parallelism": f"replicas x{world} (rows sharded, no collective)",
+        "l2": "flushed before every timed step (256 MiB write outside the event brackets)",
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from structured_compressed_linear_b200.workloads import WORKLOADS, BENCH_WORKLOAD
+    wid = args.workload or BENCH_WORKLOAD
+    layers = WORKLOADS[wid]
+    if len({L.M for L in layers}) != 1:
+        layers = [L for L in layers if L.M == max(x.M for x in layers)]
+
+    if args.impl == "reference":
+        run_reference(args, layers, wid, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from structured_compressed_linear_b200 import build
+    build.build()
+    from structured_compressed_linear_b200 import ss1
+    from structured_compressed_linear_b200.workloads import make_inputs, instance_seed  # noqa: F401
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    peaks, peak_src = load_peaks()
+    # inputs: every rank its own rows (seed offset by rank), shared weights and tables
+    objs = []
+    for L in layers:
+        X, Wc = make_inputs(L)
+        if rank:
+            g = torch.Generator().manual_seed(1000 + rank)
+            X = X[torch.randperm(X.shape[0], generator=g)]
+        layer = ss1.SS1Layer(L.K, L.N, L.c, L.BK, L.BN, L.seed)
+        Xd, Wd = X.to(dev), Wc.to(dev)
+        Yd = torch.empty((L.M, L.N), dtype=Xd.dtype, device=dev)
+        objs.append((L, layer, Xd, Wd, Yd, X))
+    kernels = [ss1.Kernel(layer.select_kernel(L.M, Xd.dtype)).name for (L, layer, Xd, *_r) in objs]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        for i, (L, layer, Xd, Wd, Yd, _) in enumerate(objs):
+            if evs is not None:
+                evs[i][0].record(stream)
+            layer.forward(Xd, Wd, out=Yd)
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    for (L, layer, *_r) in objs:
+        st, detail = layer.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {detail:#x} during warm-up")
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in objs]
+           for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        for s in range(K):
+            flush.zero_()
+            step(evs[s])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    per_layer_ms = [[evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)] for i in range(len(objs))]
+    layer_ms = [statistics.mean(v) for v in per_layer_ms]
+    step_ms = sum(layer_ms)
+    t = torch.tensor([step_ms] + layer_ms, dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, layer_ms = float(t[0]), [float(x) for x in t[1:]]
+
+    # end to end through the public API: pinned host X -> device, forward, device -> pinned host Y
+    e2e = None
+    if not args.no_e2e:
+        hostX = [x.pin_memory() for (*_r, x) in objs]
+        hostY = [torch.empty((L.M, L.N), dtype=Xd.dtype).pin_memory() for (L, _l, Xd, *_r) in objs]
+        h2d = sum(x.numel() * x.element_size() for x in hostX)
+        d2h = sum(y.numel() * y.element_size() for y in hostY)
+
+        def e2e_step():
+            for (L, layer, Xd, Wd, Yd, _), hx, hy in zip(objs, hostX, hostY):
+                Xd.copy_(hx, non_blocking=True)
+                layer.forward(Xd, Wd, out=Yd)
+                hy.copy_(Yd, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(3, min(K, 20))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / ke], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = (float(te[0]), h2d, d2h)
+
+    dense_step = sum(layer_work(L)[0] for L in layers)
+    value = world * dense_step / (step_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel over the step (sum over its launches)
+    tc_peak = peaks["bf16_tflops"] * 1e12
+    hbm_peak = peaks["hbm_gbs"] * 1e9
+    t_tc = sum(layer_work(L)[1] / tc_peak for L in layers)
+    t_hbm = sum(layer_work(L)[2] / hbm_peak for L in layers)
+    t_kernel = sum(layer_ms) * 1e-3
+    ns_frac = sum(max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) for L in layers) / t_kernel
+    if t_tc >= t_hbm:
+        achieved = sum(layer_work(L)[1] for L in layers) / t_kernel / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        achieved = sum(layer_work(L)[2] for L in layers) / t_kernel / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_src} (burst figure; MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    dom = max(set(kernels), key=kernels.count)
+    rec = traffic_record(dom)
+    roof["traffic"] = rec["dram_bytes_per_step"] if rec else None
+    roof["kernel"] = dom
+    roof["frac_slower_of_tensor_and_hbm"] = ns_frac
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if layers[0].dtype == "bf16" else "fp32", "data": "synthetic (seeded, shapes of the workload)",
+        "config": workload_config(layers, wid, world),
+        "layers": [{"K": L.K, "N": L.N, "M": L.M, "c": L.c, "kernel": k, "ms": ms,
+                    "dense_tflops": layer_work(L)[0] / (ms * 1e-3) / 1e12,
+                    "actual_tflops": layer_work(L)[1] / (ms * 1e-3) / 1e12,
+                    "gbs": layer_work(L)[2] / (ms * 1e-3) / 1e9,
+                    "roofline_frac": max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) / (ms * 1e-3)}
+                   for L, k, ms in zip(layers, kernels, layer_ms)],
+        "roofline": roof,
+        "gpu_launches": K * len(objs),
+        "clocks": sampler.summary(),
+    }
+    if e2e is not None:
+        ms_e, h2d, d2h = e2e
+        line["e2e"] = {"value": world * dense_step / (ms_e * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_e,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "note": "X copied from pinned host memory and Y read back every step; Wc resident"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, rows = oracle_sample_rate(prepare_oracle(layers), 10.0)
+        rows = min(rows, layers[0].M)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                                "sample": f"first {rows} of {layers[0].M} rows of each layer (all {len(layers)} layers), "
+                                          f"float64 definition with numpy BLAS, {dt:.1f} s timed"}
+    for (L, layer, *_r) in objs:
+        st, detail = layer.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {detail:#x}")
+        layer.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+// C ABI of the SS1 layer forward: handles, argument checks, kernel choice, status words.
+// The operation and every entry point are specified in include/ss1.h.
+#include "ss1_internal.cuh"
+
+#include <mutex>
+#include <new>
+#include <unordered_set>
+
+namespace {
+
+constexpr uint64_t kMagic = 0x5353315F4C415945ull;  // "SS1_LAYE"
+constexpr int64_t kSmallMMax = 16;                   // AUTO: M <= this uses the decode path
+
+std::mutex g_mu;
+std::unordered_set<const ss1_layer*> g_live;
+
+bool live(const ss1_layer* h) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return h != nullptr && g_live.count(h) != 0 && h->magic == kMagic;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void release(ss1_layer* L) {
+    if (!L) return;
+    if (L->d_h) cudaFree(L->d_h);
+    if (L->d_g) cudaFree(L->d_g);
+    if (L->d_src) cudaFree(L->d_src);
+    if (L->status_host) cudaFreeHost(L->status_host);
+    L->magic = 0;
+    delete L;
+}
+
+int kernel_for(const ss1_layer& L, int64_t M, int dtype) {
+    if (dtype == SS1_DTYPE_FP32) return SS1_KERNEL_SIMT;
+    if (M <= kSmallMMax && ss1::smallm_supported(L, M)) return SS1_KERNEL_SMALLM;
+    if (ss1::tc_supported(L)) return SS1_KERNEL_TC;
+    return SS1_KERNEL_SIMT;
+}
+
+}  // namespace
+
+extern "C" {
+
+SS1_API const char* ss1_strerror(int status) {
+    switch (status) {
+        case SS1_OK: return "ok";
+        case SS1_ERR_INVALID_ARG: return "invalid argument";
+        case SS1_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs sm_100)";
+        case SS1_ERR_CUDA: return "CUDA error";
+        case SS1_ERR_OUT_OF_MEMORY: return "out of memory";
+        case SS1_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case SS1_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait (device status set)";
+        case SS1_ERR_BAD_HANDLE: return "bad or destroyed handle";
+        case SS1_ERR_UNSUPPORTED_SHAPE: return "the chosen kernel does not support this shape";
+        default: return "unknown status";
+    }
+}
+
+SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t seed, ss1_handle* out) {
+    if (!out) return SS1_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (K < 1 || N < 1 || BK < 1 || BN < 1) return SS1_ERR_INVALID_ARG;
+    if (!(c == 1 || c == 2 || c == 4 || c == 8)) return SS1_ERR_INVALID_ARG;
+    if (BK > 256 || BK % c != 0 || K % BK != 0 || N % BN != 0 || BN % 16 != 0) return SS1_ERR_INVALID_ARG;
+    if (K > (int64_t)1 << 30 || N > (int64_t)1 << 30) return SS1_ERR_INVALID_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    if (prop.major != 10) return SS1_ERR_UNSUPPORTED_DEVICE;
+
+    ss1_layer* L = new (std::nothrow) ss1_layer{};
+    if (!L) return SS1_ERR_OUT_OF_MEMORY;
+    L->magic = kMagic;
+    L->device = dev;
+    L->num_sms = prop.multiProcessorCount;
+    L->K = K; L->N = N; L->c = c; L->BK = BK; L->BN = BN; L->seed = seed;
+    L->S = BK / c; L->NB = (int)(N / BN); L->KC = (int)(K / BK);
+
+    const size_t entries = (size_t)L->NB * (size_t)K;
+    if (cudaMalloc(&L->d_h, entries * sizeof(int32_t)) != cudaSuccess ||
+        cudaMalloc(&L->d_g, entries * sizeof(int8_t)) != cudaSuccess ||
+        cudaMalloc(&L->d_src, entries * sizeof(uint16_t)) != cudaSuccess ||
+        cudaHostAlloc(&L->status_host, sizeof(int32_t), cudaHostAllocMapped) != cudaSuccess) {
+        cudaGetLastError();
+        release(L);
+        return SS1_ERR_OUT_OF_MEMORY;
+    }
+    *L->status_host = 0;
+    if (cudaHostGetDevicePointer((void**)&L->status_dev, L->status_host, 0) != cudaSuccess) {
+        cudaGetLastError();
+        release(L);
+        return SS1_ERR_CUDA;
+    }
+    if (ss1::launch_hashgen(*L, 0) != cudaSuccess || cudaStreamSynchronize(0) != cudaSuccess) {
+        cudaGetLastError();
+        release(L);
+        return SS1_ERR_CUDA;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_live.insert(L);
+    }
+    *out = L;
+    return SS1_OK;
+}
+
+SS1_API int ss1_destroy(ss1_handle h) {
+    if (!h) return SS1_OK;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_live.count(h) || h->magic != kMagic) return SS1_ERR_BAD_HANDLE;
+        g_live.erase(h);
+    }
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != h->device) cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    cudaGetLastError();
+    release(h);
+    if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+    return SS1_OK;
+}
+
+SS1_API int ss1_get_info(ss1_handle h, int64_t* K, int64_t* N, int* c, int* BK, int* BN) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    if (K) *K = h->K;
+    if (N) *N = h->N;
+    if (c) *c = h->c;
+    if (BK) *BK = h->BK;
+    if (BN) *BN = h->BN;
+    return SS1_OK;
+}
+
+SS1_API int ss1_get_tables(ss1_handle h, int32_t* h_host, int8_t* g_host) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    const size_t entries = (size_t)h->NB * (size_t)h->K;
+    if (h_host && cudaMemcpy(h_host, h->d_h, entries * sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return SS1_ERR_CUDA;
+    }
+    if (g_host && cudaMemcpy(g_host, h->d_g, entries * sizeof(int8_t), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return SS1_ERR_CUDA;
+    }
+    return SS1_OK;
+}
+
+SS1_API int ss1_device_status(ss1_handle h, int32_t* detail) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    const int32_t v = __atomic_exchange_n(h->status_host, 0, __ATOMIC_ACQ_REL);
+    if (detail) *detail = v;
+    return v == 0 ? SS1_OK : SS1_ERR_DEVICE_TIMEOUT;
+}
+
+SS1_API int ss1_select_kernel(ss1_handle h, int64_t M, int dtype, int* kernel) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    if (!kernel || M < 0 || (dtype != SS1_DTYPE_BF16 && dtype != SS1_DTYPE_FP32)) return SS1_ERR_INVALID_ARG;
+    *kernel = kernel_for(*h, M, dtype);
+    return SS1_OK;
+}
+
+SS1_API int ss1_forward_with(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype, int kernel,
+                             void* stream) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    if (M < 0 || (dtype != SS1_DTYPE_BF16 && dtype != SS1_DTYPE_FP32)) return SS1_ERR_INVALID_ARG;
+    if (M > ((int64_t)1 << 31) / 2) return SS1_ERR_INVALID_ARG;
+    if (*(volatile int32_t*)h->status_host != 0) return SS1_ERR_DEVICE_TIMEOUT;
+    if (M == 0) return SS1_OK;
+    if (!X || !Wc || !Y) return SS1_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Wc) || !aligned16(Y)) return SS1_ERR_MISALIGNED;
+    if (kernel == SS1_KERNEL_AUTO) kernel = kernel_for(*h, M, dtype);
+
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    int rc = SS1_OK;
+    switch (kernel) {
+        case SS1_KERNEL_SIMT:
+            e = ss1::launch_simt(*h, X, Wc, Y, M, dtype, st);
+            break;
+        case SS1_KERNEL_SMALLM:
+            if (dtype != SS1_DTYPE_BF16 || !ss1::smallm_supported(*h, M)) rc = SS1_ERR_UNSUPPORTED_SHAPE;
+            else e = ss1::launch_smallm(*h, X, Wc, Y, M, st);
+            break;
+        case SS1_KERNEL_TC:
+            if (dtype != SS1_DTYPE_BF16 || !ss1::tc_supported(*h)) rc = SS1_ERR_UNSUPPORTED_SHAPE;
+            else e = ss1::launch_tc(*h, X, Wc, Y, M, st);
+            break;
+        default:
+            rc = SS1_ERR_INVALID_ARG;
+    }
+    if (prev != h->device) cudaSetDevice(prev);
+    if (rc != SS1_OK) return rc;
+    if (e != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    return SS1_OK;
+}
+
+SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype, void* stream) {
+    return ss1_forward_with(h, X, Wc, Y, M, dtype, SS1_KERNEL_AUTO, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Device generator of the SS1 hash and sign tables.
+//
+// "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+// "Approach": K- and N-coalescing hash functions tie the weights inside one neuron's weight
+// vector. The family is fixed here as: per (N-block nb, K-chunk kc) a seeded random map of
+// the BK chunk inputs onto S = BK / c slots, exactly c inputs per slot, random signs.
+//
+// Generator (one thread per block id b = nb * KC + kc, all integer arithmetic, so the result
+// is bit-reproducible on any machine):
+//   key      = seed ^ mix64(b + 1)                         mix64 = SplitMix64 finaliser
+//   draw(t)  = mix64(key + (t + 1) * 0x9E3779B97F4A7C15)   SplitMix64, counter form
+//   shuffle  : for i = BK-1 .. 1 (draw t = BK-1-i): j = hi32(draw) * (i + 1) >> 32;
+//              swap perm[i], perm[j]                       (Durstenfeld; Lemire reduction)
+//   signs    : g(k) = -1 if bit 63 of draw(BK - 1 + k) is set, else +1
+//   fold     : slot(k) = perm[k] mod S; the j-th source of slot s is the input k with
+//              perm[k] == s + j * S
+//   c == 1   : identity, all signs +1, no draws.
+#include "ss1_internal.cuh"
+
+namespace ss1 {
+namespace {
+
+constexpr uint64_t kGolden = 0x9E3779B97F4A7C15ull;
+
+__device__ __forceinline__ uint64_t splitmix_finalise(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int KC, int BK, int c, int S, int nblocks,
+                                                      int32_t* __restrict__ h, int8_t* __restrict__ g,
+                                                      uint16_t* __restrict__ src) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const int nb = b / KC, kc = b % KC;
+    int32_t* hrow = h + (size_t)nb * K + (size_t)kc * BK;
+    int8_t* grow = g + (size_t)nb * K + (size_t)kc * BK;
+    uint16_t* sb = src + (size_t)b * S * c;
+
+    if (c == 1) {
+        for (int k = 0; k < BK; ++k) {
+            hrow[k] = kc * S + k;
+            grow[k] = 1;
+            sb[k] = (uint16_t)k;
+        }
+        return;
+    }
+
+    uint8_t perm[256];   // value at each position
+    uint8_t where[256];  // inverse: position -> input
+    for (int k = 0; k < BK; ++k) perm[k] = (uint8_t)k;
+    const uint64_t key = seed ^ splitmix_finalise((uint64_t)b + 1ull);
+    uint64_t state = key;
+    for (int i = BK - 1; i >= 1; --i) {
+        state += kGolden;                                   // draw t = BK-1-i
+        const uint64_t r = splitmix_finalise(state);
+        const uint32_t j = (uint32_t)(((r >> 32) * (uint64_t)(i + 1)) >> 32);
+        const uint8_t tmp = perm[i];
+        perm[i] = perm[j];
+        perm[j] = tmp;
+    }
+    for (int k = 0; k < BK; ++k) {
+        state += kGolden;                                   // draw t = BK-1+k
+        const uint64_t r = splitmix_finalise(state);
+        const bool neg = (r >> 63) != 0;
+        hrow[k] = kc * S + (int)perm[k] % S;
+        grow[k] = neg ? (int8_t)-1 : (int8_t)1;
+        where[perm[k]] = (uint8_t)k;
+    }
+    for (int s = 0; s < S; ++s) {
+        for (int j = 0; j < c; ++j) {
+            const int k = where[s + j * S];
+            sb[s * c + j] = (uint16_t)(k | (grow[k] < 0 ? kSrcNegBit : 0));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st) {
+    const int nblocks = L.NB * L.KC;
+    const int threads = 128;
+    hashgen_kernel<<<(nblocks + threads - 1) / threads, threads, 0, st>>>(
+        L.seed, (int)L.K, L.KC, L.BK, L.c, L.S, nblocks, L.d_h, L.d_g, L.d_src);
+    return cudaGetLastError();
+}
+
+}  // namespace ss1

@@ -1,0 +1,51 @@
+// Internal declarations shared by the SS1 CUDA sources (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ss1.h"
+
+// Kernel-side table entry: the chunk-local input index of one slot source and its sign.
+//   bits 0..7  : k_local in [0, BK)  (BK <= 256)
+//   bit  15    : 1 if the sign is -1
+// Layout of the slot-major table: src[((nb * KC + kc) * S + s) * c + j], j = 0..c-1, where
+// the j-th source of slot s is the input whose permuted position is s + j * S.
+static constexpr uint16_t kSrcNegBit = 0x8000u;
+static constexpr uint16_t kSrcIdxMask = 0x00FFu;
+
+struct ss1_layer {
+    uint64_t magic;
+    int device;
+    int num_sms;
+    int64_t K, N;
+    int c, BK, BN, S, NB, KC;
+    uint64_t seed;
+    int32_t* d_h;        // [NB][K] compressed column of input k in block nb
+    int8_t* d_g;         // [NB][K] sign of input k in block nb
+    uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
+    int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
+    int32_t* status_dev;   // device alias of status_host
+};
+
+namespace ss1 {
+
+// Device status codes written by kernels with bounded waits: (kernel id << 8) | wait site.
+enum : int32_t { kStatusKernelTC = 1 };
+
+cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);
+
+// General CUDA-core path: any valid shape, bf16 or fp32.
+cudaError_t launch_simt(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
+                        cudaStream_t st);
+
+// Decode-sized M (bf16): streams Wc once.
+bool smallm_supported(const ss1_layer& L, int64_t M);
+cudaError_t launch_smallm(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M,
+                          cudaStream_t st);
+
+// Tensor-core path (bf16, tcgen05 + TMEM + TMA).
+bool tc_supported(const ss1_layer& L);
+cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
+
+}  // namespace ss1

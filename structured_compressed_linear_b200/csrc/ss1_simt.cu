@@ -1,0 +1,122 @@
+// General CUDA-core SS1 forward: sketch on chip, then an FMA GEMM against Wc.
+//
+// "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform",
+// section "Approach": the input is first sketched (signed additions reduce it by the
+// compression factor c) and then multiplied with the compressed weights.
+//
+// This kernel runs every valid shape in bf16 or fp32 and is the fp32 path of the library.
+// A CTA owns TM rows x TN columns that lie inside one N-block nb. Per K-chunk kc and per
+// group of up to 32 slots it
+//   1. sketches   Xs[m][s] = sum_j sign_j * X[m, kc*BK + k_j]   (fp32, in shared memory)
+//   2. stages     Wt[s][n] = Wc[n, kc*S + s]                     (fp32, transposed)
+//   3. multiplies acc[m][n] += Xs[m][s] * Wt[s][n]                (fp32 FMA, 16x16 threads)
+// and finally rounds once to the output type. Sketch sums and the GEMM are both fp32, so
+// for fp32 data the only roundings are those of fp32 arithmetic.
+#include "ss1_internal.cuh"
+
+#include <cuda_bf16.h>
+
+namespace ss1 {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kSlotGroup = 32;
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void from_f32(float& d, float v) { d = v; }
+__device__ __forceinline__ void from_f32(__nv_bfloat16& d, float v) { d = __float2bfloat16_rn(v); }
+
+template <typename T, int TM, int TN>
+__global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X, const T* __restrict__ Wc,
+                                                        T* __restrict__ Y, const uint16_t* __restrict__ src,
+                                                        int M, int K, int N, int c, int BK, int BN, int S) {
+    constexpr int RM = TM / 16, RN = TN / 16;
+    __shared__ float Xs[TM][kSlotGroup + 1];
+    __shared__ float Wt[kSlotGroup][TN];
+
+    const int n0 = blockIdx.x * TN;
+    const int nb = n0 / BN;
+    const int m0 = blockIdx.y * TM;
+    const int KC = K / BK;
+    const int Kc = K / c;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+
+    float acc[RM][RN];
+#pragma unroll
+    for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
+
+    for (int kc = 0; kc < KC; ++kc) {
+        const uint16_t* sblk = src + ((size_t)nb * KC + kc) * (size_t)S * c;
+        for (int s0 = 0; s0 < S; s0 += kSlotGroup) {
+            const int sc = min(kSlotGroup, S - s0);
+            for (int i = threadIdx.x; i < TM * kSlotGroup; i += kThreads) {
+                const int m = i / kSlotGroup, s = i % kSlotGroup;
+                float v = 0.f;
+                if (s < sc && m0 + m < M) {
+                    const T* xr = X + (size_t)(m0 + m) * K + (size_t)kc * BK;
+                    const uint16_t* e = sblk + (size_t)(s0 + s) * c;
+                    for (int j = 0; j < c; ++j) {
+                        const uint16_t t = e[j];
+                        const float x = to_f32(xr[t & kSrcIdxMask]);
+                        v += (t & kSrcNegBit) ? -x : x;
+                    }
+                }
+                Xs[m][s] = v;
+            }
+            for (int i = threadIdx.x; i < TN * kSlotGroup; i += kThreads) {
+                const int n = i / kSlotGroup, s = i % kSlotGroup;
+                Wt[s][n] = (s < sc) ? to_f32(Wc[(size_t)(n0 + n) * Kc + (size_t)kc * S + s0 + s]) : 0.f;
+            }
+            __syncthreads();
+            for (int s = 0; s < sc; ++s) {
+                float a[RM], b[RN];
+#pragma unroll
+                for (int i = 0; i < RM; ++i) a[i] = Xs[ty + 16 * i][s];
+#pragma unroll
+                for (int j = 0; j < RN; ++j) b[j] = Wt[s][tx + 16 * j];
+#pragma unroll
+                for (int i = 0; i < RM; ++i)
+#pragma unroll
+                    for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+            }
+            __syncthreads();
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < RM; ++i) {
+        const int m = m0 + ty + 16 * i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int j = 0; j < RN; ++j) from_f32(Y[(size_t)m * N + n0 + tx + 16 * j], acc[i][j]);
+    }
+}
+
+template <typename T, int TM, int TN>
+cudaError_t launch_t(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    dim3 grid((unsigned)(L.N / TN), (unsigned)((M + TM - 1) / TM));
+    simt_kernel<T, TM, TN><<<grid, kThreads, 0, st>>>((const T*)X, (const T*)Wc, (T*)Y, L.d_src, (int)M, (int)L.K,
+                                                      (int)L.N, L.c, L.BK, L.BN, L.S);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dtype(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    // TN must divide BN (BN is a multiple of 16). Small M: narrow tiles for more CTAs.
+    if (M <= 16) return launch_t<T, 16, 16>(L, X, Wc, Y, M, st);
+    if (L.BN % 64 == 0) return launch_t<T, 64, 64>(L, X, Wc, Y, M, st);
+    if (L.BN % 32 == 0) return launch_t<T, 64, 32>(L, X, Wc, Y, M, st);
+    return launch_t<T, 64, 16>(L, X, Wc, Y, M, st);
+}
+
+}  // namespace
+
+cudaError_t launch_simt(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
+                        cudaStream_t st) {
+    if (dtype == SS1_DTYPE_FP32) return launch_dtype<float>(L, X, Wc, Y, M, st);
+    return launch_dtype<__nv_bfloat16>(L, X, Wc, Y, M, st);
+}
+
+}  // namespace ss1

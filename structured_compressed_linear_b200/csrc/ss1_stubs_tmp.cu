@@ -1,0 +1,13 @@
+// Placeholders until the tensor-core and decode kernels land.
+#include "ss1_internal.cuh"
+
+namespace ss1 {
+bool smallm_supported(const ss1_layer&, int64_t) { return false; }
+cudaError_t launch_smallm(const ss1_layer&, const void*, const void*, void*, int64_t, cudaStream_t) {
+    return cudaErrorNotSupported;
+}
+bool tc_supported(const ss1_layer&) { return false; }
+cudaError_t launch_tc(const ss1_layer&, const void*, const void*, void*, int64_t, cudaStream_t) {
+    return cudaErrorNotSupported;
+}
+}  // namespace ss1

@@ -1,0 +1,67 @@
+"""The C-ABI library loads and exports every entry point that include/*.h declares (no GPU).
+
+Only calls that need no device are made here: ss1_strerror, and the argument / handle
+checks that return before touching CUDA.
+"""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+def _declared():
+    names = []
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        names += re.findall(r"SS1_API\s+[\w\s\*]+?\b(ss1_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from structured_compressed_linear_b200 import build
+    build.build()
+    from structured_compressed_linear_b200 import ss1
+    return ss1.load_library()
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for need in ("ss1_create", "ss1_forward", "ss1_destroy", "ss1_get_tables", "ss1_strerror"):
+        assert need in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from structured_compressed_linear_b200 import ss1
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in ss1.SYMBOLS, f"binding does not declare {name}"
+
+
+def test_strerror(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        s = lib.ss1_strerror(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.ss1_strerror(12345) == b"unknown status"
+
+
+def test_argument_checks_before_device(lib):
+    h = ctypes.c_void_p()
+    # invalid shapes are rejected before any CUDA call
+    assert lib.ss1_create(768, 768, 3, 64, 64, 0, ctypes.byref(h)) == -1      # c not in {1,2,4,8}
+    assert lib.ss1_create(768, 768, 2, 512, 64, 0, ctypes.byref(h)) == -1     # BK > 256
+    assert lib.ss1_create(770, 768, 2, 64, 64, 0, ctypes.byref(h)) == -1      # K % BK
+    assert lib.ss1_create(768, 760, 2, 64, 40, 0, ctypes.byref(h)) == -1      # BN % 16
+    assert lib.ss1_create(768, 768, 2, 64, 64, 0, None) == -1
+    assert h.value is None
+    # null / unknown handles
+    assert lib.ss1_forward(None, None, None, None, 1, 0, None) == -7
+    assert lib.ss1_destroy(None) == 0
+    bogus = ctypes.c_void_p(0x1000)
+    assert lib.ss1_get_info(bogus, None, None, None, None, None) == -7
+    assert lib.ss1_destroy(bogus) == -7

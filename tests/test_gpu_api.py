@@ -1,0 +1,108 @@
+"""Exactness properties and error conventions of the CUDA path through the C ABI."""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.gpu_common import get_ss1, to_np64
+
+pytestmark = pytest.mark.gpu
+
+SIMT, TC, SMALLM = 2, 1, 3
+BF16_KERNELS = [SIMT]
+
+
+def _layer(ss1, K=512, N=256, c=4, BK=128, BN=128, seed=3):
+    return ss1.SS1Layer(K, N, c, BK, BN, seed)
+
+
+@pytest.mark.parametrize("kernel", BF16_KERNELS)
+@pytest.mark.parametrize("c,BK", [(1, 128), (2, 128), (4, 128), (8, 256), (2, 256)])
+def test_one_hot_probe_bit_exact(kernel, c, BK):
+    """X = I_K: every output is one product g * Wc (exact in bf16), so Y must equal the tied
+    weight bit for bit. Pins the hash indexing and signs inside the kernel."""
+    ss1 = get_ss1()
+    K, N, BN = 512, 256, 128
+    layer = _layer(ss1, K, N, c, BK, BN, seed=11)
+    gen = torch.Generator().manual_seed(5)
+    Wc = (torch.randn(N, K // c, generator=gen) * 0.1).to(torch.bfloat16)
+    X = torch.eye(K, dtype=torch.bfloat16)
+    Y = layer.forward(X.cuda(), Wc.cuda(), kernel=kernel)
+    h, g = O.ss1_tables(K, N, c, BK, BN, 11)
+    Wfull = np.concatenate([O.expand_weight(to_np64(Wc), h, g, BN, nb) for nb in range(N // BN)])
+    assert np.array_equal(to_np64(Y), Wfull.T)
+    layer.close()
+
+
+@pytest.mark.parametrize("kernel", BF16_KERNELS)
+def test_zero_negation_linearity(kernel):
+    ss1 = get_ss1()
+    layer = _layer(ss1)
+    gen = torch.Generator().manual_seed(9)
+    X1 = torch.randn(300, 512, generator=gen).to(torch.bfloat16).cuda()
+    X2 = torch.randn(300, 512, generator=gen).to(torch.bfloat16).cuda()
+    Wc = (torch.randn(256, 128, generator=gen) * 0.05).to(torch.bfloat16).cuda()
+    Y0 = layer.forward(torch.zeros_like(X1), Wc, kernel=kernel)
+    assert torch.count_nonzero(Y0).item() == 0
+    Yp = layer.forward(X1, Wc, kernel=kernel)
+    Yn = layer.forward(-X1, Wc, kernel=kernel)
+    assert torch.equal(Yn, -Yp)
+    Ys = layer.forward((X1.float() + X2.float()).to(torch.bfloat16), Wc, kernel=kernel)
+    Y2 = layer.forward(X2, Wc, kernel=kernel)
+    ref = Yp.float() + Y2.float()
+    scale = ref.abs().amax(dim=1, keepdim=True)
+    assert float(((Ys.float() - ref).abs() / scale).max()) < 3e-2
+    layer.close()
+
+
+def test_guard_band_and_zero_rows():
+    """Rows of the output buffer past M stay untouched; M = 0 is a no-op."""
+    ss1 = get_ss1()
+    layer = _layer(ss1)
+    lib = ss1.lib()
+    gen = torch.Generator().manual_seed(1)
+    M = 129
+    X = torch.randn(M, 512, generator=gen).to(torch.bfloat16).cuda()
+    Wc = (torch.randn(256, 128, generator=gen) * 0.05).to(torch.bfloat16).cuda()
+    buf = torch.full((M + 7, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    for k in [0] + BF16_KERNELS:
+        st = torch.cuda.current_stream().cuda_stream
+        assert lib.ss1_forward_with(layer.handle, X.data_ptr(), Wc.data_ptr(), buf.data_ptr(), M, 0, k, st) == 0
+        torch.cuda.synchronize()
+        assert torch.all(buf[M:] == 7.0)
+        assert lib.ss1_forward_with(layer.handle, X.data_ptr(), Wc.data_ptr(), buf.data_ptr(), 0, 0, k, st) == 0
+    layer.close()
+
+
+def test_error_conventions():
+    ss1 = get_ss1()
+    lib = ss1.lib()
+    layer = _layer(ss1)
+    X = torch.zeros(8, 512, dtype=torch.bfloat16, device="cuda")
+    Wc = torch.zeros(256, 128, dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros(8, 256, dtype=torch.bfloat16, device="cuda")
+    h = layer.handle
+    st = torch.cuda.current_stream().cuda_stream
+    assert lib.ss1_forward(h, X.data_ptr() + 2, Wc.data_ptr(), Y.data_ptr(), 4, 0, st) == -5
+    assert lib.ss1_forward(h, None, Wc.data_ptr(), Y.data_ptr(), 4, 0, st) == -1
+    assert lib.ss1_forward(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), -1, 0, st) == -1
+    assert lib.ss1_forward(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 7, st) == -1
+    assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 0, 99, st) == -1
+    # fp32 data cannot take the tensor-core path
+    assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 1, TC, st) == -8
+    k = ctypes.c_int()
+    assert lib.ss1_select_kernel(h, 4096, 1, ctypes.byref(k)) == 0 and k.value == SIMT
+    K_, N_ = ctypes.c_int64(), ctypes.c_int64()
+    c_, bk, bn = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.ss1_get_info(h, ctypes.byref(K_), ctypes.byref(N_), ctypes.byref(c_), ctypes.byref(bk),
+                            ctypes.byref(bn)) == 0
+    assert (K_.value, N_.value, c_.value, bk.value, bn.value) == (512, 256, 4, 128, 128)
+    assert layer.device_status() == (0, 0)
+    raw = layer._h
+    layer.close()
+    assert lib.ss1_forward(raw, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 0, st) == -7
+    assert lib.ss1_destroy(raw) == -7
+    torch.cuda.synchronize()

@@ -1,0 +1,62 @@
+"""CUDA path vs CPU oracle, element by element.
+
+Small cases (whole output compared) span several tiles in M and N plus ragged M tails, for
+every kernel that supports them. The workloads run at full size in the launch the
+benchmark times (automatic kernel choice); there the oracle computes sampled rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from structured_compressed_linear_b200.workloads import WORKLOADS, Layer, make_inputs
+from tests.gpu_common import check_layer, get_ss1, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+SIMT, TC, SMALLM = 2, 1, 3
+
+
+def _small_cases():
+    cases = []
+    # fp32: the single-layer workload and ragged variants
+    for M in (1, 3, 64, 65, 130):
+        cases.append(Layer("fp32-small", M, 768, 768, 2, 64, 64, "fp32", "normal", "uniform_invsqrtk", 0))
+    cases.append(Layer("fp32-small", 77, 512, 256, 4, 128, 128, "fp32", "normal", "uniform_invsqrtk", 5))
+    cases.append(Layer("fp32-small", 33, 256, 192, 1, 64, 64, "fp32", "normal", "uniform_invsqrtk", 5))
+    # bf16: every c, both BK of the workloads, ragged M, several N-blocks
+    for c in (1, 2, 4, 8):
+        for BK in (128, 256):
+            for M in (1, 16, 200, 333):
+                cases.append(Layer("bf16-small", M, 1024, 384, c, BK, 128, "bf16", "normal", "normal_002", 3))
+    cases.append(Layer("bf16-small", 257, 1280, 640, 4, 128, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2))
+    return cases
+
+
+def _kernels_for(L: Layer):
+    ks = [SIMT]
+    return ks
+
+
+SMALL = [(L, k) for L in _small_cases() for k in _kernels_for(L)]
+
+
+@pytest.mark.parametrize("L,kernel", SMALL, ids=[f"{L.tag}:{L.BK}:{L.dtype}:k{k}" for L, k in SMALL])
+def test_small_parity(L, kernel):
+    ss1 = get_ss1()
+    check_layer(ss1, L, kernel=kernel)
+
+
+FULL = [L for wid in sorted(WORKLOADS) for L in WORKLOADS[wid]]
+
+
+@pytest.mark.parametrize("L", FULL, ids=[L.tag for L in FULL])
+def test_workload_parity_sampled(L):
+    """Full-size layers, automatic kernel choice, oracle on sampled rows (all outliers too)."""
+    ss1 = get_ss1()
+    X, Wc = make_inputs(L)
+    must = []
+    if L.x_dist == "normal_outliers":
+        must = torch.nonzero(X.float().abs().amax(dim=1) > 8.0).flatten().tolist()[:64]
+    rows = sample_rows(L.M, 48, seed=L.M + L.K, must=must)
+    check_layer(ss1, L, kernel=0, rows=rows, X=X, Wc=Wc)
