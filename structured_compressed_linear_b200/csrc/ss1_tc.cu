@@ -1,0 +1,386 @@
+// Tensor-core SS1 forward for sm_100a: TMA -> on-chip sketch -> tcgen05.mma (TMEM accumulator).
+//
+// "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+// "Approach": the input is sketched (signed hashed additions shrink it by the compression
+// factor c) and then multiplied with the compressed weights; after the sketch the work is a
+// dense contraction, so it runs on the 5th-generation tensor cores.
+//
+// One CTA computes a 128-row x 128-column output tile = rows [m0, m0+128) of N-block nb
+// (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs, S = BK / c compressed columns):
+//   * TMA warp      : X[m0:+128, kc*BK:+BK] -> smem (128B-swizzled, 64-column panels) and
+//                     Wc[nb*128:+128, kc*S:+S] -> smem (K-major, swizzle chosen by S).
+//   * sketch warps  : thread = row; Xs[row, s] = sum_j sign_j * X[row, kc*BK + k_j] in fp32,
+//                     rounded once to bf16 and written as the UMMA A operand (K-major,
+//                     same swizzle as the Wc tile). The sketch never leaves shared memory.
+//   * MMA thread    : S/16 x tcgen05.mma.kind::f16 (M=128, N=128, K=16) into one TMEM
+//                     accumulator; tcgen05.commit releases the stage.
+//   * epilogue      : the sketch warps read the fp32 accumulator with tcgen05.ld, round to
+//                     bf16 and store Y.
+// c = 1 skips the sketch: the X tile is the A operand (a plain GEMM, identity hash).
+// Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
+// handle's status word, drains the copies and MMAs in flight and returns (no trap).
+#include "ss1_internal.cuh"
+#include "ptx_sm100.cuh"
+
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace ss1 {
+namespace {
+
+constexpr int kBM = 128;         // rows per tile (UMMA M)
+constexpr int kBN = 128;         // N-block size handled (UMMA N)
+constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 sketch + epilogue
+constexpr int kSmemBudget = 200 * 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+template <int BK, int C>
+struct Cfg {
+    static constexpr int S = BK / C;
+    static constexpr int X_BYTES = kBM * BK * 2;
+    static constexpr int W_BYTES = kBN * S * 2;
+    static constexpr int A_BYTES = (C == 1) ? 0 : kBM * S * 2;
+    static constexpr int RB = S >= 64 ? 128 : 2 * S;   // bytes per row inside one swizzle panel
+    static constexpr int PANEL = 128 * RB;              // bytes of one 128-row panel
+    static constexpr uint32_t LAYOUT = S >= 64 ? ptx::kLayoutSW128 : (S == 32 ? ptx::kLayoutSW64 : ptx::kLayoutSW32);
+    static constexpr int SBO = 8 * RB;                  // byte distance of consecutive 8-row groups
+
+    static constexpr int stage_pick(bool want_x) {
+        int best_x = 1, best_w = 1, best_score = -1;
+        for (int nx = 1; nx <= 4; ++nx)
+            for (int nw = 1; nw <= 4; ++nw) {
+                const int bytes = nx * X_BYTES + nw * (W_BYTES + A_BYTES);
+                if (bytes > kSmemBudget) continue;
+                const int score = (nx < nw ? nx : nw) * 16 + nx + nw;
+                if (score > best_score) { best_score = score; best_x = nx; best_w = nw; }
+            }
+        return want_x ? best_x : best_w;
+    }
+    static constexpr int NX = stage_pick(true);
+    static constexpr int NW = stage_pick(false);
+    static constexpr int NBAR = 2 * NX + 3 * NW + 1;
+    static constexpr int SMEM = NX * X_BYTES + NW * (W_BYTES + A_BYTES) + NBAR * 8 + 16 + 1024;
+    static_assert(S % 16 == 0 && S >= 16, "UMMA K-steps of 16");
+    static_assert(BK % 64 == 0, "X panels of 64 columns");
+};
+
+__device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
+    *abort_flag = 1;
+    *(volatile int32_t*)status = (kStatusKernelTC << 8) | site;
+    __threadfence_system();
+}
+
+// Byte offset of element (row, col) in a K-major tile of `cols` columns stored as 128-row
+// panels of RB bytes per row with the matching TMA / UMMA swizzle.
+template <int RB>
+__device__ __forceinline__ uint32_t kmajor_offset(int row, int col) {
+    constexpr int per_panel = RB / 2;
+    const int p = col / per_panel;
+    const int cin = col % per_panel;
+    const uint32_t chunk = (uint32_t)(cin >> 3) ^ (uint32_t)(((row * RB) >> 7) & (RB / 16 - 1));
+    return (uint32_t)(p * 128 * RB + row * RB) + (chunk << 4) + (uint32_t)(cin & 7) * 2u;
+}
+
+template <int BK, int C>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+              __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src, int M, int N, int KC,
+              int32_t* status) {
+    using F = Cfg<BK, C>;
+    constexpr int S = F::S, NX = F::NX, NW = F::NW;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* xs = smem;
+    uint8_t* ws = xs + NX * F::X_BYTES;
+    uint8_t* as = ws + NW * F::W_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(as + NW * F::A_BYTES);
+    uint64_t* x_full = bars;
+    uint64_t* x_empty = x_full + NX;
+    uint64_t* w_full = x_empty + NX;
+    uint64_t* a_full = w_full + NW;
+    uint64_t* aw_empty = a_full + NW;
+    uint64_t* acc_full = aw_empty + NW;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nb = blockIdx.x;
+    const int m0 = blockIdx.y * kBM;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NX; ++i) {
+            ptx::mbar_init(&x_full[i], 1);
+            ptx::mbar_init(&x_empty[i], C == 1 ? 1 : 128);
+        }
+        for (int i = 0; i < NW; ++i) {
+            ptx::mbar_init(&w_full[i], 1);
+            ptx::mbar_init(&a_full[i], 128);
+            ptx::mbar_init(&aw_empty[i], 1);
+        }
+        ptx::mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, kBN);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap_w);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_acc = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int last_x = -1, last_w = -1;
+            for (int kc = 0; kc < KC; ++kc) {
+                const int xi = kc % NX, wi = kc % NW;
+                if (!ptx::mbar_wait(&x_empty[xi], ((kc / NX) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 1);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&x_full[xi], F::X_BYTES);
+#pragma unroll
+                for (int p = 0; p < BK / 64; ++p)
+                    ptx::tma_load_2d(xs + xi * F::X_BYTES + p * 128 * 128, &tmap_x, &x_full[xi], kc * BK + p * 64, m0);
+                last_x = kc;
+                if (!ptx::mbar_wait(&aw_empty[wi], ((kc / NW) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 2);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&w_full[wi], F::W_BYTES);
+#pragma unroll
+                for (int p = 0; p < (S + 63) / 64; ++p)
+                    ptx::tma_load_2d(ws + wi * F::W_BYTES + p * F::PANEL, &tmap_w, &w_full[wi], kc * S + p * 64,
+                                     nb * kBN);
+                last_w = kc;
+            }
+            if (*abort_flag) {
+                // drain: every issued copy must land before the CTA may exit
+                volatile int no_abort = 0;
+                for (int kc = (last_x - NX + 1 > 0 ? last_x - NX + 1 : 0); kc <= last_x; ++kc)
+                    ptx::mbar_wait(&x_full[kc % NX], (kc / NX) & 1, &no_abort, kWaitLimitNs);
+                for (int kc = (last_w - NW + 1 > 0 ? last_w - NW + 1 : 0); kc <= last_w; ++kc)
+                    ptx::mbar_wait(&w_full[kc % NW], (kc / NW) & 1, &no_abort, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
+            for (int kc = 0; kc < KC; ++kc) {
+                const int wi = kc % NW;
+                const uint32_t ph = (kc / NW) & 1;
+                if (!ptx::mbar_wait(&w_full[wi], ph, abort_flag, kWaitLimitNs)) { report(status, abort_flag, 3); break; }
+                const uint8_t* a_tile;
+                if constexpr (C == 1) {
+                    if (!ptx::mbar_wait(&x_full[kc % NX], (kc / NX) & 1, abort_flag, kWaitLimitNs)) {
+                        report(status, abort_flag, 4);
+                        break;
+                    }
+                    a_tile = xs + (kc % NX) * F::X_BYTES;
+                } else {
+                    if (!ptx::mbar_wait(&a_full[wi], ph, abort_flag, kWaitLimitNs)) { report(status, abort_flag, 4); break; }
+                    a_tile = as + wi * F::A_BYTES;
+                }
+                ptx::tc_fence_after();
+                const uint32_t a_base = ptx::smem_u32(a_tile);
+                const uint32_t b_base = ptx::smem_u32(ws + wi * F::W_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < S / 16; ++kk) {
+                    constexpr int per_panel = F::RB / 2;
+                    const uint32_t off = (uint32_t)((kk * 16) / per_panel) * F::PANEL + (uint32_t)((kk * 16) % per_panel) * 2u;
+                    const uint64_t ad = ptx::smem_desc(a_base + off, 16, F::SBO, F::LAYOUT);
+                    const uint64_t bd = ptx::smem_desc(b_base + off, 16, F::SBO, F::LAYOUT);
+                    ptx::umma_bf16_ss(tmem_acc, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::umma_commit(&aw_empty[wi]);
+                if constexpr (C == 1) ptx::umma_commit(&x_empty[kc % NX]);
+            }
+            ptx::umma_commit(acc_full);
+            if (*abort_flag) {
+                volatile int no_abort = 0;
+                ptx::mbar_wait(acc_full, 0, &no_abort, kWaitLimitNs);  // MMAs in flight finish before exit
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ sketch + epilogue
+        const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
+        const int row = quad * 32 + lane;       // row of the tile owned by this thread
+        if constexpr (C > 1) {
+            for (int kc = 0; kc < KC; ++kc) {
+                const int xi = kc % NX, wi = kc % NW;
+                if (!ptx::mbar_wait(&x_full[xi], (kc / NX) & 1, abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 5);
+                    break;
+                }
+                if (!ptx::mbar_wait(&aw_empty[wi], ((kc / NW) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 6);
+                    break;
+                }
+                const uint8_t* xt = xs + xi * F::X_BYTES;
+                uint8_t* at = as + wi * F::A_BYTES;
+                const uint4* tab = reinterpret_cast<const uint4*>(src + ((size_t)nb * KC + kc) * (size_t)(S * C));
+#pragma unroll 1
+                for (int s8 = 0; s8 < S / 8; ++s8) {
+                    uint4 e[C];
+#pragma unroll
+                    for (int j = 0; j < C; ++j) e[j] = __ldg(tab + s8 * C + j);
+                    const uint16_t* ent = reinterpret_cast<const uint16_t*>(e);
+                    float v[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < C; ++j) {
+                            const uint16_t en = ent[t * C + j];
+                            const int k = en & kSrcIdxMask;
+                            const uint32_t off = (uint32_t)((k >> 6) * 128 * 128) + kmajor_offset<128>(row, k & 63);
+                            const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(xt + off));
+                            acc += (en & kSrcNegBit) ? -x : x;
+                        }
+                        v[t] = acc;
+                    }
+                    uint4 packed;
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]);
+                    __nv_bfloat162 p1 = __floats2bfloat162_rn(v[2], v[3]);
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(v[4], v[5]);
+                    __nv_bfloat162 p3 = __floats2bfloat162_rn(v[6], v[7]);
+                    packed.x = *reinterpret_cast<uint32_t*>(&p0);
+                    packed.y = *reinterpret_cast<uint32_t*>(&p1);
+                    packed.z = *reinterpret_cast<uint32_t*>(&p2);
+                    packed.w = *reinterpret_cast<uint32_t*>(&p3);
+                    *reinterpret_cast<uint4*>(at + kmajor_offset<F::RB>(row, s8 * 8)) = packed;
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&x_empty[xi]);
+                ptx::mbar_arrive(&a_full[wi]);
+            }
+        }
+        // epilogue
+        bool ok = ptx::mbar_wait(acc_full, 0, abort_flag, kWaitLimitNs);
+        if (!ok) report(status, abort_flag, 7);
+        ptx::tc_fence_after();
+        ok = __all_sync(0xffffffffu, ok && !*abort_flag);   // tcgen05.ld is warp-collective
+        if (ok) {
+            const int m = m0 + row;
+            __nv_bfloat16* yrow = Y + (size_t)m * N + (size_t)nb * kBN;
+#pragma unroll 1
+            for (int col0 = 0; col0 < kBN; col0 += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld_32x32b_x32(tmem_acc + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0, r);
+                ptx::tmem_ld_wait();
+                if (m < M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 o;
+                        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[q * 8 + 2 * t]),
+                                                                     __uint_as_float(r[q * 8 + 2 * t + 1]));
+                            ow[t] = *reinterpret_cast<uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
+                    }
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_acc, kBN);
+    }
+}
+
+// ---------------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                 uint32_t box_outer, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BK, int C>
+cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    using F = Cfg<BK, C>;
+    constexpr int S = F::S;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(tc_kernel<BK, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mx, mw;
+    const CUtensorMapSwizzle wsw = S >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (S == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    if (!make_map_2d(&mx, X, (uint64_t)L.K, (uint64_t)M, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kBN, wsw))
+        return cudaErrorInvalidValue;
+    dim3 grid((unsigned)L.NB, (unsigned)((M + kBM - 1) / kBM));
+    tc_kernel<BK, C><<<grid, kThreads, F::SMEM, st>>>(mx, mw, (__nv_bfloat16*)Y, L.d_src, (int)M, (int)L.N, L.KC,
+                                                      L.status_dev);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const ss1_layer& L) {
+    if (L.BN != kBN) return false;
+    if (!(L.BK == 64 || L.BK == 128 || L.BK == 256)) return false;
+    if (L.S < 16 || L.S % 16 != 0) return false;
+    if (L.K % 8 != 0 || (L.K / L.c) % 8 != 0) return false;
+    return true;
+}
+
+cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if ((M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
+#define SS1_TC_CASE(bk, cc) \
+    if (L.BK == bk && L.c == cc) return launch_cfg<bk, cc>(L, X, Wc, Y, M, st);
+    SS1_TC_CASE(64, 1)
+    SS1_TC_CASE(64, 2)
+    SS1_TC_CASE(64, 4)
+    SS1_TC_CASE(128, 1)
+    SS1_TC_CASE(128, 2)
+    SS1_TC_CASE(128, 4)
+    SS1_TC_CASE(128, 8)
+    SS1_TC_CASE(256, 1)
+    SS1_TC_CASE(256, 2)
+    SS1_TC_CASE(256, 4)
+    SS1_TC_CASE(256, 8)
+#undef SS1_TC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ss1

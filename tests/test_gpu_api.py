@@ -12,7 +12,7 @@ from tests.gpu_common import get_ss1, to_np64
 pytestmark = pytest.mark.gpu
 
 SIMT, TC, SMALLM = 2, 1, 3
-BF16_KERNELS = [SIMT]
+BF16_KERNELS = [SIMT, TC]
 
 
 def _layer(ss1, K=512, N=256, c=4, BK=128, BN=128, seed=3):

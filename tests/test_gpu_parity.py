@@ -33,8 +33,17 @@ def _small_cases():
     return cases
 
 
+def tc_eligible(L: Layer) -> bool:
+    """Documented preconditions of the tensor-core kernel (include/ss1.h)."""
+    S = L.BK // L.c
+    return (L.dtype == "bf16" and L.BN == 128 and L.BK in (64, 128, 256) and S % 16 == 0 and S >= 16
+            and L.K % 8 == 0 and (L.K // L.c) % 8 == 0)
+
+
 def _kernels_for(L: Layer):
     ks = [SIMT]
+    if tc_eligible(L):
+        ks.append(TC)
     return ks
 
 
