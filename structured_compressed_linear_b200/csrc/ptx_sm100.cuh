@@ -149,6 +149,49 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Warp-collective: one 32-bit column of 32 lanes (lane = thread) at a run-time column.
+__device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return r;
+}
+
+// Warp-collective: 16 lanes x 256 bits. Thread t receives (lane t/4, col 2(t%4)), (lane t/4,
+// col 2(t%4)+1), (lane t/4+8, col 2(t%4)), (lane t/4+8, col 2(t%4)+1) -- the mma C-fragment layout.
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                uint32_t& r3) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(taddr));
+}
+
+// Copies a 128-row x 256-bit block described by a shared-memory matrix descriptor into TMEM
+// (row r -> lane r, 8 consecutive 32-bit columns); issued by one thread, tracked by umma_commit.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// ------------------------------------------------------------------------------ misc
+
+// Four 8x8 b16 matrices stored transposed; thread 8i+j gives the address of stored row j of matrix i.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a0),
+                 "r"(a1), "r"(a2), "r"(a3)
+                 : "memory");
+}
+
+// 1-D bulk copy global -> shared, completion counted in bytes on `bar` (addresses and size 16B-aligned).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ------------------------------------------------------------------------------ descriptors
 
 // Swizzle modes of K-major canonical layouts, as encoded in the tcgen05 smem descriptor.

@@ -26,6 +26,7 @@ void release(ss1_layer* L) {
     if (L->d_h) cudaFree(L->d_h);
     if (L->d_g) cudaFree(L->d_g);
     if (L->d_src) cudaFree(L->d_src);
+    if (L->d_gather) cudaFree(L->d_gather);
     if (L->status_host) cudaFreeHost(L->status_host);
     L->magic = 0;
     delete L;
@@ -83,6 +84,7 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
     if (cudaMalloc(&L->d_h, entries * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&L->d_g, entries * sizeof(int8_t)) != cudaSuccess ||
         cudaMalloc(&L->d_src, entries * sizeof(uint16_t)) != cudaSuccess ||
+        cudaMalloc(&L->d_gather, entries * 2 * sizeof(uint32_t)) != cudaSuccess ||
         cudaHostAlloc(&L->status_host, sizeof(int32_t), cudaHostAllocMapped) != cudaSuccess) {
         cudaGetLastError();
         release(L);
@@ -94,7 +96,8 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
         release(L);
         return SS1_ERR_CUDA;
     }
-    if (ss1::launch_hashgen(*L, 0) != cudaSuccess || cudaStreamSynchronize(0) != cudaSuccess) {
+    if (ss1::launch_hashgen(*L, 0) != cudaSuccess || ss1::launch_gather_tables(*L, 0) != cudaSuccess ||
+        cudaStreamSynchronize(0) != cudaSuccess) {
         cudaGetLastError();
         release(L);
         return SS1_ERR_CUDA;

@@ -76,7 +76,29 @@ __global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int 
     }
 }
 
+// One thread per source: the tensor-core kernel gathers X[row, k] from a TMEM word that holds
+// the bf16 pair (k & ~1, k | 1); the multiplier keeps the half of k with its sign, zeroes the other.
+__global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint32_t* __restrict__ out, int BK,
+                                    int64_t nsrc) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= nsrc) return;
+    const int64_t blk = i / BK, t = i % BK;
+    const uint16_t e = src[i];
+    const uint32_t k = e & kSrcIdxMask;
+    const bool neg = (e & kSrcNegBit) != 0;
+    const uint32_t one = neg ? 0xBF80u : 0x3F80u;   // bf16 -1 / +1
+    out[blk * 2 * BK + t] = k >> 1;
+    out[blk * 2 * BK + BK + t] = (k & 1u) ? (one << 16) : one;
+}
+
 }  // namespace
+
+cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st) {
+    const int64_t nsrc = (int64_t)L.NB * L.K;
+    const int threads = 256;
+    gather_table_kernel<<<(unsigned)((nsrc + threads - 1) / threads), threads, 0, st>>>(L.d_src, L.d_gather, L.BK, nsrc);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st) {
     const int nblocks = L.NB * L.KC;

@@ -24,6 +24,8 @@ struct ss1_layer {
     int32_t* d_h;        // [NB][K] compressed column of input k in block nb
     int8_t* d_g;         // [NB][K] sign of input k in block nb
     uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
+    uint32_t* d_gather;  // [NB][KC][2][BK] per source (slot-major): TMEM word column k/2, then the
+                         // bf16x2 multiplier (+-1 in the half that holds k, 0 in the other)
     int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
     int32_t* status_dev;   // device alias of status_host
 };
@@ -34,6 +36,8 @@ namespace ss1 {
 enum : int32_t { kStatusKernelTC = 1 };
 
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);
+// Derives d_gather from d_src (run after launch_hashgen).
+cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st);
 
 // General CUDA-core path: any valid shape, bf16 or fp32.
 cudaError_t launch_simt(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
@@ -46,6 +50,9 @@ cudaError_t launch_smallm(const ss1_layer& L, const void* X, const void* Wc, voi
 
 // Tensor-core path (bf16, tcgen05 + TMEM + TMA).
 bool tc_supported(const ss1_layer& L);
+// Transposed-tile variant (c >= 2): 128 neurons x 256 rows per tile, sketch gathered from TMEM.
+bool tc2_supported(const ss1_layer& L);
+cudaError_t launch_tc2(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 
 }  // namespace ss1

@@ -28,6 +28,9 @@
 #include <mutex>
 
 namespace ss1 {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 namespace {
 
 constexpr int kBM = 128;         // rows per tile (UMMA M)
@@ -305,22 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                  uint32_t box_outer, CUtensorMapSwizzle sw) {
-    auto fn = encode_fn();
+    auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {inner * 2};
@@ -356,6 +346,19 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
 bool tc_supported(const ss1_layer& L) {
     if (L.BN != kBN) return false;
     if (!(L.BK == 64 || L.BK == 128 || L.BK == 256)) return false;
@@ -365,6 +368,7 @@ bool tc_supported(const ss1_layer& L) {
 }
 
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if (tc2_supported(L)) return launch_tc2(L, X, Wc, Y, M, st);
     if ((M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
 #define SS1_TC_CASE(bk, cc) \
     if (L.BK == bk && L.c == cc) return launch_cfg<bk, cc>(L, X, Wc, Y, M, st);
