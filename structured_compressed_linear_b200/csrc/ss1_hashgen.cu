@@ -76,19 +76,14 @@ __global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int 
     }
 }
 
-// One thread per source: the tensor-core kernel gathers X[row, k] from a TMEM word that holds
-// the bf16 pair (k & ~1, k | 1); the multiplier keeps the half of k with its sign, zeroes the other.
-__global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint32_t* __restrict__ out, int BK,
-                                    int64_t nsrc) {
+// One thread per source: the tensor-core kernel reads X[row, k] and X[row + 128, k] as one
+// bf16x2 TMEM word at column k; the entry is k (bits 0..8) with the sign copied into bits 15
+// and 31, so (entry & 0x80008000) | bf16x2(1, 1) is the +-1 multiplier of both halves.
+__global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint32_t* __restrict__ out, int64_t nsrc) {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= nsrc) return;
-    const int64_t blk = i / BK, t = i % BK;
     const uint16_t e = src[i];
-    const uint32_t k = e & kSrcIdxMask;
-    const bool neg = (e & kSrcNegBit) != 0;
-    const uint32_t one = neg ? 0xBF80u : 0x3F80u;   // bf16 -1 / +1
-    out[blk * 2 * BK + t] = k >> 1;
-    out[blk * 2 * BK + BK + t] = (k & 1u) ? (one << 16) : one;
+    out[i] = (uint32_t)(e & kSrcIdxMask) | ((e & kSrcNegBit) ? 0x80008000u : 0u);
 }
 
 }  // namespace
@@ -96,7 +91,7 @@ __global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint32_t* 
 cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st) {
     const int64_t nsrc = (int64_t)L.NB * L.K;
     const int threads = 256;
-    gather_table_kernel<<<(unsigned)((nsrc + threads - 1) / threads), threads, 0, st>>>(L.d_src, L.d_gather, L.BK, nsrc);
+    gather_table_kernel<<<(unsigned)((nsrc + threads - 1) / threads), threads, 0, st>>>(L.d_src, L.d_gather, nsrc);
     return cudaGetLastError();
 }
 

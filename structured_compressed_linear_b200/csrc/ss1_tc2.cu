@@ -4,23 +4,24 @@
 // "Approach": the input is sketched by signed hashed additions and the sketch is multiplied
 // with the compressed weights. This kernel keeps the sketch on chip and feeds it to tcgen05.
 //
-// Tile: 128 neurons (one N-block, UMMA M = 128) x 256 rows of X (UMMA N = 256). One UMMA N of
-// 256 is what lets the tensor pipe run near its peak; the operands of one instruction must
-// share one hash, and the rows of X do, the neurons of two blocks do not.
-// Per K-chunk kc:
+// Tile: 128 neurons (one N-block, UMMA M = 128) x 256 rows of X (UMMA N = 256). An UMMA N of
+// 256 is what lets the tensor pipe run near its peak, and the operands of one instruction must
+// share one hash: rows of X do, neurons of two blocks do not. Persistent CTAs (one per SM)
+// walk the tiles with the N-block index fastest, so CTAs running side by side share X in L2.
+// Per K-chunk kc of a tile:
 //   * TMA warp   : X rows [m0, m0+256) x chunk -> 16 KB smem panels [128 rows x 64 k] (128B
-//                  swizzle); Wc[nb*128:+128, kc*S:+S] -> K-major panels; the chunk's gather
-//                  table (TMEM column and bf16x2 multiplier per source) -> smem (bulk copy).
-//   * MMA thread : tcgen05.cp copies every X panel into TMEM (row r -> lane r % 128, one
-//                  32-bit column per pair of inputs), two TMEM buffers per row half when they
-//                  fit; then issues S/16 tcgen05.mma (M=128, N=256, K=16) per chunk.
-//   * 8 sketch warps (thread = row of the tile): for slot s, Xs[row, s] = sum_j sign_j *
-//                  X[row, k_j], gathered with tcgen05.ld from TMEM and accumulated with bf16x2
-//                  FMAs whose multiplier keeps the half of the word that holds k_j; the two
-//                  halves are folded, rounded once per add, and written as the K-major UMMA B
-//                  operand in shared memory. No shared-memory bank is touched for the gather.
-//   * epilogue   : tcgen05.ld.16x256b (mma fragment layout) -> bf16 -> stmatrix.trans into a
-//                  128B-swizzled [rows x neurons] staging tile -> TMA store of Y.
+//                  swizzle), both row halves of one 64-input panel back to back; Wc[nb*128:+128,
+//                  kc*S:+S] -> K-major panels; the chunk's gather table -> smem (bulk copy).
+//   * 16 sketch warps. A thread owns rows r and r+128 of the tile (r = TMEM lane). They first
+//                  stage the X chunk into TMEM as row pairs: conflict-free 16-byte shared loads,
+//                  byte permutes to (X[r][k], X[r+128][k]), tcgen05.st -> column k. Then, for
+//                  their quarter of the slots, Xs[., s] = sum_j sign_j * X[., k_j] with one
+//                  tcgen05.ld (two rows at once) and one bf16x2 FMA per source, and write both
+//                  rows as the K-major UMMA B operand. The gather touches no shared-memory bank.
+//   * MMA warp   : S/16 x tcgen05.mma (M=128, N=256, K=16) per chunk into one accumulator.
+//   * 4 epilogue warps: tcgen05.ld.16x256b (mma fragment layout) -> bf16 -> stmatrix.trans into
+//                  a 128B-swizzled [128 rows x 128 neurons] staging tile -> TMA store of Y;
+//                  they release the accumulator as soon as its last column is read.
 // Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
 // handle's status word, drains the copies and MMAs in flight and returns (no trap).
 #include "ss1_internal.cuh"
@@ -33,18 +34,23 @@
 
 namespace ss1 {
 
-// shared with ss1_tc.cu (tensor-map encoding through the driver entry point)
+// defined in ss1_tc.cu (tensor-map encoding through the driver entry point)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 namespace {
 
 constexpr int kNeu = 128;        // neurons per tile (UMMA M) = the N-block
 constexpr int kRows = 256;       // rows of X per tile (UMMA N)
-constexpr int kWarps = 10;       // warp 0 TMA, warp 1 copy+MMA, warps 2..9 sketch (2..5 also epilogue)
+constexpr int kSketchWarps = 16;
+constexpr int kEpiWarps = 4;
+constexpr int kFirstSketch = 3;                         // warp 0 X loads, warp 1 Wc loads, warp 2 MMA
+constexpr int kFirstEpi = kFirstSketch + kSketchWarps;  // warps 19..22
+constexpr int kWarps = kFirstEpi + kEpiWarps;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSketchWarps = 8;
-constexpr int kXPanel = 128 * 128;   // bytes of one [128 rows x 64 inputs] bf16 panel
-constexpr uint32_t kAccCols = 256;   // TMEM columns of the accumulator
+constexpr int kXSlot = kRows * 128;    // bytes of one [256 rows x 64 inputs] bf16 TMA box
+constexpr int kEpiStage = 32 * 32 * 2; // per epilogue warp: [32 rows x 32 neurons] bf16
+constexpr uint32_t kAccCols = 256;     // TMEM columns of the accumulator
+constexpr int kBatch = 16;             // sources per gather batch (TMEM loads in flight per wait)
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 template <int BK, int C>
@@ -52,30 +58,30 @@ struct Cfg {
     static constexpr int S = BK / C;
     static constexpr int SP = S < 64 ? S : 64;          // slots per panel (one swizzle row)
     static constexpr int NSP = S / SP;                  // slot panels per chunk
+    static constexpr int SB = kBatch / C;               // slots per gather batch
+    static constexpr int NBATCH = SP / SB;              // batches per panel (split over 4 warps)
     static constexpr int RB = 2 * SP;                   // bytes per row of a panel
     static constexpr uint32_t LAYOUT = SP == 64 ? ptx::kLayoutSW128 : (SP == 32 ? ptx::kLayoutSW64 : ptx::kLayoutSW32);
     static constexpr int SBO = 8 * RB;
     static constexpr int W_PANEL = kNeu * RB;
     static constexpr int B_PANEL = kRows * RB;
-    static constexpr int XPH = BK / 64;                 // X panels per row half per chunk
-    static constexpr int NXB = BK <= 128 ? 2 : 1;       // TMEM X buffers
-    static constexpr int XCOLS = BK / 2;                // TMEM columns per row half per buffer
-    static constexpr int TAB = 2 * BK * 4;              // bytes of one (nb, kc) gather table
-    static constexpr int NXS = 4, NWS = 3, NBS = 2, NTS = 2;
+    static constexpr int XPH = BK / 64;                 // X boxes (64 inputs x 256 rows) per chunk
+    static constexpr int NXB = BK <= 128 ? 2 : 1;       // TMEM X buffers (BK row-pair columns each)
+    static constexpr int NXS = 3, NBS = 2, NWS = 3;
     static constexpr int OFF_X = 0;
-    static constexpr int OFF_W = OFF_X + NXS * kXPanel;
+    static constexpr int OFF_W = OFF_X + NXS * kXSlot;
     static constexpr int OFF_B = OFF_W + NWS * W_PANEL;
-    static constexpr int OFF_T = OFF_B + NBS * B_PANEL;
-    static constexpr int OFF_A = OFF_T + NTS * TAB;                 // per-warp TMEM address tables
-    static constexpr int OFF_BAR = OFF_A + kSketchWarps * BK * 4;
-    static constexpr int NBAR = 2 * NXS + 2 * NWS + 2 * NBS + 2 * NTS + 4 * NXB + 1;
+    static constexpr int OFF_E = OFF_B + NBS * B_PANEL;                 // epilogue staging
+    static constexpr int OFF_BAR = OFF_E + kEpiWarps * kEpiStage;
+    static constexpr int NBAR = 2 * NXS + 2 * NWS + 2 * NBS + 3;
     static constexpr int USED = OFF_BAR + NBAR * 8 + 16;
     // at least 120 KB so that one CTA owns the SM (it allocates all 512 TMEM columns)
     static constexpr int SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
     static_assert(S % 16 == 0 && S >= 16 && C >= 2, "UMMA K-steps of 16, sketch only for c >= 2");
-    static_assert(BK % 64 == 0 && BK <= 256, "X panels of 64 inputs");
-    static_assert(kAccCols + 2 * NXB * XCOLS <= 512, "TMEM budget");
-    static_assert(kRows * kNeu * 2 <= NXS * kXPanel, "epilogue staging overlays the X ring");
+    static_assert(BK % 64 == 0 && BK <= 256, "X boxes of 64 inputs");
+    static_assert(SB >= 2 && SP % SB == 0 && NBATCH % 4 == 0, "gather batches split over four warps");
+    static_assert(kAccCols + NXB * BK <= 512, "TMEM budget");
+    static_assert(W_PANEL % (32 * 16) == 0, "Wc panel copied in 16-byte pieces by one warp");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -93,6 +99,13 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, in
         ptx::mbar_wait(&full[i % n], (i / n) & 1, &no_abort, kWaitNs);
 }
 
+// Lane 0 waits, the warp follows: one poller per warp instead of 32.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, kWaitNs);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 template <int RB>
 __device__ __forceinline__ uint32_t kmajor_off(int row, int col) {
     const uint32_t chunk = (uint32_t)(col >> 3) ^ (uint32_t)(((row * RB) >> 7) & (RB / 16 - 1));
@@ -106,131 +119,124 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32
 
 template <int BK, int C>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-               const __grid_constant__ CUtensorMap tmap_y, const uint32_t* __restrict__ gather, int KC,
-               int32_t* status) {
+    tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __nv_bfloat16* __restrict__ Wc,
+               __nv_bfloat16* __restrict__ Y, const uint32_t* __restrict__ gather, int M, int N, int Kc, int KC,
+               int NB, int num_tiles, int32_t* status) {
     using F = Cfg<BK, C>;
-    constexpr int S = F::S, SP = F::SP, NSP = F::NSP, NXS = F::NXS, NWS = F::NWS, NBS = F::NBS, NTS = F::NTS;
+    constexpr int S = F::S, SP = F::SP, SB = F::SB, NSP = F::NSP, NXS = F::NXS, NWS = F::NWS, NBS = F::NBS;
     constexpr int NXB = F::NXB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* xring = smem + F::OFF_X;
     uint8_t* wring = smem + F::OFF_W;
     uint8_t* bring = smem + F::OFF_B;
-    uint8_t* tring = smem + F::OFF_T;
-    uint32_t* atab = reinterpret_cast<uint32_t*>(smem + F::OFF_A);
+    uint8_t* estage = smem + F::OFF_E;
     uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
     uint64_t* x_empty = x_full + NXS;
     uint64_t* w_full = x_empty + NXS;
     uint64_t* w_empty = w_full + NWS;
     uint64_t* b_full = w_empty + NWS;
     uint64_t* b_empty = b_full + NBS;
-    uint64_t* t_full = b_empty + NBS;
-    uint64_t* t_empty = t_full + NTS;
-    uint64_t* tx_full = t_empty + NTS;       // [NXB * 2], index xb * 2 + half
-    uint64_t* tx_free = tx_full + 2 * NXB;
-    uint64_t* acc_full = tx_free + 2 * NXB;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* acc_full = b_empty + NBS;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_empty + 1;         // abort path: completion of every issued MMA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int nb = blockIdx.x;
-    const int m0 = blockIdx.y * kRows;
+    const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NXS; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < NXS; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kSketchWarps); }
         for (int i = 0; i < NWS; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
-        for (int i = 0; i < NBS; ++i) { ptx::mbar_init(&b_full[i], 32 * kSketchWarps); ptx::mbar_init(&b_empty[i], 1); }
-        for (int i = 0; i < NTS; ++i) { ptx::mbar_init(&t_full[i], 1); ptx::mbar_init(&t_empty[i], 32 * kSketchWarps); }
-        for (int i = 0; i < 2 * NXB; ++i) { ptx::mbar_init(&tx_full[i], 1); ptx::mbar_init(&tx_free[i], 128); }
+        for (int i = 0; i < NBS; ++i) { ptx::mbar_init(&b_full[i], kSketchWarps); ptx::mbar_init(&b_empty[i], 1); }
         ptx::mbar_init(acc_full, 1);
+        ptx::mbar_init(acc_empty, kEpiWarps);
+        ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 2) {
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&tmap_x);
-        ptx::prefetch_tmap(&tmap_w);
-        ptx::prefetch_tmap(&tmap_y);
-    }
+    if (warp == 0 && lane == 0) ptx::prefetch_tmap(&tmap_x);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------------ X loads (TMA)
+        // One TMA instruction moves a [256 rows x 64 inputs] box (32 KB). The engine takes a
+        // roughly fixed time per instruction, so boxes are as large as the layout allows.
         if (lane == 0) {
-            int xp = 0, wp = 0, tp = 0;
-            for (int kc = 0; kc < KC && !*abort_flag; ++kc) {
-                const int ti = kc % NTS;
-                if (!ptx::mbar_wait(&t_empty[ti], ((kc / NTS) & 1) ^ 1, abort_flag, kWaitNs)) { report(status, abort_flag, 1); break; }
-                ptx::mbar_arrive_expect_tx(&t_full[ti], F::TAB);
-                ptx::bulk_load(tring + ti * F::TAB, gather + ((size_t)nb * KC + kc) * 2 * BK, F::TAB, &t_full[ti]);
-                ++tp;
-                bool ok = true;
-                for (int h = 0; h < 2 && ok; ++h)
-                    for (int p = 0; p < F::XPH; ++p) {
-                        const int slot = xp % NXS;
-                        if (!ptx::mbar_wait(&x_empty[slot], ((xp / NXS) & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; break; }
-                        ptx::mbar_arrive_expect_tx(&x_full[slot], kXPanel);
-                        ptx::tma_load_2d(xring + slot * kXPanel, &tmap_x, &x_full[slot], kc * BK + 64 * p, m0 + 128 * h);
-                        ++xp;
-                    }
-                if (!ok) { report(status, abort_flag, 2); break; }
-                for (int sp = 0; sp < NSP; ++sp) {
-                    const int wi = wp % NWS;
-                    if (!ptx::mbar_wait(&w_empty[wi], ((wp / NWS) & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&w_full[wi], F::W_PANEL);
-                    ptx::tma_load_2d(wring + wi * F::W_PANEL, &tmap_w, &w_full[wi], kc * S + sp * SP, nb * kNeu);
-                    ++wp;
-                }
-                if (!ok) { report(status, abort_flag, 3); break; }
-            }
-            if (*abort_flag) {   // every issued copy must land before the CTA may exit
-                drain_ring(x_full, NXS, xp, NXS);
-                drain_ring(w_full, NWS, wp, NWS);
-                drain_ring(t_full, NTS, tp, NTS);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ TMEM copy + MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, kRows);
             int xp = 0;
             bool ok = true;
-            for (int it = 0; it <= KC && ok; ++it) {
-                if (it < KC) {
-                    const int xb = it % NXB;
-                    for (int h = 0; h < 2 && ok; ++h) {
-                        if (!ptx::mbar_wait(&tx_free[xb * 2 + h], ((it / NXB) & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 4); break; }
-                        ptx::tc_fence_after();
-                        for (int p = 0; p < F::XPH; ++p) {
-                            const int slot = xp % NXS;
-                            if (!ptx::mbar_wait(&x_full[slot], (xp / NXS) & 1, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 5); break; }
-                            const uint32_t col = kAccCols + (uint32_t)((xb * 2 + h) * F::XCOLS + p * 32);
-                            const uint32_t src = ptx::smem_u32(xring + slot * kXPanel);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                ptx::tmem_cp_128x256b(tm + col + q * 8, ptx::smem_desc(src + q * 32, 16, 1024, ptx::kLayoutSW128));
-                            ptx::umma_commit(&x_empty[slot]);
-                            ++xp;
-                        }
-                        if (ok) ptx::umma_commit(&tx_full[xb * 2 + h]);
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile / NB) * kRows;
+                for (int kc = 0; kc < KC && ok; ++kc)
+                    for (int p = 0; p < F::XPH; ++p, ++xp) {
+                        const int slot = xp % NXS;
+                        if (!ptx::mbar_wait(&x_empty[slot], ((xp / NXS) & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 1); break; }
+                        ptx::mbar_arrive_expect_tx(&x_full[slot], kXSlot);
+                        ptx::tma_load_2d(xring + slot * kXSlot, &tmap_x, &x_full[slot], kc * BK + 64 * p, m0);
                     }
+            }
+            if (*abort_flag) drain_ring(x_full, NXS, xp, NXS);   // every issued copy lands before exit
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ Wc loads (cp.async)
+        // Wc panels take the LSU path (16-byte cp.async per lane) so that the TMA engine serves X
+        // only. A panel is published after the warp's copies land (wait_group) and a proxy fence.
+        int wp = 0, pending = -1;
+        bool ok = true;
+        auto publish = [&](int i) {
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&w_full[i % NWS]);
+        };
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int nb = tile % NB;
+            for (int kc = 0; kc < KC && ok; ++kc)
+                for (int sp = 0; sp < NSP; ++sp, ++wp) {
+                    const int wi = wp % NWS;
+                    if (!warp_wait(&w_empty[wi], ((wp / NWS) & 1) ^ 1, abort_flag)) { ok = false; if (lane == 0) report(status, abort_flag, 2); break; }
+                    uint8_t* dst = wring + wi * F::W_PANEL;
+                    const __nv_bfloat16* src = Wc + (size_t)nb * kNeu * Kc + (size_t)kc * S + sp * SP;
+                    constexpr int kPieces = F::W_PANEL / 16, kPerRow = F::RB / 16;
+#pragma unroll 4
+                    for (int i = lane; i < kPieces; i += 32) {
+                        const int r = i / kPerRow, c = i % kPerRow;
+                        ptx::cp_async_16(dst + kmajor_off<F::RB>(r, c * 8), src + (size_t)r * Kc + c * 8);
+                    }
+                    asm volatile("cp.async.commit_group;" ::: "memory");
+                    if (pending >= 0) {   // the previous panel's copies have landed
+                        asm volatile("cp.async.wait_group 1;" ::: "memory");
+                        publish(pending);
+                    }
+                    pending = wp;
                 }
-                if (it >= 1 && ok) {
-                    const int kc = it - 1;
-                    for (int sp = 0; sp < NSP; ++sp) {
-                        const int wc = kc * NSP + sp;
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        if (ok && pending >= 0) publish(pending);
+    } else if (warp == 2) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, kRows);
+            int wc = 0;
+            bool ok = true;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                // the epilogue must have read the previous tile's accumulator
+                if (!ptx::mbar_wait(acc_empty, (t & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 3); break; }
+                ptx::tc_fence_after();
+                for (int kc = 0; kc < KC && ok; ++kc) {
+                    for (int sp = 0; sp < NSP; ++sp, ++wc) {
                         const int wi = wc % NWS, bi = wc % NBS;
                         if (!ptx::mbar_wait(&w_full[wi], (wc / NWS) & 1, abort_flag, kWaitNs) ||
                             !ptx::mbar_wait(&b_full[bi], (wc / NBS) & 1, abort_flag, kWaitNs)) {
                             ok = false;
-                            report(status, abort_flag, 6);
+                            report(status, abort_flag, 4);
                             break;
                         }
                         ptx::tc_fence_after();
@@ -240,131 +246,189 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int kk = 0; kk < SP / 16; ++kk)
                             ptx::umma_bf16_ss(tm, ptx::smem_desc(a0 + kk * 32, 16, F::SBO, F::LAYOUT),
                                               ptx::smem_desc(b0 + kk * 32, 16, F::SBO, F::LAYOUT), idesc,
-                                              (wc > 0 || kk > 0) ? 1u : 0u);
+                                              (kc > 0 || sp > 0 || kk > 0) ? 1u : 0u);
                         ptx::umma_commit(&w_empty[wi]);
                         ptx::umma_commit(&b_empty[bi]);
                     }
                 }
+                if (ok) ptx::umma_commit(acc_full);
             }
-            ptx::umma_commit(acc_full);
-            if (*abort_flag) {
+            if (*abort_flag) {   // MMAs in flight finish before TMEM is released
                 volatile int no_abort = 0;
-                ptx::mbar_wait(acc_full, 0, &no_abort, kWaitNs);   // copies and MMAs in flight finish
+                ptx::umma_commit(drain);
+                ptx::mbar_wait(drain, 0, &no_abort, kWaitNs);
+            }
+        }
+    } else if (warp < kFirstEpi) {
+        // ------------------------------------------------------------------ sketch warps
+        // A thread owns row r = 32*quad + lane (its TMEM lane) and row r + 128 of the tile.
+        const int sw = warp - kFirstSketch;     // 0..15
+        const int group = sw >> 2;              // k quarter of each staged box, slot quarter of each B panel
+        const int quad = warp & 3;              // TMEM lanes 32*quad .. +31
+        const int row0 = quad * 32 + lane;
+        const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16);
+        const int G = my_tiles * KC;
+        int wc = 0, xp = 0, tile = blockIdx.x, kc = 0;
+        // Every sketch warp takes every named barrier of every chunk, also after a time-out
+        // (then it only skips the work), so that no partner warp can be left waiting on one.
+        bool dead = false;
+        for (int g = 0; g < G; ++g) {
+            const int xb = g % NXB;
+            const uint32_t xcol = kAccCols + (uint32_t)(xb * BK);   // TMEM column of input k = xcol + k
+            if constexpr (NXB == 1) {
+                // single TMEM buffer: every warp must be done gathering the previous chunk
+                ptx::named_barrier_sync(2, kSketchWarps * 32);
+            }
+            // ---- stage the chunk into TMEM as row pairs (X[r][k], X[r+128][k]) at column k
+            for (int p = 0; p < F::XPH && !dead; ++p, ++xp) {
+                const int slot = xp % NXS;
+                if (!warp_wait(&x_full[slot], (xp / NXS) & 1, abort_flag)) {
+                    dead = true;
+                    if (lane == 0) report(status, abort_flag, 5);
+                    break;
+                }
+                const uint8_t* p0 = xring + slot * kXSlot + row0 * 128;
+                const uint8_t* p1 = p0 + 128 * 128;
+                uint32_t v[16];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {   // two 16-byte chunks (8 inputs each) of this warp's 16 inputs
+                    const uint32_t chunk = (uint32_t)(group * 2 + c) ^ (uint32_t)(row0 & 7);
+                    const uint4 a = *reinterpret_cast<const uint4*>(p0 + chunk * 16);
+                    const uint4 b = *reinterpret_cast<const uint4*>(p1 + chunk * 16);
+                    v[8 * c + 0] = __byte_perm(a.x, b.x, 0x5410);
+                    v[8 * c + 1] = __byte_perm(a.x, b.x, 0x7632);
+                    v[8 * c + 2] = __byte_perm(a.y, b.y, 0x5410);
+                    v[8 * c + 3] = __byte_perm(a.y, b.y, 0x7632);
+                    v[8 * c + 4] = __byte_perm(a.z, b.z, 0x5410);
+                    v[8 * c + 5] = __byte_perm(a.z, b.z, 0x7632);
+                    v[8 * c + 6] = __byte_perm(a.w, b.w, 0x5410);
+                    v[8 * c + 7] = __byte_perm(a.w, b.w, 0x7632);
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&x_empty[slot]);
+                ptx::tmem_st_32x32b_x16(lane_base + xcol + (uint32_t)(p * 64 + group * 16), v);
+            }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            ptx::named_barrier_sync(2, kSketchWarps * 32);   // the whole chunk is in TMEM
+            ptx::tc_fence_after();
+            const uint32_t* tab = gather + ((size_t)(tile % NB) * KC + kc) * BK;
+            if (++kc == KC) { kc = 0; tile += gridDim.x; }
+            if (dead) continue;
+            const uint32_t xaddr = lane_base + xcol;
+            // ---- gather: one TMEM load and one bf16x2 FMA per source give both rows' partial sums
+            for (int sp = 0; sp < NSP; ++sp, ++wc) {
+                const int bi = wc % NBS;
+                if (!warp_wait(&b_empty[bi], ((wc / NBS) & 1) ^ 1, abort_flag)) {
+                    dead = true;
+                    if (lane == 0) report(status, abort_flag, 6);
+                    break;
+                }
+                uint8_t* bp = bring + bi * F::B_PANEL;
+#pragma unroll 1
+                for (int bt = group; bt < F::NBATCH; bt += 4) {
+                    const int e0 = (sp * SP + bt * SB) * C;   // first source of these SB slots
+                    uint32_t w[kBatch], m[kBatch];
+#pragma unroll
+                    for (int q = 0; q < kBatch / 4; ++q) {
+                        const uint4 e4 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 4 * q));
+                        const uint32_t ee[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            w[4 * q + j] = ptx::tmem_ld_32x32b_x1(xaddr + (ee[j] & 0x1FFu));
+                            m[4 * q + j] = (ee[j] & 0x80008000u) | 0x3F803F80u;   // (+-1, +-1)
+                        }
+                    }
+                    ptx::tmem_ld_wait();
+                    __nv_bfloat162 acc[SB];
+#pragma unroll
+                    for (int i = 0; i < SB; ++i) acc[i] = __floats2bfloat162_rn(0.f, 0.f);
+#pragma unroll
+                    for (int idx = 0; idx < kBatch; ++idx)
+                        acc[idx / C] = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w[idx]),
+                                               *reinterpret_cast<const __nv_bfloat162*>(&m[idx]), acc[idx / C]);
+                    uint32_t r0[SB / 2], r1[SB / 2];   // row r and row r + 128, slot pairs
+#pragma unroll
+                    for (int i = 0; i < SB / 2; ++i) {
+                        const uint32_t a = *reinterpret_cast<uint32_t*>(&acc[2 * i]);
+                        const uint32_t b = *reinterpret_cast<uint32_t*>(&acc[2 * i + 1]);
+                        r0[i] = __byte_perm(a, b, 0x5410);
+                        r1[i] = __byte_perm(a, b, 0x7632);
+                    }
+                    const int s0 = bt * SB;   // first slot inside the panel
+                    uint8_t* d0 = bp + kmajor_off<F::RB>(row0, s0);
+                    uint8_t* d1 = bp + kmajor_off<F::RB>(row0 + 128, s0);
+                    if constexpr (SB == 8) {
+                        *reinterpret_cast<uint4*>(d0) = make_uint4(r0[0], r0[1], r0[2], r0[3]);
+                        *reinterpret_cast<uint4*>(d1) = make_uint4(r1[0], r1[1], r1[2], r1[3]);
+                    } else if constexpr (SB == 4) {
+                        *reinterpret_cast<uint2*>(d0) = make_uint2(r0[0], r0[1]);
+                        *reinterpret_cast<uint2*>(d1) = make_uint2(r1[0], r1[1]);
+                    } else {
+                        *reinterpret_cast<uint32_t*>(d0) = r0[0];
+                        *reinterpret_cast<uint32_t*>(d1) = r1[0];
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&b_full[bi]);
             }
         }
     } else {
-        // ------------------------------------------------------------------ sketch warps
-        const int sw = warp - 2;                     // 0..7
-        const int half = sw >> 2;                    // rows [128*half, 128*half + 128) of the tile
-        const int quad = warp & 3;                   // TMEM lanes 32*quad .. +31
-        const int row = half * 128 + quad * 32 + lane;
-        uint32_t* mytab = atab + sw * BK;
-        for (int kc = 0; kc < KC; ++kc) {
-            const int xb = kc % NXB, ti = kc % NTS;
-            if (!ptx::mbar_wait(&tx_full[xb * 2 + half], (kc / NXB) & 1, abort_flag, kWaitNs) ||
-                !ptx::mbar_wait(&t_full[ti], (kc / NTS) & 1, abort_flag, kWaitNs)) {
-                report(status, abort_flag, 7);
-                break;
-            }
+        // ------------------------------------------------------------------ epilogue warps
+        // Warp `quad` owns neurons [32*quad, 32*quad + 32) of the tile. Per block of 32 rows:
+        // 8 x tcgen05.ld.16x256b (mma fragment layout) -> bf16 -> stmatrix.trans into a private
+        // [32 rows x 32 neurons] staging tile -> 16-byte coalesced stores of Y rows.
+        const int quad = warp & 3;
+        uint8_t* stg = estage + (warp - kFirstEpi) * kEpiStage;
+        const int mi = lane >> 3, mj = lane & 7;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            const int nb = tile % NB, m0 = (tile / NB) * kRows;
+            bool ok = warp_wait(acc_full, t & 1, abort_flag);
+            if (!ok) { if (lane == 0) report(status, abort_flag, 7); break; }
             ptx::tc_fence_after();
-            const uint32_t xbase = tm + ((uint32_t)(quad * 32) << 16) + kAccCols + (uint32_t)((xb * 2 + half) * F::XCOLS);
-            const uint32_t* tcol = reinterpret_cast<const uint32_t*>(tring + ti * F::TAB);
-            const uint32_t* tmul = tcol + BK;
-            __syncwarp();
-            for (int i = lane; i < BK; i += 32) mytab[i] = xbase + tcol[i];
-            __syncwarp();
-            bool ok = true;
-            for (int sp = 0; sp < NSP; ++sp) {
-                const int wc = kc * NSP + sp;
-                const int bi = wc % NBS;
-                if (!ptx::mbar_wait(&b_empty[bi], ((wc / NBS) & 1) ^ 1, abort_flag, kWaitNs)) { ok = false; break; }
-                uint8_t* bp = bring + bi * F::B_PANEL;
 #pragma unroll 1
-                for (int s8 = 0; s8 < SP / 8; ++s8) {
-                    const int e0 = (sp * SP + s8 * 8) * C;   // first source of these 8 slots
-                    uint32_t w[8 * C];
+            for (int rb = 0; rb < kRows; rb += 32) {
+                uint32_t r[4][8];
 #pragma unroll
-                    for (int q = 0; q < 2 * C; ++q) {
-                        const uint4 t4 = *reinterpret_cast<const uint4*>(mytab + e0 + 4 * q);
-                        w[4 * q + 0] = ptx::tmem_ld_32x32b_x1(t4.x);
-                        w[4 * q + 1] = ptx::tmem_ld_32x32b_x1(t4.y);
-                        w[4 * q + 2] = ptx::tmem_ld_32x32b_x1(t4.z);
-                        w[4 * q + 3] = ptx::tmem_ld_32x32b_x1(t4.w);
-                    }
-                    ptx::tmem_ld_wait();
-                    __nv_bfloat162 acc[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = __floats2bfloat162_rn(0.f, 0.f);
-#pragma unroll
-                    for (int q = 0; q < 2 * C; ++q) {
-                        const uint4 m4 = *reinterpret_cast<const uint4*>(tmul + e0 + 4 * q);
-                        const uint32_t mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int idx = 4 * q + j;
-                            acc[idx / C] = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w[idx]),
-                                                   *reinterpret_cast<const __nv_bfloat162*>(&mm[j]), acc[idx / C]);
-                        }
-                    }
-                    uint32_t out[4];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const uint32_t a = *reinterpret_cast<uint32_t*>(&acc[2 * p]);
-                        const uint32_t b = *reinterpret_cast<uint32_t*>(&acc[2 * p + 1]);
-                        const uint32_t lo = __byte_perm(a, b, 0x5410), hi = __byte_perm(a, b, 0x7632);
-                        __nv_bfloat162 r = __hadd2(*reinterpret_cast<const __nv_bfloat162*>(&lo),
-                                                   *reinterpret_cast<const __nv_bfloat162*>(&hi));
-                        out[p] = *reinterpret_cast<uint32_t*>(&r);
-                    }
-                    *reinterpret_cast<uint4*>(bp + kmajor_off<F::RB>(row, s8 * 8)) = make_uint4(out[0], out[1], out[2], out[3]);
+                for (int b = 0; b < 4; ++b) {
+                    const uint32_t col = (uint32_t)(rb + 8 * b);
+                    ptx::tmem_ld_16x256b(tm + ((uint32_t)(quad * 32) << 16) + col, r[b][0], r[b][1], r[b][2], r[b][3]);
+                    ptx::tmem_ld_16x256b(tm + ((uint32_t)(quad * 32 + 16) << 16) + col, r[b][4], r[b][5], r[b][6], r[b][7]);
                 }
-                ptx::fence_proxy_async_smem();
-                ptx::mbar_arrive(&b_full[bi]);
-            }
-            if (!ok) { report(status, abort_flag, 8); break; }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&tx_free[xb * 2 + half]);
-            ptx::mbar_arrive(&t_empty[ti]);
-        }
-
-        // ------------------------------------------------------------------ epilogue (warps 2..5)
-        if (warp <= 5) {
-            bool ok = ptx::mbar_wait(acc_full, 0, abort_flag, kWaitNs);
-            if (!ok) report(status, abort_flag, 9);
-            ptx::tc_fence_after();
-            ok = __all_sync(0xffffffffu, ok && !*abort_flag);
-            uint8_t* stage = xring;   // [2 boxes][256 rows][64 neurons] bf16, 128B-swizzled
-            if (ok) {
-                const int mi = lane >> 3, mj = lane & 7;
-                const int n = quad * 32 + mi * 8;          // first neuron of this thread's 8x8 matrix
-                const int box = n >> 6, nin = n & 63;
-#pragma unroll 1
-                for (int c0 = 0; c0 < kRows; c0 += 8) {
-                    uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
-                    ptx::tmem_ld_16x256b(tm + ((uint32_t)(quad * 32) << 16) + c0, r0, r1, r2, r3);
-                    ptx::tmem_ld_16x256b(tm + ((uint32_t)(quad * 32 + 16) << 16) + c0, r4, r5, r6, r7);
-                    ptx::tmem_ld_wait();
-                    const int rrow = c0 + mj;
-                    const uint32_t off = (uint32_t)(box * (kRows * 128) + rrow * 128) +
-                                         ((uint32_t)((nin >> 3) ^ (rrow & 7)) << 4);
-                    ptx::stmatrix_x4_trans(ptx::smem_u32(stage + off), pack_bf16x2(r0, r1), pack_bf16x2(r2, r3),
-                                           pack_bf16x2(r4, r5), pack_bf16x2(r6, r7));
+                ptx::tmem_ld_wait();
+                if (rb == kRows - 32) {   // accumulator fully read: the next tile's MMAs may start
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(acc_empty);
                 }
-                ptx::fence_proxy_async_smem();
-            }
-            ptx::named_barrier_sync(1, 128);
-            if (warp == 2 && lane == 0 && !*abort_flag) {
-                ptx::tma_store_2d(&tmap_y, stage, nb * kNeu, m0);
-                ptx::tma_store_2d(&tmap_y, stage + kRows * 128, nb * kNeu + 64, m0);
-                ptx::tma_store_commit();
-                ptx::tma_store_wait0();
+                // staging row y (0..31) holds neurons 0..31 as 64 bytes; 16-byte chunk c of row y
+                // sits at chunk position c ^ ((y >> 1) & 3) so that both stmatrix and the reads
+                // below touch distinct banks
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int y = 8 * b + mj;                      // staging row of this thread's address
+                    const uint32_t off = (uint32_t)(y * 64) + ((uint32_t)(mi ^ ((y >> 1) & 3)) << 4);
+                    ptx::stmatrix_x4_trans(ptx::smem_u32(stg + off), pack_bf16x2(r[b][0], r[b][1]), pack_bf16x2(r[b][2], r[b][3]),
+                                           pack_bf16x2(r[b][4], r[b][5]), pack_bf16x2(r[b][6], r[b][7]));
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {   // 32 rows x 4 chunks = 128 pieces of 16 bytes
+                    const int piece = i * 32 + lane, y = piece >> 2, c = piece & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(stg + y * 64 + ((c ^ ((y >> 1) & 3)) << 4));
+                    const int m = m0 + rb + y;
+                    if (m < M) *reinterpret_cast<uint4*>(Y + (size_t)m * N + (size_t)nb * kNeu + quad * 32 + c * 8) = v;
+                }
+                __syncwarp();
             }
         }
     }
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 2) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tm, 512);
     }
@@ -392,15 +456,13 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
         attr_err = cudaFuncSetAttribute(tc2_kernel<BK, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    const CUtensorMapSwizzle wsw = F::SP == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                               : (F::SP == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-    CUtensorMap mx, mw, my;
-    if (!make_map(&mx, X, (uint64_t)L.K, (uint64_t)M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, F::SP, kNeu, wsw) ||
-        !make_map(&my, Y, (uint64_t)L.N, (uint64_t)M, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    dim3 grid((unsigned)L.NB, (unsigned)((M + kRows - 1) / kRows));
-    tc2_kernel<BK, C><<<grid, kThreads, F::SMEM, st>>>(mx, mw, my, L.d_gather, L.KC, L.status_dev);
+    CUtensorMap mx;
+    if (!make_map(&mx, X, (uint64_t)L.K, (uint64_t)M, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+    const int64_t mtiles = (M + kRows - 1) / kRows;
+    const int64_t tiles = mtiles * L.NB;
+    const int grid = (int)(tiles < L.num_sms ? tiles : L.num_sms);
+    tc2_kernel<BK, C><<<grid, kThreads, F::SMEM, st>>>(mx, (const __nv_bfloat16*)Wc, (__nv_bfloat16*)Y, L.d_gather, (int)M,
+                                                       (int)L.N, (int)(L.K / L.c), L.KC, L.NB, (int)tiles, L.status_dev);
     return cudaGetLastError();
 }
 
@@ -415,7 +477,7 @@ bool tc2_supported(const ss1_layer& L) {
 }
 
 cudaError_t launch_tc2(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    if ((M + kRows - 1) / kRows > 65535) return cudaErrorInvalidValue;
+    if ((M + kRows - 1) / kRows * L.NB > (int64_t)1 << 30) return cudaErrorInvalidValue;
 #define SS1_TC2_CASE(bk, cc) \
     if (L.BK == bk && L.c == cc) return launch_cfg<bk, cc>(L, X, Wc, Y, M, st);
     SS1_TC2_CASE(64, 2)
