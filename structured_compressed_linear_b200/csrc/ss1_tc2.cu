@@ -80,6 +80,7 @@ struct Cfg {
     static_assert(S % 16 == 0 && S >= 16 && C >= 2, "UMMA K-steps of 16, sketch only for c >= 2");
     static_assert(BK % 64 == 0 && BK <= 256, "X boxes of 64 inputs");
     static_assert(SB >= 2 && SP % SB == 0 && NBATCH % 4 == 0, "gather batches split over four warps");
+    static_assert((NBATCH / 4) % (NBATCH / 4 < 2 ? NBATCH / 4 : 2) == 0, "load rounds cover a warp's batches");
     static_assert(kAccCols + NXB * BK <= 512, "TMEM budget");
     static_assert(W_PANEL % (32 * 16) == 0, "Wc panel copied in 16-byte pieces by one warp");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -276,8 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int xb = g % NXB;
             const uint32_t xcol = kAccCols + (uint32_t)(xb * BK);   // TMEM column of input k = xcol + k
             if constexpr (NXB == 1) {
-                // single TMEM buffer: every warp must be done gathering the previous chunk
+                // single TMEM buffer: every warp's loads of the previous chunk are ordered before
+                // any warp's stores of this one (tcgen05 fences around the thread barrier)
+                ptx::tc_fence_before();
                 ptx::named_barrier_sync(2, kSketchWarps * 32);
+                ptx::tc_fence_after();
             }
             // ---- stage the chunk into TMEM as row pairs (X[r][k], X[r+128][k]) at column k
             for (int p = 0; p < F::XPH && !dead; ++p, ++xp) {
@@ -314,9 +318,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const uint32_t* tab = gather + ((size_t)(tile % NB) * KC + kc) * BK;
             if (++kc == KC) { kc = 0; tile += gridDim.x; }
+            // the next chunk's table lines are pulled into L1 now, so that its gathers do not
+            // wait for an L2 round trip before they can even form their TMEM addresses
+            if (tile < num_tiles) {
+                const uint32_t* next = gather + ((size_t)(tile % NB) * KC + kc) * BK;
+                for (int sp = 0; sp < NSP; ++sp)
+                    for (int bt = group; bt < F::NBATCH; bt += 4)
+                        if (lane == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(next + (sp * SP + bt * SB) * C));
+            }
             if (dead) continue;
             const uint32_t xaddr = lane_base + xcol;
-            // ---- gather: one TMEM load and one bf16x2 FMA per source give both rows' partial sums
+            // ---- gather: one TMEM load and one bf16x2 FMA per source give both rows' partial sums.
+            // All of this warp's sources of a panel (kPerWarp batches) are in flight before one wait.
+            constexpr int kPerWarp = F::NBATCH / 4 < 2 ? F::NBATCH / 4 : 2;   // batches per load round
             for (int sp = 0; sp < NSP; ++sp, ++wc) {
                 const int bi = wc % NBS;
                 if (!warp_wait(&b_empty[bi], ((wc / NBS) & 1) ^ 1, abort_flag)) {
@@ -326,47 +340,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 uint8_t* bp = bring + bi * F::B_PANEL;
 #pragma unroll 1
-                for (int bt = group; bt < F::NBATCH; bt += 4) {
-                    const int e0 = (sp * SP + bt * SB) * C;   // first source of these SB slots
-                    uint32_t w[kBatch], m[kBatch];
+                for (int bt0 = group; bt0 < F::NBATCH; bt0 += 4 * kPerWarp) {
+                    uint32_t w[kPerWarp][kBatch], m[kPerWarp][kBatch];
 #pragma unroll
-                    for (int q = 0; q < kBatch / 4; ++q) {
-                        const uint4 e4 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 4 * q));
-                        const uint32_t ee[4] = {e4.x, e4.y, e4.z, e4.w};
+                    for (int u = 0; u < kPerWarp; ++u) {
+                        const int e0 = (sp * SP + (bt0 + 4 * u) * SB) * C;   // first source of batch u
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            w[4 * q + j] = ptx::tmem_ld_32x32b_x1(xaddr + (ee[j] & 0x1FFu));
-                            m[4 * q + j] = (ee[j] & 0x80008000u) | 0x3F803F80u;   // (+-1, +-1)
+                        for (int q = 0; q < kBatch / 4; ++q) {
+                            const uint4 e4 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 4 * q));
+                            const uint32_t ee[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                w[u][4 * q + j] = ptx::tmem_ld_32x32b_x1(xaddr + (ee[j] & 0x1FFu));
+                                m[u][4 * q + j] = (ee[j] & 0x80008000u) | 0x3F803F80u;   // (+-1, +-1)
+                            }
                         }
                     }
                     ptx::tmem_ld_wait();
-                    __nv_bfloat162 acc[SB];
 #pragma unroll
-                    for (int i = 0; i < SB; ++i) acc[i] = __floats2bfloat162_rn(0.f, 0.f);
+                    for (int u = 0; u < kPerWarp; ++u) {
+                        __nv_bfloat162 acc[SB];
 #pragma unroll
-                    for (int idx = 0; idx < kBatch; ++idx)
-                        acc[idx / C] = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w[idx]),
-                                               *reinterpret_cast<const __nv_bfloat162*>(&m[idx]), acc[idx / C]);
-                    uint32_t r0[SB / 2], r1[SB / 2];   // row r and row r + 128, slot pairs
+                        for (int i = 0; i < SB; ++i) acc[i] = __floats2bfloat162_rn(0.f, 0.f);
 #pragma unroll
-                    for (int i = 0; i < SB / 2; ++i) {
-                        const uint32_t a = *reinterpret_cast<uint32_t*>(&acc[2 * i]);
-                        const uint32_t b = *reinterpret_cast<uint32_t*>(&acc[2 * i + 1]);
-                        r0[i] = __byte_perm(a, b, 0x5410);
-                        r1[i] = __byte_perm(a, b, 0x7632);
-                    }
-                    const int s0 = bt * SB;   // first slot inside the panel
-                    uint8_t* d0 = bp + kmajor_off<F::RB>(row0, s0);
-                    uint8_t* d1 = bp + kmajor_off<F::RB>(row0 + 128, s0);
-                    if constexpr (SB == 8) {
-                        *reinterpret_cast<uint4*>(d0) = make_uint4(r0[0], r0[1], r0[2], r0[3]);
-                        *reinterpret_cast<uint4*>(d1) = make_uint4(r1[0], r1[1], r1[2], r1[3]);
-                    } else if constexpr (SB == 4) {
-                        *reinterpret_cast<uint2*>(d0) = make_uint2(r0[0], r0[1]);
-                        *reinterpret_cast<uint2*>(d1) = make_uint2(r1[0], r1[1]);
-                    } else {
-                        *reinterpret_cast<uint32_t*>(d0) = r0[0];
-                        *reinterpret_cast<uint32_t*>(d1) = r1[0];
+                        for (int idx = 0; idx < kBatch; ++idx)
+                            acc[idx / C] = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&w[u][idx]),
+                                                   *reinterpret_cast<const __nv_bfloat162*>(&m[u][idx]), acc[idx / C]);
+                        uint32_t r0[SB / 2], r1[SB / 2];   // row r and row r + 128, slot pairs
+#pragma unroll
+                        for (int i = 0; i < SB / 2; ++i) {
+                            const uint32_t a = *reinterpret_cast<uint32_t*>(&acc[2 * i]);
+                            const uint32_t b = *reinterpret_cast<uint32_t*>(&acc[2 * i + 1]);
+                            r0[i] = __byte_perm(a, b, 0x5410);
+                            r1[i] = __byte_perm(a, b, 0x7632);
+                        }
+                        const int s0 = (bt0 + 4 * u) * SB;   // first slot inside the panel
+                        uint8_t* d0 = bp + kmajor_off<F::RB>(row0, s0);
+                        uint8_t* d1 = bp + kmajor_off<F::RB>(row0 + 128, s0);
+                        if constexpr (SB == 8) {
+                            *reinterpret_cast<uint4*>(d0) = make_uint4(r0[0], r0[1], r0[2], r0[3]);
+                            *reinterpret_cast<uint4*>(d1) = make_uint4(r1[0], r1[1], r1[2], r1[3]);
+                        } else if constexpr (SB == 4) {
+                            *reinterpret_cast<uint2*>(d0) = make_uint2(r0[0], r0[1]);
+                            *reinterpret_cast<uint2*>(d1) = make_uint2(r1[0], r1[1]);
+                        } else {
+                            *reinterpret_cast<uint32_t*>(d0) = r0[0];
+                            *reinterpret_cast<uint32_t*>(d1) = r1[0];
+                        }
                     }
                 }
                 ptx::fence_proxy_async_smem();

@@ -106,3 +106,22 @@ def test_error_conventions():
     assert lib.ss1_forward(raw, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 0, st) == -7
     assert lib.ss1_destroy(raw) == -7
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("c,BK", [(2, 256), (8, 256), (2, 128), (4, 128)])
+def test_repeated_calls_bit_identical(c, BK):
+    """The tensor-core kernel has a fixed reduction order: repeated calls give identical bits.
+    Guards the ordering between one chunk's TMEM gathers and the next chunk's TMEM staging
+    (a missing tcgen05 fence there showed up as run-to-run differences)."""
+    ss1 = get_ss1()
+    K, N, M = 4096, 1024, 2048
+    layer = _layer(ss1, K, N, c, BK, 128, seed=17)
+    gen = torch.Generator().manual_seed(23)
+    X = torch.randn(M, K, generator=gen).to(torch.bfloat16).cuda()
+    Wc = (torch.randn(N, K // c, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    first = layer.forward(X, Wc, kernel=TC)
+    for _ in range(4):
+        assert torch.equal(layer.forward(X, Wc, kernel=TC), first)
+    torch.cuda.synchronize()
+    assert layer.device_status() == (0, 0)
+    layer.close()
