@@ -102,7 +102,8 @@ SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, in
  * ss1_forward_with -- ss1_forward with an explicit kernel (enum ss1_kernel). Same arguments,
  * ownership and errors; additionally UNSUPPORTED_SHAPE when the chosen kernel cannot run this
  * (dtype, M, shape): TC needs bf16, S = BK / c a multiple of 16, BN == 128 and K % 8 == 0;
- * SMALLM needs bf16 and M <= 64; SIMT runs every valid shape.
+ * SMALLM needs bf16, M <= 64, S = BK / c a power of two >= 8, BN a multiple of 8 and K, K / c
+ * multiples of 8; SIMT runs every valid shape.
  */
 SS1_API int ss1_forward_with(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
                              int kernel, void* stream);

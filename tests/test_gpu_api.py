@@ -12,7 +12,13 @@ from tests.gpu_common import get_ss1, to_np64
 pytestmark = pytest.mark.gpu
 
 SIMT, TC, SMALLM = 2, 1, 3
-BF16_KERNELS = [SIMT, TC]
+BF16_KERNELS = [SIMT, TC, SMALLM]
+SMALLM_MAX_ROWS = 64
+
+
+def _rows(kernel, M):
+    """Row count a test uses with this kernel: the small-M kernel takes at most 64 rows."""
+    return min(M, SMALLM_MAX_ROWS) if kernel == SMALLM else M
 
 
 def _layer(ss1, K=512, N=256, c=4, BK=128, BN=128, seed=3):
@@ -30,7 +36,8 @@ def test_one_hot_probe_bit_exact(kernel, c, BK):
     gen = torch.Generator().manual_seed(5)
     Wc = (torch.randn(N, K // c, generator=gen) * 0.1).to(torch.bfloat16)
     X = torch.eye(K, dtype=torch.bfloat16)
-    Y = layer.forward(X.cuda(), Wc.cuda(), kernel=kernel)
+    step = _rows(kernel, K)
+    Y = torch.cat([layer.forward(X[r:r + step].cuda(), Wc.cuda(), kernel=kernel) for r in range(0, K, step)])
     h, g = O.ss1_tables(K, N, c, BK, BN, 11)
     Wfull = np.concatenate([O.expand_weight(to_np64(Wc), h, g, BN, nb) for nb in range(N // BN)])
     assert np.array_equal(to_np64(Y), Wfull.T)
@@ -42,8 +49,9 @@ def test_zero_negation_linearity(kernel):
     ss1 = get_ss1()
     layer = _layer(ss1)
     gen = torch.Generator().manual_seed(9)
-    X1 = torch.randn(300, 512, generator=gen).to(torch.bfloat16).cuda()
-    X2 = torch.randn(300, 512, generator=gen).to(torch.bfloat16).cuda()
+    M = _rows(kernel, 300)
+    X1 = torch.randn(M, 512, generator=gen).to(torch.bfloat16).cuda()
+    X2 = torch.randn(M, 512, generator=gen).to(torch.bfloat16).cuda()
     Wc = (torch.randn(256, 128, generator=gen) * 0.05).to(torch.bfloat16).cuda()
     Y0 = layer.forward(torch.zeros_like(X1), Wc, kernel=kernel)
     assert torch.count_nonzero(Y0).item() == 0
@@ -64,11 +72,11 @@ def test_guard_band_and_zero_rows():
     layer = _layer(ss1)
     lib = ss1.lib()
     gen = torch.Generator().manual_seed(1)
-    M = 129
-    X = torch.randn(M, 512, generator=gen).to(torch.bfloat16).cuda()
     Wc = (torch.randn(256, 128, generator=gen) * 0.05).to(torch.bfloat16).cuda()
-    buf = torch.full((M + 7, 256), 7.0, dtype=torch.bfloat16, device="cuda")
     for k in [0] + BF16_KERNELS:
+        M = _rows(k, 129) - 2   # ragged against every row tile
+        X = torch.randn(M, 512, generator=gen).to(torch.bfloat16).cuda()
+        buf = torch.full((M + 7, 256), 7.0, dtype=torch.bfloat16, device="cuda")
         st = torch.cuda.current_stream().cuda_stream
         assert lib.ss1_forward_with(layer.handle, X.data_ptr(), Wc.data_ptr(), buf.data_ptr(), M, 0, k, st) == 0
         torch.cuda.synchronize()
@@ -91,8 +99,10 @@ def test_error_conventions():
     assert lib.ss1_forward(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), -1, 0, st) == -1
     assert lib.ss1_forward(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 7, st) == -1
     assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 0, 99, st) == -1
-    # fp32 data cannot take the tensor-core path
+    # fp32 data cannot take the tensor-core or small-M path; the small-M path takes <= 64 rows
     assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 1, TC, st) == -8
+    assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 4, 1, SMALLM, st) == -8
+    assert lib.ss1_forward_with(h, X.data_ptr(), Wc.data_ptr(), Y.data_ptr(), 65, 0, SMALLM, st) == -8
     k = ctypes.c_int()
     assert lib.ss1_select_kernel(h, 4096, 1, ctypes.byref(k)) == 0 and k.value == SIMT
     K_, N_ = ctypes.c_int64(), ctypes.c_int64()
@@ -122,6 +132,23 @@ def test_repeated_calls_bit_identical(c, BK):
     first = layer.forward(X, Wc, kernel=TC)
     for _ in range(4):
         assert torch.equal(layer.forward(X, Wc, kernel=TC), first)
+    torch.cuda.synchronize()
+    assert layer.device_status() == (0, 0)
+    layer.close()
+
+
+@pytest.mark.parametrize("M", [1, 5, 8, 40, 64])
+def test_small_m_repeated_calls_bit_identical(M):
+    """The small-M kernel reduces its K split in a fixed order: repeated calls agree bit for bit."""
+    ss1 = get_ss1()
+    K, N = 4096, 14336
+    layer = _layer(ss1, K, N, 2, 256, 128, seed=19)
+    gen = torch.Generator().manual_seed(29)
+    X = torch.randn(M, K, generator=gen).to(torch.bfloat16).cuda()
+    Wc = (torch.randn(N, K // 2, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    first = layer.forward(X, Wc, kernel=SMALLM)
+    for _ in range(3):
+        assert torch.equal(layer.forward(X, Wc, kernel=SMALLM), first)
     torch.cuda.synchronize()
     assert layer.device_status() == (0, 0)
     layer.close()

@@ -30,6 +30,15 @@ def _small_cases():
             for M in (1, 16, 200, 333):
                 cases.append(Layer("bf16-small", M, 1024, 384, c, BK, 128, "bf16", "normal", "normal_002", 3))
     cases.append(Layer("bf16-small", 257, 1280, 640, 4, 128, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2))
+    # decode-sized rows: every row-group width, ragged groups, narrow N-blocks, K past one segment
+    for M in (2, 3, 5, 8, 9, 37, 64):
+        cases.append(Layer("bf16-small", M, 3072, 320, 2, 128, 64, "bf16", "normal", "normal_002", 4))
+    # a K-chunk that is not a power of two (S = 24): outside the small-M kernel's shapes
+    cases.append(Layer("bf16-small", 4, 960, 256, 2, 48, 128, "bf16", "normal", "normal_002", 4))
+    for c in (1, 4, 8):
+        cases.append(Layer("bf16-small", 6, 4608, 256, c, 256, 32, "bf16", "normal_outliers", "normal_002", 6))
+    # wide N: the widest neuron group per CTA
+    cases.append(Layer("bf16-small", 8, 1024, 19456, 4, 128, 128, "bf16", "normal", "normal_002", 7))
     return cases
 
 
@@ -40,10 +49,19 @@ def tc_eligible(L: Layer) -> bool:
             and L.K % 8 == 0 and (L.K // L.c) % 8 == 0)
 
 
+def smallm_eligible(L: Layer) -> bool:
+    """Documented preconditions of the small-M kernel (include/ss1.h)."""
+    S = L.BK // L.c
+    return (L.dtype == "bf16" and 1 <= L.M <= 64 and S >= 8 and S & (S - 1) == 0 and L.BN % 8 == 0
+            and L.K % 8 == 0 and (L.K // L.c) % 8 == 0)
+
+
 def _kernels_for(L: Layer):
     ks = [SIMT]
     if tc_eligible(L):
         ks.append(TC)
+    if smallm_eligible(L):
+        ks.append(SMALLM)
     return ks
 
 
