@@ -21,7 +21,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -40,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=None)
@@ -68,11 +67,19 @@ def layer_work(L):
     return dense, actual, byts
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "TC": ["ss1_tc.cu", "ss1_tc2.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
+    "SMALLM": ["ss1_smallm.cu", "ss1_internal.cuh"],
+    "SIMT": ["ss1_simt.cu", "ss1_internal.cuh"],
+}
+
+
+def kernel_source_hash(kernel_name):
+    """Hash of the sources a kernel is built from; a traffic record holds only for the same hash."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "structured_compressed_linear_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh"))):
-        with open(p, "rb") as f:
+    for name in KERNEL_SOURCES.get(kernel_name, []):
+        with open(os.path.join(pkg, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -85,7 +92,7 @@ def traffic_record(kernel_name):
     with open(p) as f:
         d = json.load(f)
     rec = d.get(kernel_name)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel_name):
         return None
     return rec
 
@@ -209,11 +216,13 @@ def run_reference(args, layers, wid, rank, world):
     prepared = prepare_oracle(layers, max_rows=2048)
     threads = oracle_threads()
     rows = None
+    # each step a bounded sample, so that the whole run stays within a few minutes
+    budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        _, _, rows = oracle_sample_rate(prepared, 2.0, rows)
+        _, _, rows = oracle_sample_rate(prepared, budget, rows)
     times = []
     for _ in range(args.steps):
-        _, dt, rows = oracle_sample_rate(prepared, 2.0, rows)
+        _, dt, rows = oracle_sample_rate(prepared, budget, rows)
         times.append(dt)
     mean_t = statistics.mean(times)
     dense_sample = sum(2.0 * min(rows, L.M) * L.N * L.K for L in layers)
@@ -360,25 +369,30 @@ def main():
     dense_step = sum(layer_work(L)[0] for L in layers)
     value = world * dense_step / (step_ms * 1e-3) / 1e12
 
-    # roofline of the dominant kernel over the step (sum over its launches)
+    # roofline of the dominant kernel over the step (sum over its launches, one per layer)
     tc_peak = peaks["bf16_tflops"] * 1e12
     hbm_peak = peaks["hbm_gbs"] * 1e9
-    t_tc = sum(layer_work(L)[1] / tc_peak for L in layers)
-    t_hbm = sum(layer_work(L)[2] / hbm_peak for L in layers)
-    t_kernel = sum(layer_ms) * 1e-3
-    ns_frac = sum(max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) for L in layers) / t_kernel
+    dom = max(set(kernels), key=kernels.count)
+    dom_layers = [(L, ms) for L, k, ms in zip(layers, kernels, layer_ms) if k == dom]
+    t_tc = sum(layer_work(L)[1] / tc_peak for L, _ in dom_layers)
+    t_hbm = sum(layer_work(L)[2] / hbm_peak for L, _ in dom_layers)
+    t_kernel = sum(ms for _, ms in dom_layers) * 1e-3
+    ns_frac = sum(max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) for L in layers) / (step_ms * 1e-3)
     if t_tc >= t_hbm:
-        achieved = sum(layer_work(L)[1] for L in layers) / t_kernel / 1e12
+        achieved = sum(layer_work(L)[1] for L, _ in dom_layers) / t_kernel / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     else:
-        achieved = sum(layer_work(L)[2] for L in layers) / t_kernel / 1e9
+        achieved = sum(layer_work(L)[2] for L, _ in dom_layers) / t_kernel / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} (burst figure; MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    dom = max(set(kernels), key=kernels.count)
     rec = traffic_record(dom)
     roof["traffic"] = rec["dram_bytes_per_step"] if rec else None
     roof["kernel"] = dom
+    roof["launches_per_step"] = kernels.count(dom)
+    roof["per"] = "one step: the sum over that kernel's launches (one per layer)"
+    roof["algorithmic_bytes"] = sum(layer_work(L)[2] for L, k in zip(layers, kernels) if k == dom)
+    roof["algorithmic_flops"] = sum(layer_work(L)[1] for L, k in zip(layers, kernels) if k == dom)
     roof["frac_slower_of_tensor_and_hbm"] = ns_frac
 
     line = {
