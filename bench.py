@@ -240,6 +240,28 @@ def run_reference(args, layers, wid, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def rank_rows(X, rank):
+    """Rank r's rows: rank 0 keeps the seeded rows, others a rank-seeded permutation of them."""
+    import torch
+    if rank == 0:
+        return X
+    g = torch.Generator().manual_seed(1000 + rank)
+    return X[torch.randperm(X.shape[0], generator=g)]
+
+
+def max_over_ranks(values, world):
+    """Element-wise max of a float64 tensor over all ranks (the slowest rank's timings)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(values, op=dist.ReduceOp.MAX)
+    return values
+
+
+def whole_job_value(dense_flops_per_rank_step, step_ms, world):
+    """Dense-equivalent TFLOP/s of the whole job: every rank's work over the slowest rank's time."""
+    return world * dense_flops_per_rank_step / (step_ms * 1e-3) / 1e12
+
+
 def workload_config(layers, wid, world):
     L0 = layers[0]
     return {
@@ -285,9 +307,7 @@ def main():
     objs = []
     for L in layers:
         X, Wc = make_inputs(L)
-        if rank:
-            g = torch.Generator().manual_seed(1000 + rank)
-            X = X[torch.randperm(X.shape[0], generator=g)]
+        X = rank_rows(X, rank)
         layer = ss1.SS1Layer(L.K, L.N, L.c, L.BK, L.BN, L.seed)
         Xd, Wd = X.to(dev), Wc.to(dev)
         Yd = torch.empty((L.M, L.N), dtype=Xd.dtype, device=dev)
@@ -330,9 +350,7 @@ def main():
     per_layer_ms = [[evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)] for i in range(len(objs))]
     layer_ms = [statistics.mean(v) for v in per_layer_ms]
     step_ms = sum(layer_ms)
-    t = torch.tensor([step_ms] + layer_ms, dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = max_over_ranks(torch.tensor([step_ms] + layer_ms, dtype=torch.float64, device=dev), world)
     step_ms, layer_ms = float(t[0]), [float(x) for x in t[1:]]
 
     # end to end through the public API: pinned host X -> device, forward, device -> pinned host Y
@@ -361,13 +379,11 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / ke], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(torch.tensor([e0.elapsed_time(e1) / ke], dtype=torch.float64, device=dev), world)
         e2e = (float(te[0]), h2d, d2h)
 
     dense_step = sum(layer_work(L)[0] for L in layers)
-    value = world * dense_step / (step_ms * 1e-3) / 1e12
+    value = whole_job_value(dense_step, step_ms, world)
 
     # roofline of the dominant kernel over the step (sum over its launches, one per layer)
     tc_peak = peaks["bf16_tflops"] * 1e12
@@ -412,7 +428,7 @@ def main():
     }
     if e2e is not None:
         ms_e, h2d, d2h = e2e
-        line["e2e"] = {"value": world * dense_step / (ms_e * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_e,
+        line["e2e"] = {"value": whole_job_value(dense_step, ms_e, world), "unit": UNIT, "ms_per_step": ms_e,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "note": "X copied from pinned host memory and Y read back every step; Wc resident"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
