@@ -84,7 +84,7 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
     if (cudaMalloc(&L->d_h, entries * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&L->d_g, entries * sizeof(int8_t)) != cudaSuccess ||
         cudaMalloc(&L->d_src, entries * sizeof(uint16_t)) != cudaSuccess ||
-        cudaMalloc(&L->d_gather, entries * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&L->d_gather, entries * sizeof(uint2)) != cudaSuccess ||
         cudaHostAlloc(&L->status_host, sizeof(int32_t), cudaHostAllocMapped) != cudaSuccess) {
         cudaGetLastError();
         release(L);

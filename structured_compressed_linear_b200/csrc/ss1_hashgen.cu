@@ -77,13 +77,13 @@ __global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int 
 }
 
 // One thread per source: the tensor-core kernel reads X[row, k] and X[row + 128, k] as one
-// bf16x2 TMEM word at column k; the entry is k (bits 0..8) with the sign copied into bits 15
-// and 31, so (entry & 0x80008000) | bf16x2(1, 1) is the +-1 multiplier of both halves.
-__global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint32_t* __restrict__ out, int64_t nsrc) {
+// bf16x2 TMEM word at column k; the entry is {k, the source's sign as the bf16x2 pair (+-1, +-1)},
+// ready to be added to a TMEM address and used as an FMA multiplier without further work.
+__global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint2* __restrict__ out, int64_t nsrc) {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= nsrc) return;
     const uint16_t e = src[i];
-    out[i] = (uint32_t)(e & kSrcIdxMask) | ((e & kSrcNegBit) ? 0x80008000u : 0u);
+    out[i] = make_uint2((uint32_t)(e & kSrcIdxMask), (e & kSrcNegBit) ? 0xBF80BF80u : 0x3F803F80u);
 }
 
 }  // namespace

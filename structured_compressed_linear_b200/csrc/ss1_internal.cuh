@@ -24,7 +24,7 @@ struct ss1_layer {
     int32_t* d_h;        // [NB][K] compressed column of input k in block nb
     int8_t* d_g;         // [NB][K] sign of input k in block nb
     uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
-    uint32_t* d_gather;  // [NB][KC][BK] per source (slot-major): k | sign in bits 15 and 31
+    uint2* d_gather;     // [NB][KC][BK] per source (slot-major): {k, bf16x2 multiplier (+-1, +-1)}
     int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
     int32_t* status_dev;   // device alias of status_host
 };

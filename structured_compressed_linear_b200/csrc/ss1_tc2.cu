@@ -9,19 +9,21 @@
 // share one hash: rows of X do, neurons of two blocks do not. Persistent CTAs (one per SM)
 // walk the tiles with the N-block index fastest, so CTAs running side by side share X in L2.
 // Per K-chunk kc of a tile:
-//   * TMA warp   : X rows [m0, m0+256) x chunk -> 16 KB smem panels [128 rows x 64 k] (128B
-//                  swizzle), both row halves of one 64-input panel back to back; Wc[nb*128:+128,
-//                  kc*S:+S] -> K-major panels; the chunk's gather table -> smem (bulk copy).
+//   * X warp     : X rows [m0, m0+256) x 64 inputs per TMA box (32 KB, 128B swizzle) into a
+//                  3-slot ring.
+//   * Wc warp    : Wc[nb*128:+128, kc*S:+S] with 16-byte cp.async into K-major swizzled panels
+//                  (the UMMA A operand), 3-slot ring.
 //   * 16 sketch warps. A thread owns rows r and r+128 of the tile (r = TMEM lane). They first
 //                  stage the X chunk into TMEM as row pairs: conflict-free 16-byte shared loads,
 //                  byte permutes to (X[r][k], X[r+128][k]), tcgen05.st -> column k. Then, for
 //                  their quarter of the slots, Xs[., s] = sum_j sign_j * X[., k_j] with one
-//                  tcgen05.ld (two rows at once) and one bf16x2 FMA per source, and write both
-//                  rows as the K-major UMMA B operand. The gather touches no shared-memory bank.
+//                  tcgen05.ld (two rows at once) and one bf16x2 FMA per source, whose TMEM
+//                  column and +-1 multiplier come ready-made from the table (L1-resident), and
+//                  write both rows as the K-major UMMA B operand (2-slot ring).
 //   * MMA warp   : S/16 x tcgen05.mma (M=128, N=256, K=16) per chunk into one accumulator.
 //   * 4 epilogue warps: tcgen05.ld.16x256b (mma fragment layout) -> bf16 -> stmatrix.trans into
-//                  a 128B-swizzled [128 rows x 128 neurons] staging tile -> TMA store of Y;
-//                  they release the accumulator as soon as its last column is read.
+//                  a private swizzled [32 rows x 32 neurons] staging tile -> 16-byte stores of
+//                  Y rows; they release the accumulator as soon as its last column is read.
 // Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
 // handle's status word, drains the copies and MMAs in flight and returns (no trap).
 #include "ss1_internal.cuh"
@@ -68,6 +70,7 @@ struct Cfg {
     static constexpr int XPH = BK / 64;                 // X boxes (64 inputs x 256 rows) per chunk
     static constexpr int NXB = BK <= 128 ? 2 : 1;       // TMEM X buffers (BK row-pair columns each)
     static constexpr int NXS = 3, NBS = 2, NWS = 3;
+    static constexpr int TEAMS = NXB;                   // sketch teams: one per TMEM staging buffer
     static constexpr int OFF_X = 0;
     static constexpr int OFF_W = OFF_X + NXS * kXSlot;
     static constexpr int OFF_B = OFF_W + NWS * W_PANEL;
@@ -79,8 +82,9 @@ struct Cfg {
     static constexpr int SMEM = (USED + 1024 > 120 * 1024) ? USED + 1024 : 120 * 1024;
     static_assert(S % 16 == 0 && S >= 16 && C >= 2, "UMMA K-steps of 16, sketch only for c >= 2");
     static_assert(BK % 64 == 0 && BK <= 256, "X boxes of 64 inputs");
-    static_assert(SB >= 2 && SP % SB == 0 && NBATCH % 4 == 0, "gather batches split over four warps");
-    static_assert((NBATCH / 4) % (NBATCH / 4 < 2 ? NBATCH / 4 : 2) == 0, "load rounds cover a warp's batches");
+    static constexpr int GROUPS = 4 / TEAMS;            // slot parts per team (warps per lane quarter)
+    static_assert(SB >= 2 && SP % SB == 0 && NBATCH % GROUPS == 0, "gather batches split over a team's slot parts");
+    static_assert((NBATCH / GROUPS) % (NBATCH / GROUPS < 2 ? NBATCH / GROUPS : 2) == 0, "load rounds cover a warp's batches");
     static_assert(kAccCols + NXB * BK <= 512, "TMEM budget");
     static_assert(W_PANEL % (32 * 16) == 0, "Wc panel copied in 16-byte pieces by one warp");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -121,7 +125,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32
 template <int BK, int C>
 __global__ void __launch_bounds__(kThreads, 1)
     tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __nv_bfloat16* __restrict__ Wc,
-               __nv_bfloat16* __restrict__ Y, const uint32_t* __restrict__ gather, int M, int N, int Kc, int KC,
+               __nv_bfloat16* __restrict__ Y, const uint2* __restrict__ gather_tab, int M, int N, int Kc, int KC,
                int NB, int num_tiles, int32_t* status) {
     using F = Cfg<BK, C>;
     constexpr int S = F::S, SP = F::SP, SB = F::SB, NSP = F::NSP, NXS = F::NXS, NWS = F::NWS, NBS = F::NBS;
@@ -148,9 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NXS; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kSketchWarps); }
+        for (int i = 0; i < NXS; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kSketchWarps / F::TEAMS); }
         for (int i = 0; i < NWS; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
-        for (int i = 0; i < NBS; ++i) { ptx::mbar_init(&b_full[i], kSketchWarps); ptx::mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < NBS; ++i) { ptx::mbar_init(&b_full[i], kSketchWarps / F::TEAMS); ptx::mbar_init(&b_empty[i], 1); }
         ptx::mbar_init(acc_full, 1);
         ptx::mbar_init(acc_empty, kEpiWarps);
         ptx::mbar_init(drain, 1);
@@ -269,23 +273,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = quad * 32 + lane;
         const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16);
         const int G = my_tiles * KC;
-        int wc = 0, xp = 0, tile = blockIdx.x, kc = 0;
-        // Every sketch warp takes every named barrier of every chunk, also after a time-out
-        // (then it only skips the work), so that no partner warp can be left waiting on one.
+        // Teams: with two TMEM staging buffers the 16 warps form two teams of 8 that take
+        // alternate chunks, each with its own buffer, B slot and named barrier, so that one
+        // team's staging (shared-memory reads) overlaps the other's gathering (TMEM reads).
+        // With one buffer all 16 warps form one team.
+        constexpr int kTeams = F::TEAMS, kTeamWarps = kSketchWarps / kTeams, kGroups = kTeamWarps / 4;
+        const int team = sw / kTeamWarps;
+        const int tgroup = (sw % kTeamWarps) >> 2;   // input part of each staged box, slot part of each panel
+        const int bar_id = 2 + team;
+        // Every warp of a team takes every named barrier of each of the team's chunks, also
+        // after a time-out (then it only skips the work), so no partner can be left waiting.
         bool dead = false;
-        for (int g = 0; g < G; ++g) {
-            const int xb = g % NXB;
-            const uint32_t xcol = kAccCols + (uint32_t)(xb * BK);   // TMEM column of input k = xcol + k
-            if constexpr (NXB == 1) {
-                // single TMEM buffer: every warp's loads of the previous chunk are ordered before
-                // any warp's stores of this one (tcgen05 fences around the thread barrier)
-                ptx::tc_fence_before();
-                ptx::named_barrier_sync(2, kSketchWarps * 32);
-                ptx::tc_fence_after();
-            }
-            // ---- stage the chunk into TMEM as row pairs (X[r][k], X[r+128][k]) at column k
-            for (int p = 0; p < F::XPH && !dead; ++p, ++xp) {
-                const int slot = xp % NXS;
+        // Stage chunk g into TMEM buffer xb as row pairs (X[r][k], X[r+128][k]) at column k.
+        // This warp copies 64 / kGroups inputs of each box; the tcgen05.st stay in flight.
+        auto stage = [&](int g, int xb) {
+            constexpr int kIn = 64 / kGroups;        // inputs of a box per warp (16 or 32)
+            const uint32_t xcol = kAccCols + (uint32_t)(xb * BK);
+            for (int p = 0; p < F::XPH && !dead; ++p) {
+                const int xp = g * F::XPH + p, slot = xp % NXS;
                 if (!warp_wait(&x_full[slot], (xp / NXS) & 1, abort_flag)) {
                     dead = true;
                     if (lane == 0) report(status, abort_flag, 5);
@@ -293,10 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint8_t* p0 = xring + slot * kXSlot + row0 * 128;
                 const uint8_t* p1 = p0 + 128 * 128;
-                uint32_t v[16];
+                uint32_t v[kIn];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {   // two 16-byte chunks (8 inputs each) of this warp's 16 inputs
-                    const uint32_t chunk = (uint32_t)(group * 2 + c) ^ (uint32_t)(row0 & 7);
+                for (int c = 0; c < kIn / 8; ++c) {   // 16-byte chunks (8 inputs each)
+                    const uint32_t chunk = (uint32_t)(tgroup * (kIn / 8) + c) ^ (uint32_t)(row0 & 7);
                     const uint4 a = *reinterpret_cast<const uint4*>(p0 + chunk * 16);
                     const uint4 b = *reinterpret_cast<const uint4*>(p1 + chunk * 16);
                     v[8 * c + 0] = __byte_perm(a.x, b.x, 0x5410);
@@ -310,29 +315,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&x_empty[slot]);
-                ptx::tmem_st_32x32b_x16(lane_base + xcol + (uint32_t)(p * 64 + group * 16), v);
+#pragma unroll
+                for (int h = 0; h < kIn / 16; ++h)
+                    ptx::tmem_st_32x32b_x16(lane_base + xcol + (uint32_t)(p * 64 + tgroup * kIn + 16 * h),
+                                            *reinterpret_cast<const uint32_t(*)[16]>(v + 16 * h));
             }
-            ptx::tmem_st_wait();
+        };
+        // The team's stores of the staged chunk complete and become visible to its loads;
+        // its loads issued before are ordered before any later store.
+        auto team_barrier = [&](bool wait_st) {
+            if (wait_st) ptx::tmem_st_wait();
             ptx::tc_fence_before();
-            ptx::named_barrier_sync(2, kSketchWarps * 32);   // the whole chunk is in TMEM
+            ptx::named_barrier_sync(bar_id, kTeamWarps * 32);
             ptx::tc_fence_after();
-            const uint32_t* tab = gather + ((size_t)(tile % NB) * KC + kc) * BK;
-            if (++kc == KC) { kc = 0; tile += gridDim.x; }
-            // the next chunk's table lines are pulled into L1 now, so that its gathers do not
-            // wait for an L2 round trip before they can even form their TMEM addresses
-            if (tile < num_tiles) {
-                const uint32_t* next = gather + ((size_t)(tile % NB) * KC + kc) * BK;
-                for (int sp = 0; sp < NSP; ++sp)
-                    for (int bt = group; bt < F::NBATCH; bt += 4)
-                        if (lane == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(next + (sp * SP + bt * SB) * C));
-            }
-            if (dead) continue;
-            const uint32_t xaddr = lane_base + xcol;
-            // ---- gather: one TMEM load and one bf16x2 FMA per source give both rows' partial sums.
-            // All of this warp's sources of a panel (kPerWarp batches) are in flight before one wait.
-            constexpr int kPerWarp = F::NBATCH / 4 < 2 ? F::NBATCH / 4 : 2;   // batches per load round
-            for (int sp = 0; sp < NSP; ++sp, ++wc) {
-                const int bi = wc % NBS;
+        };
+        // Gather the sketch of chunk g (in TMEM buffer xb) into its B slots: one TMEM load
+        // and one bf16x2 FMA per source give both rows' partial sums. A warp takes the
+        // batches tgroup, tgroup + kGroups, ... of each panel for its 32 lanes; a load round
+        // has kPerWarp batches' sources in flight before one wait.
+        auto gather = [&](int g, int xb, const uint2* tab) {
+            const uint32_t xaddr = lane_base + kAccCols + (uint32_t)(xb * BK);
+            constexpr int kMyBatches = F::NBATCH / kGroups;   // batches of a panel per warp
+            constexpr int kPerWarp = kMyBatches < 2 ? kMyBatches : 2;
+            for (int sp = 0; sp < NSP; ++sp) {
+                const int wc = g * NSP + sp, bi = wc % NBS;
                 if (!warp_wait(&b_empty[bi], ((wc / NBS) & 1) ^ 1, abort_flag)) {
                     dead = true;
                     if (lane == 0) report(status, abort_flag, 6);
@@ -340,20 +346,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 uint8_t* bp = bring + bi * F::B_PANEL;
 #pragma unroll 1
-                for (int bt0 = group; bt0 < F::NBATCH; bt0 += 4 * kPerWarp) {
+                for (int bt0 = tgroup; bt0 < F::NBATCH; bt0 += kGroups * kPerWarp) {
                     uint32_t w[kPerWarp][kBatch], m[kPerWarp][kBatch];
 #pragma unroll
                     for (int u = 0; u < kPerWarp; ++u) {
-                        const int e0 = (sp * SP + (bt0 + 4 * u) * SB) * C;   // first source of batch u
+                        const int e0 = (sp * SP + (bt0 + kGroups * u) * SB) * C;   // first source of batch u
 #pragma unroll
-                        for (int q = 0; q < kBatch / 4; ++q) {
-                            const uint4 e4 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 4 * q));
-                            const uint32_t ee[4] = {e4.x, e4.y, e4.z, e4.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                w[u][4 * q + j] = ptx::tmem_ld_32x32b_x1(xaddr + (ee[j] & 0x1FFu));
-                                m[u][4 * q + j] = (ee[j] & 0x80008000u) | 0x3F803F80u;   // (+-1, +-1)
-                            }
+                        for (int q = 0; q < kBatch / 2; ++q) {   // two {column, multiplier} entries per load
+                            const uint4 e2 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 2 * q));
+                            w[u][2 * q] = ptx::tmem_ld_32x32b_x1(xaddr + e2.x);
+                            m[u][2 * q] = e2.y;
+                            w[u][2 * q + 1] = ptx::tmem_ld_32x32b_x1(xaddr + e2.z);
+                            m[u][2 * q + 1] = e2.w;
                         }
                     }
                     ptx::tmem_ld_wait();
@@ -369,12 +373,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t r0[SB / 2], r1[SB / 2];   // row r and row r + 128, slot pairs
 #pragma unroll
                         for (int i = 0; i < SB / 2; ++i) {
-                            const uint32_t a = *reinterpret_cast<uint32_t*>(&acc[2 * i]);
-                            const uint32_t b = *reinterpret_cast<uint32_t*>(&acc[2 * i + 1]);
-                            r0[i] = __byte_perm(a, b, 0x5410);
-                            r1[i] = __byte_perm(a, b, 0x7632);
+                            const uint32_t x0 = *reinterpret_cast<uint32_t*>(&acc[2 * i]);
+                            const uint32_t x1 = *reinterpret_cast<uint32_t*>(&acc[2 * i + 1]);
+                            r0[i] = __byte_perm(x0, x1, 0x5410);
+                            r1[i] = __byte_perm(x0, x1, 0x7632);
                         }
-                        const int s0 = (bt0 + 4 * u) * SB;   // first slot inside the panel
+                        const int s0 = (bt0 + kGroups * u) * SB;   // first slot inside the panel
                         uint8_t* d0 = bp + kmajor_off<F::RB>(row0, s0);
                         uint8_t* d1 = bp + kmajor_off<F::RB>(row0 + 128, s0);
                         if constexpr (SB == 8) {
@@ -393,6 +397,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&b_full[bi]);
             }
+        };
+        // Table of chunk g; the lines of this team's next chunk are pulled into L1 now, so that
+        // its gathers do not wait for an L2 round trip before they can form TMEM addresses.
+        auto table = [&](int g) -> const uint2* {
+            const int tile = blockIdx.x + (g / KC) * gridDim.x, kc = g % KC;
+            const int gn = g + kTeams, tn = blockIdx.x + (gn / KC) * gridDim.x, kn = gn % KC;
+            if (gn < G) {
+                const uint2* next = gather_tab + ((size_t)(tn % NB) * KC + kn) * BK;
+                for (int sp = 0; sp < NSP; ++sp)
+                    for (int bt = tgroup; bt < F::NBATCH; bt += kGroups)
+                        if (lane == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(next + (sp * SP + bt * SB) * C));
+            }
+            return gather_tab + ((size_t)(tile % NB) * KC + kc) * BK;
+        };
+        for (int g = team; g < G; g += kTeams) {
+            const int xb = kTeams == 2 ? team : 0;
+            stage(g, xb);
+            team_barrier(true);
+            const uint2* tab = table(g);
+            if (!dead) gather(g, xb, tab);
+            team_barrier(false);   // this chunk's loads retire before the buffer is restaged
         }
     } else {
         // ------------------------------------------------------------------ epilogue warps
