@@ -68,7 +68,7 @@ def layer_work(L):
 
 
 KERNEL_SOURCES = {
-    "TC": ["ss1_tc.cu", "ss1_tc2.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
+    "TC": ["ss1_tc.cu", "ss1_tc2.cu", "ss1_tc3.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
     "SMALLM": ["ss1_smallm.cu", "ss1_internal.cuh"],
     "SIMT": ["ss1_simt.cu", "ss1_internal.cuh"],
 }

@@ -27,6 +27,7 @@ void release(ss1_layer* L) {
     if (L->d_g) cudaFree(L->d_g);
     if (L->d_src) cudaFree(L->d_src);
     if (L->d_gather) cudaFree(L->d_gather);
+    if (L->d_slot) cudaFree(L->d_slot);
     if (L->status_host) cudaFreeHost(L->status_host);
     L->magic = 0;
     delete L;
@@ -85,6 +86,7 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
         cudaMalloc(&L->d_g, entries * sizeof(int8_t)) != cudaSuccess ||
         cudaMalloc(&L->d_src, entries * sizeof(uint16_t)) != cudaSuccess ||
         cudaMalloc(&L->d_gather, entries * sizeof(uint2)) != cudaSuccess ||
+        cudaMalloc(&L->d_slot, entries * sizeof(uint16_t)) != cudaSuccess ||
         cudaHostAlloc(&L->status_host, sizeof(int32_t), cudaHostAllocMapped) != cudaSuccess) {
         cudaGetLastError();
         release(L);

@@ -86,12 +86,25 @@ __global__ void gather_table_kernel(const uint16_t* __restrict__ src, uint2* __r
     out[i] = make_uint2((uint32_t)(e & kSrcIdxMask), (e & kSrcNegBit) ? 0xBF80BF80u : 0x3F803F80u);
 }
 
+// One thread per (N-block, input): the input's slot inside its K-chunk and its sign, in the
+// canonical input order -- what the sketch-matrix builder of the tensor-core kernel reads.
+__global__ void slot_table_kernel(const int32_t* __restrict__ h, const int8_t* __restrict__ g, uint16_t* __restrict__ out,
+                                  int64_t n, int K, int BK, int S) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int k = (int)(i % K);
+    const int slot = h[i] - (k / BK) * S;
+    out[i] = (uint16_t)(slot | (g[i] < 0 ? kSrcNegBit : 0));
+}
+
 }  // namespace
 
 cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st) {
     const int64_t nsrc = (int64_t)L.NB * L.K;
     const int threads = 256;
-    gather_table_kernel<<<(unsigned)((nsrc + threads - 1) / threads), threads, 0, st>>>(L.d_src, L.d_gather, nsrc);
+    const unsigned blocks = (unsigned)((nsrc + threads - 1) / threads);
+    gather_table_kernel<<<blocks, threads, 0, st>>>(L.d_src, L.d_gather, nsrc);
+    slot_table_kernel<<<blocks, threads, 0, st>>>(L.d_h, L.d_g, L.d_slot, nsrc, (int)L.K, L.BK, L.S);
     return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ struct ss1_layer {
     int8_t* d_g;         // [NB][K] sign of input k in block nb
     uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
     uint2* d_gather;     // [NB][KC][BK] per source (slot-major): {k, bf16x2 multiplier (+-1, +-1)}
+    uint16_t* d_slot;    // [NB][K] per input: slot inside its chunk (bits 0..7) | kSrcNegBit if the sign is -1
     int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
     int32_t* status_dev;   // device alias of status_host
 };
@@ -52,6 +53,10 @@ bool tc_supported(const ss1_layer& L);
 // Transposed-tile variant (c >= 2): 128 neurons x 256 rows per tile, sketch gathered from TMEM.
 bool tc2_supported(const ss1_layer& L);
 cudaError_t launch_tc2(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
+// Sketch-as-GEMM variant (c >= 2): the sketch of each chunk is a tcgen05.mma with an on-chip
+// 0/+-1 matrix; 128 rows x one or two N-blocks per tile.
+bool tc3_supported(const ss1_layer& L);
+cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 
 }  // namespace ss1

@@ -1,0 +1,601 @@
+// Tensor-core SS1 forward for sm_100a with the sketch itself computed by tcgen05.mma.
+//
+// "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+// "Approach": the input is sketched (signed hashed additions shrink each K-chunk by the
+// compression factor c) and the sketch is multiplied with the compressed weights. Per
+// (N-block nb, K-chunk kc) the sketch is a linear map of the chunk,
+//
+//     Xs_nb[m, s] = sum_k X[m, k] * P_nb,kc[s, k],   P[s, k] = g_nb(k) if slot_nb(k) == s else 0,
+//
+// a 0/+-1 matrix with exactly one non-zero per input k. So the sketch is a small GEMM whose
+// result is exact in the fp32 accumulator (c signed bf16 terms), rounded once to bf16. Both
+// products run on the tensor cores; the CUDA cores only build P and convert the sketch.
+//
+// Tile: 128 rows of X (UMMA M) x Q N-blocks (Q = 2 for most shapes). Per K-chunk:
+//   * X-load warp : X[m0:+128, chunk] as [128 x 64] TMA boxes (128B swizzle) into a ring.
+//   * W-load warp : the Q N-blocks' Wc[nb*128:+128, kc*S:+S] as TMA boxes into a second ring.
+//   * build warp  : writes the Q sketch matrices of the chunk, stacked as the [Q*S x BK] K-major
+//                   B operand, into a ring of zeroed panels: only the BK*Q non-zeros are written,
+//                   and cleared again before a panel is reused. Its table entries arrive through
+//                   a cp.async ring several units ahead. Once a segment's panels are written and
+//                   its X boxes have landed it raises sk_ready.
+//   * MMA warp    : sketch  D_s[128 rows x Q*S] (fp32, TMEM) = X_chunk * P^T  (BK/16 UMMAs)
+//                   main    D_j[128 rows x 128] += Xs_j (A operand from TMEM) * Wc_j^T  (S/16 UMMAs
+//                   per N-block j). The sketch of chunk i+1 is issued before the main product of
+//                   chunk i, so the tensor pipe stays busy while chunk i is converted. This warp
+//                   waits on two kinds of barrier only (sk_ready, mm_ready): an mbarrier wait
+//                   costs about as much as two N = 128 UMMAs and the tensor pipe's queue is
+//                   short, so every wait in the issuing thread is a bubble in the pipe.
+//   * 8 convert warps (two per TMEM lane quarter, one per half of the sketch columns): fp32 ->
+//                   bf16 in place in TMEM (the A-operand layout: lane = row, two consecutive slots
+//                   per 32-bit column). D_s is double-buffered. The first convert warp also waits
+//                   for the chunk's Wc (and for the accumulator at a tile's first chunk) and then
+//                   all eight raise mm_ready.
+//   * 4 epilogue warps: accumulators -> bf16 (round to nearest even) -> swizzled shared-memory
+//                   staging -> TMA bulk stores of [32 rows x 32 neurons] boxes (rows past M are
+//                   clipped by the tensor map).
+// Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
+// handle's status word, drains the copies and MMAs in flight and returns (no trap).
+#include "ss1_internal.cuh"
+#include "ptx_sm100.cuh"
+
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace ss1 {
+
+// defined in ss1_tc.cu (tensor-map encoding through the driver entry point)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+namespace {
+
+constexpr int kRows = 128;                 // rows of X per tile (UMMA M)
+constexpr int kNeu = 128;                  // neurons per N-block (UMMA N of the main product)
+constexpr int kUnitK = 64;                 // inputs per X box / sketch panel (one 128-byte swizzle row)
+constexpr int kXUnit = kRows * 128;        // bytes of one X box [128 rows x 64 inputs]
+constexpr int kWarpLoadX = 0, kWarpMma = 1, kWarpBuild = 2, kWarpLoadW = 3, kFirstConv = 4, kConvWarps = 8;
+constexpr int kFirstEpi = kFirstConv + kConvWarps, kEpiWarps = 4;
+constexpr int kWarps = kFirstEpi + kEpiWarps;
+constexpr int kThreads = kWarps * 32;
+constexpr int kEpiBox = 32 * 32 * 2;       // one [32 rows x 32 neurons] bf16 store box
+constexpr int kTabUnits = 8;               // table staging ring of the build warp (units)
+constexpr int kSmemBudget = 225 * 1024;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint16_t kBf16One = 0x3F80u, kBf16MinusOne = 0xBF80u;
+
+template <int BK, int C, int Q>
+struct Cfg {
+    static constexpr int S = BK / C;
+    static constexpr int QS = Q * S;                     // N of the sketch UMMA
+    static constexpr int HW = QS / 2;                    // sketch columns per convert warp
+    static constexpr int U = BK / kUnitK;                // X boxes / sketch panels per chunk
+    static constexpr int SU = U < 2 ? U : 2;             // units per sketch segment (one sk_ready)
+    static constexpr int NSEG = U / SU;                  // segments per chunk
+    static constexpr int P_UNIT = QS * 128;              // bytes of one sketch panel [QS x 64]
+    static constexpr int RB = S >= 64 ? 128 : 2 * S;     // Wc operand: bytes per row of a panel
+    static constexpr uint32_t WLAYOUT = S >= 64 ? ptx::kLayoutSW128 : (S == 32 ? ptx::kLayoutSW64 : ptx::kLayoutSW32);
+    static constexpr int WSBO = 8 * RB;
+    static constexpr int W_PANEL = kNeu * RB;            // bytes of one Wc panel
+    static constexpr int W_NB = kNeu * S * 2;            // one N-block's Wc chunk
+    static constexpr int W_STAGE = Q * W_NB;
+    static constexpr int NP = 2 * SU;                    // sketch panels: two segments
+    static constexpr int NW = 2;
+    static constexpr int NE = 2 * Q;                     // sketch-matrix entries per lane and unit
+    static constexpr int TAB_UNIT = Q * kUnitK * 2;      // bytes of one unit's table entries
+    static constexpr int EPI = kEpiWarps * 2 * kEpiBox;
+    static constexpr int CLR = ((NP * NE * 32 * 2 + 15) / 16) * 16;
+    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + kTabUnits * TAB_UNIT + CLR;
+    static constexpr int NX_FIT = (kSmemBudget - FIXED) / kXUnit;
+    static constexpr int NX = NX_FIT < 2 * U + 1 ? NX_FIT : 2 * U + 1;
+    // TMEM columns: Q accumulators (x NACC buffers), then two sketch buffers
+    static constexpr int ACC_COLS = Q * kNeu;
+    static constexpr int NACC = (2 * ACC_COLS + 2 * QS <= 512) ? 2 : 1;
+    static constexpr int DS_COL = NACC * ACC_COLS;
+    // shared memory (the swizzled buffers first, each a multiple of 1 KB)
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_P = OFF_X + NX * kXUnit;
+    static constexpr int OFF_W = OFF_P + NP * P_UNIT;
+    static constexpr int OFF_E = OFF_W + NW * W_STAGE;
+    static constexpr int OFF_TAB = OFF_E + EPI;
+    static constexpr int OFF_CLR = OFF_TAB + kTabUnits * TAB_UNIT;
+    static constexpr int OFF_BAR = OFF_CLR + CLR;
+    static constexpr int NBAR = 2 * NX + NP + 2 + 2 * NW + 2 + 2 + 2 * NACC + 1;
+    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static_assert(BK % kUnitK == 0 && BK <= 256 && U % SU == 0, "chunks of whole 64-input units");
+    static_assert(S % 16 == 0 && S >= 16 && S <= 128, "UMMA K-steps of 16 over the slots");
+    static_assert(QS % 32 == 0 && QS <= 256 && HW % 16 == 0, "sketch UMMA N and conversion halves");
+    static_assert(DS_COL + 2 * QS <= 512, "TMEM budget");
+    static_assert(NX >= 2 * SU && SMEM <= 227 * 1024, "shared memory budget: X ring holds two segments");
+    static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+__device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
+    *abort_flag = 1;
+    *(volatile int32_t*)status = (kStatusKernelTC << 8) | (0x80 + site);
+    __threadfence_system();
+}
+
+// Lane 0 waits, the warp follows: one poller per warp instead of 32.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, kWaitNs);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Slot and phase of a ring position, advanced without divisions.
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    int n;
+    __device__ explicit Ring(int n_) : n(n_) {}
+    __device__ __forceinline__ void next() {
+        if (++slot == n) { slot = 0; phase ^= 1u; }
+    }
+};
+
+// Waits for the last `depth` completions of a ring of `n` full-barriers after `issued` fills
+// (used only to drain copies in flight after an abort).
+__device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, int depth) {
+    volatile int no_abort = 0;
+    for (int i = (issued - depth > 0 ? issued - depth : 0); i < issued; ++i)
+        ptx::mbar_wait(&full[i % n], (uint32_t)((i / n) & 1), &no_abort, kWaitNs);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(lo_f32), __uint_as_float(hi_f32));
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Byte offset of element (row, kl) of a K-major [rows x 64] panel with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_off(int row, int kl) {
+    return (uint32_t)(row * 128) + ((uint32_t)((kl >> 3) ^ (row & 7)) << 4) + (uint32_t)(kl & 7) * 2u;
+}
+
+template <int BK, int C, int Q>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc3_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               const __grid_constant__ CUtensorMap tmap_y, const uint16_t* __restrict__ slot_tab, int K, int KC, int NG,
+               int num_tiles, int32_t* status) {
+    using F = Cfg<BK, C, Q>;
+    constexpr int S = F::S, QS = F::QS, HW = F::HW, U = F::U, SU = F::SU, NSEG = F::NSEG;
+    constexpr int NX = F::NX, NP = F::NP, NW = F::NW, NACC = F::NACC;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* xring = smem + F::OFF_X;
+    uint8_t* pring = smem + F::OFF_P;
+    uint8_t* wring = smem + F::OFF_W;
+    uint8_t* estage = smem + F::OFF_E;
+    uint16_t* tab = reinterpret_cast<uint16_t*>(smem + F::OFF_TAB);
+    uint16_t* clr = reinterpret_cast<uint16_t*>(smem + F::OFF_CLR);
+    uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
+    uint64_t* x_empty = x_full + NX;
+    uint64_t* p_empty = x_empty + NX;
+    uint64_t* sk_ready = p_empty + NP;    // [2] panels + X boxes of a sketch segment ready
+    uint64_t* w_full = sk_ready + 2;
+    uint64_t* w_empty = w_full + NW;
+    uint64_t* s_full = w_empty + NW;      // [2] sketch product of a chunk is in D_s[b]
+    uint64_t* mm_ready = s_full + 2;      // [2] D_s[b] in bf16, Wc (and the accumulator) ready
+    uint64_t* acc_full = mm_ready + 2;    // [NACC]
+    uint64_t* acc_empty = acc_full + NACC;
+    uint64_t* drain = acc_empty + NACC;   // abort path: completion of every issued MMA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int G = my_tiles * KC;   // chunks this CTA processes
+
+    // the sketch panels start zeroed; only their non-zeros are ever written afterwards
+    for (int i = threadIdx.x; i < NP * F::P_UNIT / 16; i += kThreads)
+        reinterpret_cast<uint4*>(pring)[i] = make_uint4(0u, 0u, 0u, 0u);
+    ptx::fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < NP; ++i) ptx::mbar_init(&p_empty[i], 1);
+        for (int i = 0; i < NW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&sk_ready[i], 1);
+            ptx::mbar_init(&s_full[i], 1);
+            ptx::mbar_init(&mm_ready[i], kConvWarps);
+        }
+        for (int i = 0; i < NACC; ++i) { ptx::mbar_init(&acc_full[i], 1); ptx::mbar_init(&acc_empty[i], kEpiWarps); }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    if (warp == kWarpLoadX && lane == 0) ptx::prefetch_tmap(&tmap_x);
+    if (warp == kWarpLoadW && lane == 0) ptx::prefetch_tmap(&tmap_w);
+    if (warp == kFirstEpi && lane == 0) ptx::prefetch_tmap(&tmap_y);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    if (warp == kWarpLoadX) {
+        // ------------------------------------------------------------------ TMA loads of X
+        if (lane == 0) {
+            Ring xr(NX);
+            int nx = 0;
+            bool ok = true;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                const int m0 = (((int)blockIdx.x + t * (int)gridDim.x) / NG) * kRows;
+                for (int kc = 0; kc < KC && ok; ++kc)
+                    for (int u = 0; u < U; ++u) {
+                        if (!ptx::mbar_wait(&x_empty[xr.slot], xr.phase ^ 1u, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 1); break; }
+                        ptx::mbar_arrive_expect_tx(&x_full[xr.slot], kXUnit);
+                        ptx::tma_load_2d(xring + xr.slot * kXUnit, &tmap_x, &x_full[xr.slot], kc * BK + u * kUnitK, m0);
+                        xr.next();
+                        ++nx;
+                    }
+            }
+            if (*abort_flag) drain_ring(x_full, NX, nx, NX);   // every issued copy lands before exit
+        }
+    } else if (warp == kWarpLoadW) {
+        // ------------------------------------------------------------------ TMA loads of Wc
+        if (lane == 0) {
+            Ring wr(NW);
+            int nw = 0;
+            bool ok = true;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                const int nb0 = (((int)blockIdx.x + t * (int)gridDim.x) % NG) * Q;
+                for (int kc = 0; kc < KC && ok; ++kc) {
+                    if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 2); break; }
+                    ptx::mbar_arrive_expect_tx(&w_full[wr.slot], F::W_STAGE);
+                    uint8_t* wdst = wring + wr.slot * F::W_STAGE;
+#pragma unroll
+                    for (int j = 0; j < Q; ++j)
+#pragma unroll
+                        for (int p = 0; p < (S + 63) / 64; ++p)
+                            ptx::tma_load_2d(wdst + j * F::W_NB + p * F::W_PANEL, &tmap_w, &w_full[wr.slot], kc * S + p * 64,
+                                             (nb0 + j) * kNeu);
+                    wr.next();
+                    ++nw;
+                }
+            }
+            if (*abort_flag) drain_ring(w_full, NW, nw, NW);
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------------------ MMA issue
+        // The whole warp walks the schedule (waits are warp-wide); lane 0 issues.
+        constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, QS);
+        constexpr uint32_t idesc_m = ptx::idesc_bf16_f32(kRows, kNeu);
+        const uint64_t xdesc0 = ptx::smem_desc(ptx::smem_u32(xring), 16, 1024, ptx::kLayoutSW128);
+        const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(pring), 16, 1024, ptx::kLayoutSW128);
+        const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, F::WSBO, F::WLAYOUT);
+        const bool leader = lane == 0;
+        Ring xr(NX), pr(NP), wr(NW);
+        int seg = 0;
+        bool ok = true;
+        // sketch of chunk i into D_s[i & 1], one sk_ready wait per segment of SU units
+        auto sketch = [&](int i) {
+            const uint32_t ds = tm + (uint32_t)(F::DS_COL + (i & 1) * QS);
+            for (int sg = 0; sg < NSEG; ++sg, ++seg) {
+                if (!warp_wait(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag)) {
+                    ok = false;
+                    if (leader) report(status, abort_flag, 3);
+                    return;
+                }
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int su = 0; su < SU; ++su) {
+                    if (leader) {
+                        const uint64_t xd = xdesc0 + (uint64_t)((xr.slot * kXUnit) >> 4);
+                        const uint64_t pd = pdesc0 + (uint64_t)((pr.slot * F::P_UNIT) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < kUnitK / 16; ++kk)
+                            ptx::umma_bf16_ss(ds, xd + (uint64_t)(kk * 2), pd + (uint64_t)(kk * 2), idesc_s,
+                                              (sg > 0 || su > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_commit(&x_empty[xr.slot]);
+                        ptx::umma_commit(&p_empty[pr.slot]);
+                    }
+                    xr.next();
+                    pr.next();
+                }
+            }
+            if (leader) ptx::umma_commit(&s_full[i & 1]);
+            __syncwarp();
+        };
+        // main product of chunk i (kc of tile t): D_j += Xs_j * Wc_j^T
+        auto main_mma = [&](int i, int t, int kc) {
+            const int b = i & 1, a = NACC == 2 ? (t & 1) : 0;
+            if (!warp_wait(&mm_ready[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
+                ok = false;
+                if (leader) report(status, abort_flag, 4);
+                return;
+            }
+            ptx::tc_fence_after();
+            if (leader) {
+                const uint32_t xs = tm + (uint32_t)(F::DS_COL + b * QS);
+                const uint64_t wd = wdesc0 + (uint64_t)((wr.slot * F::W_STAGE) >> 4);
+#pragma unroll
+                for (int j = 0; j < Q; ++j)
+#pragma unroll
+                    for (int kk = 0; kk < S / 16; ++kk) {
+                        constexpr int per_panel = F::RB / 2;   // slots per Wc panel row
+                        const uint32_t off = (uint32_t)(j * F::W_NB + ((kk * 16) / per_panel) * F::W_PANEL +
+                                                        ((kk * 16) % per_panel) * 2);
+                        // slots s0 .. s0+15 in bf16: converted in place inside their half's columns
+                        const int s0 = j * S + kk * 16;
+                        const uint32_t acol = (uint32_t)((s0 / HW) * HW + (s0 % HW) / 2);
+                        ptx::umma_bf16_ts(tm + (uint32_t)(a * F::ACC_COLS + j * kNeu), xs + acol, wd + (uint64_t)(off >> 4),
+                                          idesc_m, (kc > 0 || kk > 0) ? 1u : 0u);
+                    }
+                ptx::umma_commit(&w_empty[wr.slot]);
+                if (kc == KC - 1) ptx::umma_commit(&acc_full[a]);
+            }
+            __syncwarp();
+            wr.next();
+        };
+        if (G > 0) sketch(0);
+        int t = 0, kc = 0;
+        for (int i = 0; i < G && ok; ++i) {
+            if (i + 1 < G) sketch(i + 1);
+            if (!ok) break;
+            main_mma(i, t, kc);
+            if (++kc == KC) { kc = 0; ++t; }
+        }
+        if (*abort_flag && leader) {   // MMAs in flight finish before TMEM is released
+            volatile int no_abort = 0;
+            ptx::umma_commit(drain);
+            ptx::mbar_wait(drain, 0, &no_abort, kWaitNs);
+        }
+        __syncwarp();
+    } else if (warp == kWarpBuild) {
+        // ------------------------------------------------------------------ sketch matrices
+        // Panel u of chunk kc for the tile's N-blocks nb0 .. nb0+Q-1: entry (j*S + slot(k), k)
+        // = sign(k) for the 64 inputs k of the unit; every other entry stays zero. A lane writes
+        // inputs lane and lane + 32 of each N-block and records where, so that the entries can
+        // be cleared when the panel comes round again. The unit's table entries (Q lines of
+        // 128 bytes) were copied into a staging ring kTabUnits - 1 units earlier.
+        const int units = G * U;
+        auto unit_src = [&](int pu) -> const uint16_t* {   // table entries of unit pu, N-block nb0
+            const int i = pu / U, u = pu % U;
+            const int tile = (int)blockIdx.x + (i / KC) * (int)gridDim.x, kc = i % KC;
+            return slot_tab + (size_t)((tile % NG) * Q) * K + (size_t)kc * BK + u * kUnitK;
+        };
+        auto stage_unit = [&](int pu) {   // lanes 0 .. 8Q-1 copy 16 bytes each; always one group
+            if (pu < units && lane < 8 * Q) {
+                const int j = lane >> 3, part = lane & 7;
+                ptx::cp_async_ca_16(tab + (pu % kTabUnits) * (Q * kUnitK) + j * kUnitK + part * 8,
+                                    unit_src(pu) + (size_t)j * K + part * 8);
+            }
+            ptx::cp_async_commit();
+        };
+        for (int pu = 0; pu < kTabUnits - 1; ++pu) stage_unit(pu);
+        Ring pr(NP), xr(NX);
+        int pu = 0;
+        bool ok = true;
+        for (int g = 0; g < G * NSEG && ok; ++g) {
+            for (int su = 0; su < SU; ++su, ++pu) {
+                stage_unit(pu + kTabUnits - 1);
+                ptx::cp_async_wait<kTabUnits - 1>();   // unit pu's group has landed
+                __syncwarp();
+                const uint16_t* te = tab + (pu % kTabUnits) * (Q * kUnitK);
+                uint16_t e[F::NE];
+#pragma unroll
+                for (int j = 0; j < Q; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) e[2 * j + h] = te[j * kUnitK + lane + 32 * h];
+                if (!warp_wait(&p_empty[pr.slot], pr.phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    if (lane == 0) report(status, abort_flag, 5);
+                    break;
+                }
+                uint8_t* panel = pring + pr.slot * F::P_UNIT;
+                uint16_t* rec = clr + pr.slot * (F::NE * 32) + lane;
+                if (pu >= NP) {   // clear the non-zeros this panel held NP units ago
+#pragma unroll
+                    for (int x = 0; x < F::NE; ++x) *reinterpret_cast<uint16_t*>(panel + rec[32 * x]) = 0;
+                }
+#pragma unroll
+                for (int j = 0; j < Q; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint16_t en = e[2 * j + h];
+                        const uint32_t off = sw128_off(j * S + (en & kSrcIdxMask), lane + 32 * h);
+                        *reinterpret_cast<uint16_t*>(panel + off) = (en & kSrcNegBit) ? kBf16MinusOne : kBf16One;
+                        rec[32 * (2 * j + h)] = (uint16_t)off;
+                    }
+                pr.next();
+            }
+            if (!ok) break;
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            for (int su = 0; su < SU; ++su) {   // the segment's X boxes have landed
+                if (!warp_wait(&x_full[xr.slot], xr.phase, abort_flag)) {
+                    ok = false;
+                    if (lane == 0) report(status, abort_flag, 8);
+                    break;
+                }
+                xr.next();
+            }
+            if (!ok) break;
+            if (lane == 0) ptx::mbar_arrive(&sk_ready[g & 1]);
+        }
+        ptx::cp_async_wait<0>();
+    } else if (warp >= kFirstConv && warp < kFirstConv + kConvWarps) {
+        // ------------------------------------------------------------------ sketch conversion
+        // Warp (quarter, half) converts fp32 sketch columns [half*HW, half*HW + HW) of its 32
+        // lanes to bf16 pairs written to columns [half*HW, half*HW + HW/2): all of its loads
+        // complete before the first store, and no other warp reads these columns.
+        const int quad = warp & 3, half = (warp - kFirstConv) >> 2;
+        const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)(F::DS_COL + half * HW);
+        Ring wr(NW);
+        int t = 0, kc = 0;
+        for (int i = 0; i < G; ++i) {
+            const int b = i & 1;
+            if (!warp_wait(&s_full[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 6);
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t base = lane_base + (uint32_t)(b * QS);
+            uint32_t r[HW];
+#pragma unroll
+            for (int c0 = 0; c0 < HW; c0 += 16) ptx::tmem_ld_32x32b_x16(base + (uint32_t)c0, r + c0);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int p = 0; p < HW / 2; ++p) r[p] = pack_bf16x2(r[2 * p], r[2 * p + 1]);
+#pragma unroll
+            for (int c0 = 0; c0 < HW / 2; c0 += 8) ptx::tmem_st_32x32b_x8(base + (uint32_t)c0, r + c0);
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            // the first convert warp also waits for the chunk's Wc and, at a tile's first
+            // chunk, for the epilogue to have read the accumulator
+            if (warp == kFirstConv) {
+                const int a = NACC == 2 ? (t & 1) : 0;
+                if (!warp_wait(&w_full[wr.slot], wr.phase, abort_flag) ||
+                    (kc == 0 && !warp_wait(&acc_empty[a], (uint32_t)(((t / NACC) & 1) ^ 1), abort_flag))) {
+                    if (lane == 0) report(status, abort_flag, 9);
+                    break;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&mm_ready[b]);
+            wr.next();
+            if (++kc == KC) { kc = 0; ++t; }
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        // Warp `quad` owns rows [32 quad, 32 quad + 32) of the tile. Per [32 x 32] block: two
+        // blocks' TMEM loads in flight, bf16 rounding, a swizzled (64-byte) staging box, one TMA
+        // store; two staging boxes alternate so that a store's read overlaps the next block.
+        const int quad = warp & 3;
+        uint8_t* stg = estage + (warp - kFirstEpi) * 2 * kEpiBox;
+        const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16);
+        int nst = 0;
+        for (int t = 0; t < my_tiles; ++t) {
+            const int tile = (int)blockIdx.x + t * (int)gridDim.x;
+            const int a = NACC == 2 ? (t & 1) : 0;
+            if (!warp_wait(&acc_full[a], (uint32_t)((t / NACC) & 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 7);
+                break;
+            }
+            ptx::tc_fence_after();
+            const int row0 = (tile / NG) * kRows + quad * 32;
+            const int col0 = (tile % NG) * Q * kNeu;
+            auto store_block = [&](int q, const uint32_t (&r)[32]) {
+                uint8_t* box = stg + (nst & 1) * kEpiBox;
+                if (lane == 0) ptx::tma_store_wait_read1();   // the store two blocks ago has read `box`
+                __syncwarp();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)
+                    *reinterpret_cast<uint4*>(box + lane * 64 + ((ch ^ ((lane >> 1) & 3)) << 4)) =
+                        make_uint4(pack_bf16x2(r[8 * ch + 0], r[8 * ch + 1]), pack_bf16x2(r[8 * ch + 2], r[8 * ch + 3]),
+                                   pack_bf16x2(r[8 * ch + 4], r[8 * ch + 5]), pack_bf16x2(r[8 * ch + 6], r[8 * ch + 7]));
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::tma_store_2d(&tmap_y, box, col0 + q * 32, row0);
+                    ptx::tma_store_commit();
+                }
+                ++nst;
+            };
+#pragma unroll 1
+            for (int q = 0; q < 4 * Q; q += 2) {
+                uint32_t ra[32], rb[32];
+                ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32), ra);
+                ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32 + 32), rb);
+                ptx::tmem_ld_wait();
+                if (q + 2 == 4 * Q) {   // accumulator read: the next tile's MMAs may start
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[a]);
+                }
+                store_block(q, ra);
+                store_block(q + 1, rb);
+            }
+        }
+        if (lane == 0) ptx::tma_store_wait0();
+        __syncwarp();
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tm, 512);
+    }
+}
+
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle sw) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BK, int C, int Q>
+cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    using F = Cfg<BK, C, Q>;
+    constexpr int S = F::S;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(tc3_kernel<BK, C, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mx, mw, my;
+    const CUtensorMapSwizzle wsw = S >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (S == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    if (!make_map(&mx, X, (uint64_t)L.K, (uint64_t)M, kUnitK, kRows, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+    if (!make_map(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kNeu, wsw)) return cudaErrorInvalidValue;
+    if (!make_map(&my, Y, (uint64_t)L.N, (uint64_t)M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
+    const int NG = L.NB / Q;
+    const int64_t tiles = (M + kRows - 1) / kRows * NG;
+    const int grid = (int)(tiles < L.num_sms ? tiles : L.num_sms);
+    tc3_kernel<BK, C, Q><<<grid, kThreads, F::SMEM, st>>>(mx, mw, my, L.d_slot, (int)L.K, L.KC, NG, (int)tiles,
+                                                          L.status_dev);
+    return cudaGetLastError();
+}
+
+// N-blocks per tile: two where the N-blocks pair up (the sketch UMMA then has N = 2 S), one
+// for S = 128 (already N = 128) or an odd count of N-blocks.
+int pick_q(const ss1_layer& L) {
+    if (L.S == 128) return 1;
+    return L.NB % 2 == 0 ? 2 : 1;
+}
+
+}  // namespace
+
+bool tc3_supported(const ss1_layer& L) {
+    if (L.BN != kNeu || L.c < 2) return false;
+    if (!(L.BK == 128 || L.BK == 256)) return false;
+    if (!(L.S == 16 || L.S == 32 || L.S == 64 || L.S == 128)) return false;
+    if ((pick_q(L) * L.S) % 32 != 0) return false;
+    if (L.K % 8 != 0 || (L.K / L.c) % 8 != 0 || L.N % 8 != 0) return false;
+    return true;
+}
+
+cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if ((M + kRows - 1) / kRows * L.NB > (int64_t)1 << 30) return cudaErrorInvalidValue;
+    const int q = pick_q(L);
+#define SS1_TC3_CASE(bk, cc, qq) \
+    if (L.BK == bk && L.c == cc && q == qq) return launch_cfg<bk, cc, qq>(L, X, Wc, Y, M, st);
+    SS1_TC3_CASE(128, 2, 2)
+    SS1_TC3_CASE(128, 2, 1)
+    SS1_TC3_CASE(128, 4, 2)
+    SS1_TC3_CASE(128, 4, 1)
+    SS1_TC3_CASE(128, 8, 2)
+    SS1_TC3_CASE(256, 2, 1)
+    SS1_TC3_CASE(256, 4, 2)
+    SS1_TC3_CASE(256, 4, 1)
+    SS1_TC3_CASE(256, 8, 2)
+    SS1_TC3_CASE(256, 8, 1)
+#undef SS1_TC3_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ss1

@@ -26,7 +26,7 @@ def _layer(ss1, K=512, N=256, c=4, BK=128, BN=128, seed=3):
 
 
 @pytest.mark.parametrize("kernel", BF16_KERNELS)
-@pytest.mark.parametrize("c,BK", [(1, 128), (2, 128), (4, 128), (8, 256), (2, 256)])
+@pytest.mark.parametrize("c,BK", [(1, 128), (2, 128), (4, 128), (8, 128), (8, 256), (2, 256)])
 def test_one_hot_probe_bit_exact(kernel, c, BK):
     """X = I_K: every output is one product g * Wc (exact in bf16), so Y must equal the tied
     weight bit for bit. Pins the hash indexing and signs inside the kernel."""

@@ -30,6 +30,11 @@ def _small_cases():
             for M in (1, 16, 200, 333):
                 cases.append(Layer("bf16-small", M, 1024, 384, c, BK, 128, "bf16", "normal", "normal_002", 3))
     cases.append(Layer("bf16-small", 257, 1280, 640, 4, 128, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2))
+    # an even count of N-blocks: the tensor-core kernel pairs N-blocks in one tile (every c, both BK)
+    for c in (2, 4, 8):
+        for BK in (128, 256):
+            for M in (130, 333):
+                cases.append(Layer("bf16-small", M, 768, 768, c, BK, 128, "bf16", "normal", "uniform_invsqrtk", 8))
     # decode-sized rows: every row-group width, ragged groups, narrow N-blocks, K past one segment
     for M in (2, 3, 5, 8, 9, 37, 64):
         cases.append(Layer("bf16-small", M, 3072, 320, 2, 128, 64, "bf16", "normal", "normal_002", 4))
