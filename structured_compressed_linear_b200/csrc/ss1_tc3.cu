@@ -55,9 +55,10 @@ constexpr int kRows = 128;                 // rows of X per tile (UMMA M)
 constexpr int kNeu = 128;                  // neurons per N-block (UMMA N of the main product)
 constexpr int kUnitK = 64;                 // inputs per X box / sketch panel (one 128-byte swizzle row)
 constexpr int kXUnit = kRows * 128;        // bytes of one X box [128 rows x 64 inputs]
-constexpr int kWarpLoadX = 0, kWarpMma = 1, kWarpBuild = 2, kWarpLoadW = 3, kFirstConv = 4, kConvWarps = 8;
+constexpr int kWarpLoadX = 0, kWarpSketch = 1, kWarpBuild = 2, kWarpLoadW = 3, kFirstConv = 4, kConvWarps = 8;
 constexpr int kFirstEpi = kFirstConv + kConvWarps, kEpiWarps = 4;
-constexpr int kWarps = kFirstEpi + kEpiWarps;
+constexpr int kWarpMain = kFirstEpi + kEpiWarps;
+constexpr int kWarps = kWarpMain + 1;
 constexpr int kThreads = kWarps * 32;
 constexpr int kEpiBox = 32 * 32 * 2;       // one [32 rows x 32 neurons] bf16 store box
 constexpr int kTabUnits = 8;               // table staging ring of the build warp (units)
@@ -85,14 +86,16 @@ struct Cfg {
     static constexpr int NE = 2 * Q;                     // sketch-matrix entries per lane and unit
     static constexpr int TAB_UNIT = Q * kUnitK * 2;      // bytes of one unit's table entries
     static constexpr int EPI = kEpiWarps * 2 * kEpiBox;
-    static constexpr int CLR = ((NP * NE * 32 * 2 + 15) / 16) * 16;
+    static constexpr int CLR = 0;
     static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + kTabUnits * TAB_UNIT + CLR;
     static constexpr int NX_FIT = (kSmemBudget - FIXED) / kXUnit;
     static constexpr int NX = NX_FIT < 2 * U + 1 ? NX_FIT : 2 * U + 1;
-    // TMEM columns: Q accumulators (x NACC buffers), then two sketch buffers
+    // TMEM columns: Q accumulators (x NACC buffers), the fp32 sketch D_s (QS columns), then two
+    // bf16 sketch buffers Xs (QS / 2 columns each: two slots per column)
     static constexpr int ACC_COLS = Q * kNeu;
     static constexpr int NACC = (2 * ACC_COLS + 2 * QS <= 512) ? 2 : 1;
     static constexpr int DS_COL = NACC * ACC_COLS;
+    static constexpr int XS_COL = DS_COL + QS;
     // shared memory (the swizzled buffers first, each a multiple of 1 KB)
     static constexpr int OFF_X = 0;
     static constexpr int OFF_P = OFF_X + NX * kXUnit;
@@ -101,7 +104,7 @@ struct Cfg {
     static constexpr int OFF_TAB = OFF_E + EPI;
     static constexpr int OFF_CLR = OFF_TAB + kTabUnits * TAB_UNIT;
     static constexpr int OFF_BAR = OFF_CLR + CLR;
-    static constexpr int NBAR = 2 * NX + NP + 2 + 2 * NW + 2 + 2 + 2 * NACC + 1;
+    static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 1 + 2 + 2 * NACC + 2;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(BK % kUnitK == 0 && BK <= 256 && U % SU == 0, "chunks of whole 64-input units");
     static_assert(S % 16 == 0 && S >= 16 && S <= 128, "UMMA K-steps of 16 over the slots");
@@ -122,6 +125,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, kWaitNs);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Wait of an MMA-issuing warp: every lane polls the barrier without suspending (one shared-memory
+// broadcast per poll), so the issue resumes as soon as the phase completes.
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+    bool ok = ptx::mbar_test(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = ptx::globaltimer_ns();
+        for (uint32_t n = 1;; ++n) {
+            if (ptx::mbar_test(bar, parity)) { ok = true; break; }
+            if ((n & 63) == 0 && (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitNs)) break;
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
 }
 
 // Slot and phase of a ring position, advanced without divisions.
@@ -168,19 +185,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* wring = smem + F::OFF_W;
     uint8_t* estage = smem + F::OFF_E;
     uint16_t* tab = reinterpret_cast<uint16_t*>(smem + F::OFF_TAB);
-    uint16_t* clr = reinterpret_cast<uint16_t*>(smem + F::OFF_CLR);
+    // One tcgen05.commit per sketch segment (seg_done) tells every consumer at once: the X
+    // loader and the build warp that the segment's X boxes and panels are free, the convert
+    // warps (at a chunk's last segment) that the sketch is in D_s. Commits from the issuing
+    // thread are kept few because each one costs about as much as a short UMMA.
     uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
-    uint64_t* x_empty = x_full + NX;
-    uint64_t* p_empty = x_empty + NX;
-    uint64_t* sk_ready = p_empty + NP;    // [2] panels + X boxes of a sketch segment ready
+    uint64_t* seg_done = x_full + NX;     // [4] sketch segment g completed (g % 4)
+    uint64_t* sk_ready = seg_done + 4;    // [2] panels + X boxes of a sketch segment ready
     uint64_t* w_full = sk_ready + 2;
     uint64_t* w_empty = w_full + NW;
-    uint64_t* s_full = w_empty + NW;      // [2] sketch product of a chunk is in D_s[b]
-    uint64_t* mm_ready = s_full + 2;      // [2] D_s[b] in bf16, Wc (and the accumulator) ready
-    uint64_t* acc_full = mm_ready + 2;    // [NACC]
+    uint64_t* mm_ready = w_empty + NW;    // [2] Xs[b] written, Wc (and the accumulator) ready
+    uint64_t* ds_free = mm_ready + 2;     // the convert warps have read D_s
+    uint64_t* main_done = ds_free + 1;    // [2] main product of a chunk done reading Xs[b]
+    uint64_t* acc_full = main_done + 2;   // [NACC]
     uint64_t* acc_empty = acc_full + NACC;
-    uint64_t* drain = acc_empty + NACC;   // abort path: completion of every issued MMA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* drain = acc_empty + NACC;   // [2] abort path: completion of every MMA a warp issued
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -192,20 +212,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<uint4*>(pring)[i] = make_uint4(0u, 0u, 0u, 0u);
     ptx::fence_proxy_async_smem();
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 1); }
-        for (int i = 0; i < NP; ++i) ptx::mbar_init(&p_empty[i], 1);
+        for (int i = 0; i < NX; ++i) ptx::mbar_init(&x_full[i], 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&seg_done[i], 1);
         for (int i = 0; i < NW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&sk_ready[i], 1);
-            ptx::mbar_init(&s_full[i], 1);
             ptx::mbar_init(&mm_ready[i], kConvWarps);
+            ptx::mbar_init(&main_done[i], 1);
+            ptx::mbar_init(&drain[i], 1);
         }
+        ptx::mbar_init(ds_free, kConvWarps);
         for (int i = 0; i < NACC; ++i) { ptx::mbar_init(&acc_full[i], 1); ptx::mbar_init(&acc_empty[i], kEpiWarps); }
-        ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == kWarpMma) {
+    if (warp == kWarpSketch) {
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
@@ -227,7 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m0 = (((int)blockIdx.x + t * (int)gridDim.x) / NG) * kRows;
                 for (int kc = 0; kc < KC && ok; ++kc)
                     for (int u = 0; u < U; ++u) {
-                        if (!ptx::mbar_wait(&x_empty[xr.slot], xr.phase ^ 1u, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 1); break; }
+                        if (nx >= NX) {   // the slot's previous unit belongs to segment gp
+                            const int gp = (nx - NX) / SU;
+                            if (!ptx::mbar_wait(&seg_done[gp & 3], (uint32_t)((gp >> 2) & 1), abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 1); break; }
+                        }
                         ptx::mbar_arrive_expect_tx(&x_full[xr.slot], kXUnit);
                         ptx::tma_load_2d(xring + xr.slot * kXUnit, &tmap_x, &x_full[xr.slot], kc * BK + u * kUnitK, m0);
                         xr.next();
@@ -260,59 +284,74 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (*abort_flag) drain_ring(w_full, NW, nw, NW);
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------------ MMA issue
-        // The whole warp walks the schedule (waits are warp-wide); lane 0 issues.
+    } else if (warp == kWarpSketch) {
+        // ------------------------------------------------------------------ sketch products
+        // D_s[128 rows x QS] = X_chunk * P^T, one sk_ready wait per segment of SU units; the
+        // chunk's first segment also waits until the convert warps have read the previous
+        // sketch out of D_s. The whole warp walks the schedule; lane 0 issues.
         constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, QS);
-        constexpr uint32_t idesc_m = ptx::idesc_bf16_f32(kRows, kNeu);
         const uint64_t xdesc0 = ptx::smem_desc(ptx::smem_u32(xring), 16, 1024, ptx::kLayoutSW128);
         const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(pring), 16, 1024, ptx::kLayoutSW128);
-        const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, F::WSBO, F::WLAYOUT);
+        const uint32_t ds = tm + (uint32_t)F::DS_COL;
         const bool leader = lane == 0;
-        Ring xr(NX), pr(NP), wr(NW);
+        Ring xr(NX);
         int seg = 0;
         bool ok = true;
-        // sketch of chunk i into D_s[i & 1], one sk_ready wait per segment of SU units
-        auto sketch = [&](int i) {
-            const uint32_t ds = tm + (uint32_t)(F::DS_COL + (i & 1) * QS);
+        for (int i = 0; i < G && ok; ++i) {
             for (int sg = 0; sg < NSEG; ++sg, ++seg) {
-                if (!warp_wait(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag)) {
+                if (!warp_wait_spin(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag) ||
+                    (sg == 0 && i > 0 && !warp_wait_spin(ds_free, (uint32_t)((i - 1) & 1), abort_flag))) {
                     ok = false;
                     if (leader) report(status, abort_flag, 3);
-                    return;
+                    break;
                 }
                 ptx::tc_fence_after();
+                uint64_t xd[SU], pd[SU];
 #pragma unroll
                 for (int su = 0; su < SU; ++su) {
-                    if (leader) {
-                        const uint64_t xd = xdesc0 + (uint64_t)((xr.slot * kXUnit) >> 4);
-                        const uint64_t pd = pdesc0 + (uint64_t)((pr.slot * F::P_UNIT) >> 4);
+                    xd[su] = xdesc0 + (uint64_t)((xr.slot * kXUnit) >> 4);
+                    pd[su] = pdesc0 + (uint64_t)((((seg & 1) * SU + su) * F::P_UNIT) >> 4);
+                    xr.next();
+                }
+                if (leader) {
+#pragma unroll
+                    for (int su = 0; su < SU; ++su)
 #pragma unroll
                         for (int kk = 0; kk < kUnitK / 16; ++kk)
-                            ptx::umma_bf16_ss(ds, xd + (uint64_t)(kk * 2), pd + (uint64_t)(kk * 2), idesc_s,
+                            ptx::umma_bf16_ss(ds, xd[su] + (uint64_t)(kk * 2), pd[su] + (uint64_t)(kk * 2), idesc_s,
                                               (sg > 0 || su > 0 || kk > 0) ? 1u : 0u);
-                        ptx::umma_commit(&x_empty[xr.slot]);
-                        ptx::umma_commit(&p_empty[pr.slot]);
-                    }
-                    xr.next();
-                    pr.next();
+                    ptx::umma_commit(&seg_done[seg & 3]);
                 }
+                __syncwarp();
             }
-            if (leader) ptx::umma_commit(&s_full[i & 1]);
-            __syncwarp();
-        };
-        // main product of chunk i (kc of tile t): D_j += Xs_j * Wc_j^T
-        auto main_mma = [&](int i, int t, int kc) {
+        }
+        if (*abort_flag && leader) {   // MMAs in flight finish before TMEM is released
+            volatile int no_abort = 0;
+            ptx::umma_commit(&drain[0]);
+            ptx::mbar_wait(&drain[0], 0, &no_abort, kWaitNs);
+        }
+        __syncwarp();
+    } else if (warp == kWarpMain) {
+        // ------------------------------------------------------------------ compressed products
+        // D_j[128 rows x 128] += Xs_j (A operand from TMEM) * Wc_j^T for the tile's Q N-blocks;
+        // one mm_ready wait per chunk. A second issuing warp, so that one warp's waits overlap
+        // the other's MMAs in the tensor pipe.
+        constexpr uint32_t idesc_m = ptx::idesc_bf16_f32(kRows, kNeu);
+        const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, F::WSBO, F::WLAYOUT);
+        const bool leader = lane == 0;
+        Ring wr(NW);
+        int t = 0, kc = 0;
+        for (int i = 0; i < G; ++i) {
             const int b = i & 1, a = NACC == 2 ? (t & 1) : 0;
-            if (!warp_wait(&mm_ready[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
-                ok = false;
+            if (!warp_wait_spin(&mm_ready[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
                 if (leader) report(status, abort_flag, 4);
-                return;
+                break;
             }
             ptx::tc_fence_after();
+            const uint32_t xs = tm + (uint32_t)(F::XS_COL + b * (QS / 2));
+            const uint32_t acc = tm + (uint32_t)(a * F::ACC_COLS);
+            const uint64_t wd = wdesc0 + (uint64_t)((wr.slot * F::W_STAGE) >> 4);
             if (leader) {
-                const uint32_t xs = tm + (uint32_t)(F::DS_COL + b * QS);
-                const uint64_t wd = wdesc0 + (uint64_t)((wr.slot * F::W_STAGE) >> 4);
 #pragma unroll
                 for (int j = 0; j < Q; ++j)
 #pragma unroll
@@ -320,39 +359,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         constexpr int per_panel = F::RB / 2;   // slots per Wc panel row
                         const uint32_t off = (uint32_t)(j * F::W_NB + ((kk * 16) / per_panel) * F::W_PANEL +
                                                         ((kk * 16) % per_panel) * 2);
-                        // slots s0 .. s0+15 in bf16: converted in place inside their half's columns
-                        const int s0 = j * S + kk * 16;
-                        const uint32_t acol = (uint32_t)((s0 / HW) * HW + (s0 % HW) / 2);
-                        ptx::umma_bf16_ts(tm + (uint32_t)(a * F::ACC_COLS + j * kNeu), xs + acol, wd + (uint64_t)(off >> 4),
-                                          idesc_m, (kc > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_bf16_ts(acc + (uint32_t)(j * kNeu), xs + (uint32_t)((j * S + kk * 16) / 2),
+                                          wd + (uint64_t)(off >> 4), idesc_m, (kc > 0 || kk > 0) ? 1u : 0u);
                     }
                 ptx::umma_commit(&w_empty[wr.slot]);
+                ptx::umma_commit(&main_done[b]);
                 if (kc == KC - 1) ptx::umma_commit(&acc_full[a]);
             }
             __syncwarp();
             wr.next();
-        };
-        if (G > 0) sketch(0);
-        int t = 0, kc = 0;
-        for (int i = 0; i < G && ok; ++i) {
-            if (i + 1 < G) sketch(i + 1);
-            if (!ok) break;
-            main_mma(i, t, kc);
             if (++kc == KC) { kc = 0; ++t; }
         }
-        if (*abort_flag && leader) {   // MMAs in flight finish before TMEM is released
+        if (*abort_flag && leader) {
             volatile int no_abort = 0;
-            ptx::umma_commit(drain);
-            ptx::mbar_wait(drain, 0, &no_abort, kWaitNs);
+            ptx::umma_commit(&drain[1]);
+            ptx::mbar_wait(&drain[1], 0, &no_abort, kWaitNs);
         }
         __syncwarp();
     } else if (warp == kWarpBuild) {
         // ------------------------------------------------------------------ sketch matrices
         // Panel u of chunk kc for the tile's N-blocks nb0 .. nb0+Q-1: entry (j*S + slot(k), k)
         // = sign(k) for the 64 inputs k of the unit; every other entry stays zero. A lane writes
-        // inputs lane and lane + 32 of each N-block and records where, so that the entries can
-        // be cleared when the panel comes round again. The unit's table entries (Q lines of
-        // 128 bytes) were copied into a staging ring kTabUnits - 1 units earlier.
+        // inputs lane and lane + 32 of each N-block. Shared memory is slow to reach while the
+        // tensor core streams operands from it, so this warp keeps its accesses few and
+        // independent: the table entries of a segment come from a cp.async staging ring filled
+        // D units ahead and are read in one batch; the offsets to clear when a panel comes
+        // round again stay in registers (segments alternate between two panel pairs).
+        constexpr int D = kTabUnits - SU;   // staging lookahead in units
         const int units = G * U;
         auto unit_src = [&](int pu) -> const uint16_t* {   // table entries of unit pu, N-block nb0
             const int i = pu / U, u = pu % U;
@@ -367,83 +400,99 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::cp_async_commit();
         };
-        for (int pu = 0; pu < kTabUnits - 1; ++pu) stage_unit(pu);
-        Ring pr(NP), xr(NX);
-        int pu = 0;
+        for (int pu = 0; pu < D; ++pu) stage_unit(pu);
+        Ring xr(NX);
         bool ok = true;
-        for (int g = 0; g < G * NSEG && ok; ++g) {
-            for (int su = 0; su < SU; ++su, ++pu) {
-                stage_unit(pu + kTabUnits - 1);
-                ptx::cp_async_wait<kTabUnits - 1>();   // unit pu's group has landed
-                __syncwarp();
-                const uint16_t* te = tab + (pu % kTabUnits) * (Q * kUnitK);
-                uint16_t e[F::NE];
+        uint32_t held0[SU * F::NE], held1[SU * F::NE];   // offsets written into panel pair 0 / 1
+        auto segment = [&](int g, uint32_t (&held)[SU * F::NE]) {
+            const int pu0 = g * SU;
+#pragma unroll
+            for (int su = 0; su < SU; ++su) stage_unit(pu0 + su + D);
+            ptx::cp_async_wait<D>();   // the segment's own groups have landed
+            __syncwarp();
+            uint16_t e[SU * F::NE];
+#pragma unroll
+            for (int su = 0; su < SU; ++su) {
+                const uint16_t* te = tab + ((pu0 + su) % kTabUnits) * (Q * kUnitK);
 #pragma unroll
                 for (int j = 0; j < Q; ++j)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) e[2 * j + h] = te[j * kUnitK + lane + 32 * h];
-                if (!warp_wait(&p_empty[pr.slot], pr.phase ^ 1u, abort_flag)) {
+                    for (int h = 0; h < 2; ++h) e[su * F::NE + 2 * j + h] = te[j * kUnitK + lane + 32 * h];
+            }
+            uint8_t* pair = pring + (g & 1) * SU * F::P_UNIT;
+            if (g >= 2) {   // the pair's previous segment (g - 2) has been multiplied
+                if (!warp_wait(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 5);
-                    break;
+                    return;
                 }
-                uint8_t* panel = pring + pr.slot * F::P_UNIT;
-                uint16_t* rec = clr + pr.slot * (F::NE * 32) + lane;
-                if (pu >= NP) {   // clear the non-zeros this panel held NP units ago
 #pragma unroll
-                    for (int x = 0; x < F::NE; ++x) *reinterpret_cast<uint16_t*>(panel + rec[32 * x]) = 0;
-                }
+                for (int x = 0; x < SU * F::NE; ++x) *reinterpret_cast<uint16_t*>(pair + held[x]) = 0;
+            }
+#pragma unroll
+            for (int su = 0; su < SU; ++su)
 #pragma unroll
                 for (int j = 0; j < Q; ++j)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint16_t en = e[2 * j + h];
-                        const uint32_t off = sw128_off(j * S + (en & kSrcIdxMask), lane + 32 * h);
-                        *reinterpret_cast<uint16_t*>(panel + off) = (en & kSrcNegBit) ? kBf16MinusOne : kBf16One;
-                        rec[32 * (2 * j + h)] = (uint16_t)off;
+                        const uint16_t en = e[su * F::NE + 2 * j + h];
+                        const uint32_t off = (uint32_t)(su * F::P_UNIT) + sw128_off(j * S + (en & kSrcIdxMask), lane + 32 * h);
+                        *reinterpret_cast<uint16_t*>(pair + off) = (en & kSrcNegBit) ? kBf16MinusOne : kBf16One;
+                        held[su * F::NE + 2 * j + h] = off;
                     }
-                pr.next();
-            }
-            if (!ok) break;
             ptx::fence_proxy_async_smem();
             __syncwarp();
             for (int su = 0; su < SU; ++su) {   // the segment's X boxes have landed
                 if (!warp_wait(&x_full[xr.slot], xr.phase, abort_flag)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 8);
-                    break;
+                    return;
                 }
                 xr.next();
             }
-            if (!ok) break;
             if (lane == 0) ptx::mbar_arrive(&sk_ready[g & 1]);
+        };
+        const int nseg = G * NSEG;
+        for (int g = 0; g < nseg && ok; g += 2) {
+            segment(g, held0);
+            if (ok && g + 1 < nseg) segment(g + 1, held1);
         }
         ptx::cp_async_wait<0>();
     } else if (warp >= kFirstConv && warp < kFirstConv + kConvWarps) {
         // ------------------------------------------------------------------ sketch conversion
-        // Warp (quarter, half) converts fp32 sketch columns [half*HW, half*HW + HW) of its 32
-        // lanes to bf16 pairs written to columns [half*HW, half*HW + HW/2): all of its loads
-        // complete before the first store, and no other warp reads these columns.
+        // Warp (quarter, half) reads fp32 sketch columns [half*HW, half*HW + HW) of D_s for its 32
+        // lanes, releases D_s (ds_free), rounds them to bf16 pairs and writes them to columns
+        // [half*HW/2, half*HW/2 + HW/2) of Xs[b] once the main product of chunk i-2 has read it.
         const int quad = warp & 3, half = (warp - kFirstConv) >> 2;
-        const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)(F::DS_COL + half * HW);
+        const uint32_t lanes = (uint32_t)(quad * 32) << 16;
+        const uint32_t src = tm + lanes + (uint32_t)(F::DS_COL + half * HW);
         Ring wr(NW);
         int t = 0, kc = 0;
         for (int i = 0; i < G; ++i) {
             const int b = i & 1;
-            if (!warp_wait(&s_full[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
+            const int gl = i * NSEG + NSEG - 1;   // the chunk's last sketch segment
+            if (!warp_wait(&seg_done[gl & 3], (uint32_t)((gl >> 2) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 6);
                 break;
             }
             ptx::tc_fence_after();
-            const uint32_t base = lane_base + (uint32_t)(b * QS);
             uint32_t r[HW];
 #pragma unroll
-            for (int c0 = 0; c0 < HW; c0 += 16) ptx::tmem_ld_32x32b_x16(base + (uint32_t)c0, r + c0);
+            for (int c0 = 0; c0 < HW; c0 += 16) ptx::tmem_ld_32x32b_x16(src + (uint32_t)c0, r + c0);
             ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ds_free);
 #pragma unroll
             for (int p = 0; p < HW / 2; ++p) r[p] = pack_bf16x2(r[2 * p], r[2 * p + 1]);
+            if (i >= 2 && !warp_wait(&main_done[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 10);
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t dst = tm + lanes + (uint32_t)(F::XS_COL + b * (QS / 2) + half * (HW / 2));
 #pragma unroll
-            for (int c0 = 0; c0 < HW / 2; c0 += 8) ptx::tmem_st_32x32b_x8(base + (uint32_t)c0, r + c0);
+            for (int c = 0; c < HW / 2; c += 8) ptx::tmem_st_32x32b_x8(dst + (uint32_t)c, r + c);
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             // the first convert warp also waits for the chunk's Wc and, at a tile's first
@@ -518,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == kWarpMma) {
+    if (warp == kWarpSketch) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tm, 512);
     }
