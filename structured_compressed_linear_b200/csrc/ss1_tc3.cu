@@ -58,7 +58,9 @@ constexpr int kXUnit = kRows * 128;        // bytes of one X box [128 rows x 64 
 constexpr int kWarpLoadX = 0, kWarpSketch = 1, kWarpBuild = 2, kWarpLoadW = 3, kFirstConv = 4, kConvWarps = 8;
 constexpr int kFirstEpi = kFirstConv + kConvWarps, kEpiWarps = 4;
 constexpr int kWarpMain = kFirstEpi + kEpiWarps;
-constexpr int kWarps = kWarpMain + 1;
+constexpr int kFirstBuildExtra = kWarpMain + 1;   // further build warps (warp kWarpBuild is the first)
+constexpr int kMaxBuildWarps = 4;
+constexpr int kWarps = kFirstBuildExtra + kMaxBuildWarps - 1;
 constexpr int kThreads = kWarps * 32;
 constexpr int kEpiBox = 32 * 32 * 2;       // one [32 rows x 32 neurons] bf16 store box
 constexpr int kTabUnits = 8;               // table staging ring of the build warp (units)
@@ -83,11 +85,11 @@ struct Cfg {
     static constexpr int W_STAGE = Q * W_NB;
     static constexpr int NP = 2 * SU;                    // sketch panels: two segments
     static constexpr int NW = 2;
-    static constexpr int NE = 2 * Q;                     // sketch-matrix entries per lane and unit
-    static constexpr int TAB_UNIT = Q * kUnitK * 2;      // bytes of one unit's table entries
+    static constexpr int NBW = SU * Q;                   // build warps in use: one per (unit, N-block)
+    static constexpr int TAB_UNIT = kUnitK * 2;          // bytes of one (unit, N-block)'s table entries
     static constexpr int EPI = kEpiWarps * 2 * kEpiBox;
     static constexpr int CLR = 0;
-    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + kTabUnits * TAB_UNIT + CLR;
+    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + kMaxBuildWarps * kTabUnits * TAB_UNIT + CLR;
     static constexpr int NX_FIT = (kSmemBudget - FIXED) / kXUnit;
     static constexpr int NX = NX_FIT < 2 * U + 1 ? NX_FIT : 2 * U + 1;
     // TMEM columns: Q accumulators (x NACC buffers), the fp32 sketch D_s (QS columns), then two
@@ -102,7 +104,7 @@ struct Cfg {
     static constexpr int OFF_W = OFF_P + NP * P_UNIT;
     static constexpr int OFF_E = OFF_W + NW * W_STAGE;
     static constexpr int OFF_TAB = OFF_E + EPI;
-    static constexpr int OFF_CLR = OFF_TAB + kTabUnits * TAB_UNIT;
+    static constexpr int OFF_CLR = OFF_TAB + kMaxBuildWarps * kTabUnits * TAB_UNIT;
     static constexpr int OFF_BAR = OFF_CLR + CLR;
     static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 1 + 2 + 2 * NACC + 2;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
@@ -112,6 +114,7 @@ struct Cfg {
     static_assert(DS_COL + 2 * QS <= 512, "TMEM budget");
     static_assert(NX >= 2 * SU && SMEM <= 227 * 1024, "shared memory budget: X ring holds two segments");
     static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0, "swizzle atoms stay aligned");
+    static_assert(NBW <= kMaxBuildWarps, "build warps");
 };
 
 __device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) ptx::mbar_init(&seg_done[i], 1);
         for (int i = 0; i < NW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&sk_ready[i], 1);
+            ptx::mbar_init(&sk_ready[i], F::NBW);
             ptx::mbar_init(&mm_ready[i], kConvWarps);
             ptx::mbar_init(&main_done[i], 1);
             ptx::mbar_init(&drain[i], 1);
@@ -376,83 +379,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_wait(&drain[1], 0, &no_abort, kWaitNs);
         }
         __syncwarp();
-    } else if (warp == kWarpBuild) {
+    } else if (warp == kWarpBuild || (warp >= kFirstBuildExtra && warp < kFirstBuildExtra + F::NBW - 1)) {
         // ------------------------------------------------------------------ sketch matrices
         // Panel u of chunk kc for the tile's N-blocks nb0 .. nb0+Q-1: entry (j*S + slot(k), k)
-        // = sign(k) for the 64 inputs k of the unit; every other entry stays zero. A lane writes
-        // inputs lane and lane + 32 of each N-block. Shared memory is slow to reach while the
-        // tensor core streams operands from it, so this warp keeps its accesses few and
-        // independent: the table entries of a segment come from a cp.async staging ring filled
-        // D units ahead and are read in one batch; the offsets to clear when a panel comes
-        // round again stay in registers (segments alternate between two panel pairs).
-        constexpr int D = kTabUnits - SU;   // staging lookahead in units
-        const int units = G * U;
-        auto unit_src = [&](int pu) -> const uint16_t* {   // table entries of unit pu, N-block nb0
-            const int i = pu / U, u = pu % U;
+        // = sign(k) for the 64 inputs k of the unit; every other entry stays zero. Build warp
+        // bw writes unit su = bw % SU of each segment for N-block j = bw / SU: inputs lane and
+        // lane + 32. Shared memory is slow to reach while the tensor core streams operands from
+        // it, so the work is split over NBW warps whose latency chains overlap, each keeping its
+        // accesses few: its table entries come from a cp.async ring filled D units ahead, and
+        // the offsets to clear when a panel comes round again stay in registers (segments
+        // alternate between two panel pairs). The warps of the first N-block also wait for
+        // their unit's X box, so sk_ready (all NBW warps) means the whole segment is ready.
+        const int bw = warp == kWarpBuild ? 0 : warp - kFirstBuildExtra + 1;
+        const int su = bw % SU, j = bw / SU;
+        constexpr int D = kTabUnits - 1;   // staging lookahead in segments
+        const int nseg = G * NSEG;
+        uint16_t* mytab = tab + bw * (kTabUnits * kUnitK);
+        auto seg_src = [&](int g) -> const uint16_t* {   // table entries of (segment g, su, j)
+            const int pu = g * SU + su, i = pu / U, u = pu % U;
             const int tile = (int)blockIdx.x + (i / KC) * (int)gridDim.x, kc = i % KC;
-            return slot_tab + (size_t)((tile % NG) * Q) * K + (size_t)kc * BK + u * kUnitK;
+            return slot_tab + (size_t)((tile % NG) * Q + j) * K + (size_t)kc * BK + u * kUnitK;
         };
-        auto stage_unit = [&](int pu) {   // lanes 0 .. 8Q-1 copy 16 bytes each; always one group
-            if (pu < units && lane < 8 * Q) {
-                const int j = lane >> 3, part = lane & 7;
-                ptx::cp_async_ca_16(tab + (pu % kTabUnits) * (Q * kUnitK) + j * kUnitK + part * 8,
-                                    unit_src(pu) + (size_t)j * K + part * 8);
-            }
+        auto stage = [&](int g) {   // lanes 0..7 copy 16 bytes each; always one group
+            if (g < nseg && lane < 8) ptx::cp_async_ca_16(mytab + (g % kTabUnits) * kUnitK + lane * 8, seg_src(g) + lane * 8);
             ptx::cp_async_commit();
         };
-        for (int pu = 0; pu < D; ++pu) stage_unit(pu);
-        Ring xr(NX);
+        for (int g = 0; g < D; ++g) stage(g);
         bool ok = true;
-        uint32_t held0[SU * F::NE], held1[SU * F::NE];   // offsets written into panel pair 0 / 1
-        auto segment = [&](int g, uint32_t (&held)[SU * F::NE]) {
-            const int pu0 = g * SU;
-#pragma unroll
-            for (int su = 0; su < SU; ++su) stage_unit(pu0 + su + D);
-            ptx::cp_async_wait<D>();   // the segment's own groups have landed
+        uint32_t held0[2], held1[2];   // offsets written into this warp's panel of pair 0 / 1
+        auto segment = [&](int g, uint32_t (&held)[2]) {
+            stage(g + D);
+            ptx::cp_async_wait<D>();   // segment g's group has landed
             __syncwarp();
-            uint16_t e[SU * F::NE];
-#pragma unroll
-            for (int su = 0; su < SU; ++su) {
-                const uint16_t* te = tab + ((pu0 + su) % kTabUnits) * (Q * kUnitK);
-#pragma unroll
-                for (int j = 0; j < Q; ++j)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) e[su * F::NE + 2 * j + h] = te[j * kUnitK + lane + 32 * h];
-            }
-            uint8_t* pair = pring + (g & 1) * SU * F::P_UNIT;
+            const uint16_t* te = mytab + (g % kTabUnits) * kUnitK;
+            const uint16_t e0 = te[lane], e1 = te[lane + 32];
+            uint8_t* panel = pring + ((g & 1) * SU + su) * F::P_UNIT;
             if (g >= 2) {   // the pair's previous segment (g - 2) has been multiplied
-                if (!warp_wait(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag)) {
+                if (!warp_wait_spin(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 5);
                     return;
                 }
-#pragma unroll
-                for (int x = 0; x < SU * F::NE; ++x) *reinterpret_cast<uint16_t*>(pair + held[x]) = 0;
+                *reinterpret_cast<uint16_t*>(panel + held[0]) = 0;
+                *reinterpret_cast<uint16_t*>(panel + held[1]) = 0;
             }
-#pragma unroll
-            for (int su = 0; su < SU; ++su)
-#pragma unroll
-                for (int j = 0; j < Q; ++j)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint16_t en = e[su * F::NE + 2 * j + h];
-                        const uint32_t off = (uint32_t)(su * F::P_UNIT) + sw128_off(j * S + (en & kSrcIdxMask), lane + 32 * h);
-                        *reinterpret_cast<uint16_t*>(pair + off) = (en & kSrcNegBit) ? kBf16MinusOne : kBf16One;
-                        held[su * F::NE + 2 * j + h] = off;
-                    }
+            held[0] = sw128_off(j * S + (e0 & kSrcIdxMask), lane);
+            held[1] = sw128_off(j * S + (e1 & kSrcIdxMask), lane + 32);
+            *reinterpret_cast<uint16_t*>(panel + held[0]) = (e0 & kSrcNegBit) ? kBf16MinusOne : kBf16One;
+            *reinterpret_cast<uint16_t*>(panel + held[1]) = (e1 & kSrcNegBit) ? kBf16MinusOne : kBf16One;
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            for (int su = 0; su < SU; ++su) {   // the segment's X boxes have landed
-                if (!warp_wait(&x_full[xr.slot], xr.phase, abort_flag)) {
+            if (j == 0) {   // unit su of the segment: its X box has landed
+                const int xu = g * SU + su;
+                if (!warp_wait_spin(&x_full[xu % NX], (uint32_t)((xu / NX) & 1), abort_flag)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 8);
                     return;
                 }
-                xr.next();
             }
             if (lane == 0) ptx::mbar_arrive(&sk_ready[g & 1]);
         };
-        const int nseg = G * NSEG;
         for (int g = 0; g < nseg && ok; g += 2) {
             segment(g, held0);
             if (ok && g + 1 < nseg) segment(g + 1, held1);
@@ -471,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < G; ++i) {
             const int b = i & 1;
             const int gl = i * NSEG + NSEG - 1;   // the chunk's last sketch segment
-            if (!warp_wait(&seg_done[gl & 3], (uint32_t)((gl >> 2) & 1), abort_flag)) {
+            if (!warp_wait_spin(&seg_done[gl & 3], (uint32_t)((gl >> 2) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 6);
                 break;
             }
@@ -485,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) ptx::mbar_arrive(ds_free);
 #pragma unroll
             for (int p = 0; p < HW / 2; ++p) r[p] = pack_bf16x2(r[2 * p], r[2 * p + 1]);
-            if (i >= 2 && !warp_wait(&main_done[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
+            if (i >= 2 && !warp_wait_spin(&main_done[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 10);
                 break;
             }
@@ -499,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // chunk, for the epilogue to have read the accumulator
             if (warp == kFirstConv) {
                 const int a = NACC == 2 ? (t & 1) : 0;
-                if (!warp_wait(&w_full[wr.slot], wr.phase, abort_flag) ||
+                if (!warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag) ||
                     (kc == 0 && !warp_wait(&acc_empty[a], (uint32_t)(((t / NACC) & 1) ^ 1), abort_flag))) {
                     if (lane == 0) report(status, abort_flag, 9);
                     break;
@@ -510,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             wr.next();
             if (++kc == KC) { kc = 0; ++t; }
         }
-    } else {
+    } else if (warp >= kFirstEpi && warp < kFirstEpi + kEpiWarps) {
         // ------------------------------------------------------------------ epilogue
         // Warp `quad` owns rows [32 quad, 32 quad + 32) of the tile. Per [32 x 32] block: two
         // blocks' TMEM loads in flight, bf16 rounding, a swizzled (64-byte) staging box, one TMA
