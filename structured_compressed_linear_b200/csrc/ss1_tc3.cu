@@ -63,7 +63,6 @@ constexpr int kMaxBuildWarps = 4;
 constexpr int kWarps = kFirstBuildExtra + kMaxBuildWarps - 1;
 constexpr int kThreads = kWarps * 32;
 constexpr int kEpiBox = 32 * 32 * 2;       // one [32 rows x 32 neurons] bf16 store box
-constexpr int kTabUnits = 8;               // table staging ring of the build warp (units)
 constexpr int kSmemBudget = 225 * 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint16_t kBf16One = 0x3F80u, kBf16MinusOne = 0xBF80u;
@@ -86,32 +85,34 @@ struct Cfg {
     static constexpr int NP = 2 * SU;                    // sketch panels: two segments
     static constexpr int NW = 2;
     static constexpr int NBW = SU * Q;                   // build warps in use: one per (unit, N-block)
-    static constexpr int TAB_UNIT = kUnitK * 2;          // bytes of one (unit, N-block)'s table entries
     static constexpr int EPI = kEpiWarps * 2 * kEpiBox;
     static constexpr int CLR = 0;
-    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + kMaxBuildWarps * kTabUnits * TAB_UNIT + CLR;
+    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + CLR;
     static constexpr int NX_FIT = (kSmemBudget - FIXED) / kXUnit;
     static constexpr int NX = NX_FIT < 2 * U + 1 ? NX_FIT : 2 * U + 1;
-    // TMEM columns: Q accumulators (x NACC buffers), the fp32 sketch D_s (QS columns), then two
-    // bf16 sketch buffers Xs (QS / 2 columns each: two slots per column)
+    // TMEM columns: Q accumulators (x NACC buffers), two fp32 sketch buffers D_s (QS columns each)
+    // and, where the columns allow (SEP), two bf16 sketch buffers Xs (QS / 2 columns each, two
+    // slots per column); otherwise the bf16 sketch is written inside its D_s buffer (in place).
+    // Preference: two accumulators (the epilogue overlaps the next tile), then SEP.
     static constexpr int ACC_COLS = Q * kNeu;
     static constexpr int NACC = (2 * ACC_COLS + 2 * QS <= 512) ? 2 : 1;
+    static constexpr bool SEP = NACC * ACC_COLS + 3 * QS <= 512;
     static constexpr int DS_COL = NACC * ACC_COLS;
-    static constexpr int XS_COL = DS_COL + QS;
+    static constexpr int XS_COL = DS_COL + 2 * QS;
     // shared memory (the swizzled buffers first, each a multiple of 1 KB)
     static constexpr int OFF_X = 0;
     static constexpr int OFF_P = OFF_X + NX * kXUnit;
     static constexpr int OFF_W = OFF_P + NP * P_UNIT;
     static constexpr int OFF_E = OFF_W + NW * W_STAGE;
     static constexpr int OFF_TAB = OFF_E + EPI;
-    static constexpr int OFF_CLR = OFF_TAB + kMaxBuildWarps * kTabUnits * TAB_UNIT;
+    static constexpr int OFF_CLR = OFF_TAB;
     static constexpr int OFF_BAR = OFF_CLR + CLR;
-    static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 1 + 2 + 2 * NACC + 2;
+    static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 2 + 2 + NACC + NACC * Q + 2;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(BK % kUnitK == 0 && BK <= 256 && U % SU == 0, "chunks of whole 64-input units");
     static_assert(S % 16 == 0 && S >= 16 && S <= 128, "UMMA K-steps of 16 over the slots");
     static_assert(QS % 32 == 0 && QS <= 256 && HW % 16 == 0, "sketch UMMA N and conversion halves");
-    static_assert(DS_COL + 2 * QS <= 512, "TMEM budget");
+    static_assert(DS_COL + 2 * QS + (SEP ? QS : 0) <= 512, "TMEM budget");
     static_assert(NX >= 2 * SU && SMEM <= 227 * 1024, "shared memory budget: X ring holds two segments");
     static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0, "swizzle atoms stay aligned");
     static_assert(NBW <= kMaxBuildWarps, "build warps");
@@ -187,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* pring = smem + F::OFF_P;
     uint8_t* wring = smem + F::OFF_W;
     uint8_t* estage = smem + F::OFF_E;
-    uint16_t* tab = reinterpret_cast<uint16_t*>(smem + F::OFF_TAB);
     // One tcgen05.commit per sketch segment (seg_done) tells every consumer at once: the X
     // loader and the build warp that the segment's X boxes and panels are free, the convert
     // warps (at a chunk's last segment) that the sketch is in D_s. Commits from the issuing
@@ -198,11 +198,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* w_full = sk_ready + 2;
     uint64_t* w_empty = w_full + NW;
     uint64_t* mm_ready = w_empty + NW;    // [2] Xs[b] written, Wc (and the accumulator) ready
-    uint64_t* ds_free = mm_ready + 2;     // the convert warps have read D_s
-    uint64_t* main_done = ds_free + 1;    // [2] main product of a chunk done reading Xs[b]
-    uint64_t* acc_full = main_done + 2;   // [NACC]
-    uint64_t* acc_empty = acc_full + NACC;
-    uint64_t* drain = acc_empty + NACC;   // [2] abort path: completion of every MMA a warp issued
+    uint64_t* ds_free = mm_ready + 2;     // [2] D_s[b] may take the next sketch: SEP, the convert warps
+                                          // have read it; in place, the main product has read its Xs
+    uint64_t* xs_free = ds_free + 2;      // [2] (SEP) the main product has read Xs[b]
+    uint64_t* acc_full = xs_free + 2;     // [NACC]
+    uint64_t* acc_empty = acc_full + NACC;   // [NACC][Q] the epilogue has read N-block j's columns
+    uint64_t* drain = acc_empty + NACC * Q;  // [2] abort path: completion of every MMA a warp issued
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -221,11 +222,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&sk_ready[i], F::NBW);
             ptx::mbar_init(&mm_ready[i], kConvWarps);
-            ptx::mbar_init(&main_done[i], 1);
+            ptx::mbar_init(&ds_free[i], F::SEP ? kConvWarps : 1);
+            ptx::mbar_init(&xs_free[i], 1);
             ptx::mbar_init(&drain[i], 1);
         }
-        ptx::mbar_init(ds_free, kConvWarps);
-        for (int i = 0; i < NACC; ++i) { ptx::mbar_init(&acc_full[i], 1); ptx::mbar_init(&acc_empty[i], kEpiWarps); }
+        for (int i = 0; i < NACC; ++i) ptx::mbar_init(&acc_full[i], 1);
+        for (int i = 0; i < NACC * Q; ++i) ptx::mbar_init(&acc_empty[i], kEpiWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -289,21 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWarpSketch) {
         // ------------------------------------------------------------------ sketch products
-        // D_s[128 rows x QS] = X_chunk * P^T, one sk_ready wait per segment of SU units; the
-        // chunk's first segment also waits until the convert warps have read the previous
-        // sketch out of D_s. The whole warp walks the schedule; lane 0 issues.
+        // D_s[i & 1][128 rows x QS] = X_chunk * P^T, one sk_ready wait per segment of SU units;
+        // the chunk's first segment also waits until the buffer's previous chunk (i - 2) has
+        // released it. The whole warp walks the schedule; lane 0 issues.
         constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kRows, QS);
         const uint64_t xdesc0 = ptx::smem_desc(ptx::smem_u32(xring), 16, 1024, ptx::kLayoutSW128);
         const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(pring), 16, 1024, ptx::kLayoutSW128);
-        const uint32_t ds = tm + (uint32_t)F::DS_COL;
         const bool leader = lane == 0;
         Ring xr(NX);
         int seg = 0;
         bool ok = true;
         for (int i = 0; i < G && ok; ++i) {
+            const uint32_t ds = tm + (uint32_t)(F::DS_COL + (i & 1) * QS);
             for (int sg = 0; sg < NSEG; ++sg, ++seg) {
                 if (!warp_wait_spin(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag) ||
-                    (sg == 0 && i > 0 && !warp_wait_spin(ds_free, (uint32_t)((i - 1) & 1), abort_flag))) {
+                    (sg == 0 && i >= 2 && !warp_wait_spin(&ds_free[i & 1], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag))) {
                     ok = false;
                     if (leader) report(status, abort_flag, 3);
                     break;
@@ -351,25 +353,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             ptx::tc_fence_after();
-            const uint32_t xs = tm + (uint32_t)(F::XS_COL + b * (QS / 2));
+            const uint32_t xs = tm + (uint32_t)(F::SEP ? F::XS_COL + b * (QS / 2) : F::DS_COL + b * QS);
+            const uint32_t acc_par = (uint32_t)(((t / NACC) & 1) ^ 1);   // n-th use of buffer a waits use n-1
             const uint32_t acc = tm + (uint32_t)(a * F::ACC_COLS);
             const uint64_t wd = wdesc0 + (uint64_t)((wr.slot * F::W_STAGE) >> 4);
+            bool stalled = false;
             if (leader) {
 #pragma unroll
-                for (int j = 0; j < Q; ++j)
+                for (int j = 0; j < Q; ++j) {
+                    // a tile's first chunk: N-block j's accumulator columns have been read out
+                    if (kc == 0) {
+                        if (!ptx::mbar_wait(&acc_empty[a * Q + j], acc_par, abort_flag, kWaitNs)) {
+                            report(status, abort_flag, 11);
+                            stalled = true;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                    }
 #pragma unroll
                     for (int kk = 0; kk < S / 16; ++kk) {
                         constexpr int per_panel = F::RB / 2;   // slots per Wc panel row
                         const uint32_t off = (uint32_t)(j * F::W_NB + ((kk * 16) / per_panel) * F::W_PANEL +
                                                         ((kk * 16) % per_panel) * 2);
-                        ptx::umma_bf16_ts(acc + (uint32_t)(j * kNeu), xs + (uint32_t)((j * S + kk * 16) / 2),
-                                          wd + (uint64_t)(off >> 4), idesc_m, (kc > 0 || kk > 0) ? 1u : 0u);
+                        // slots s0 .. s0+15 in bf16: SEP, column s0 / 2 of Xs[b]; in place, inside
+                        // the converting warp's half of D_s[b]
+                        const int s0 = j * S + kk * 16;
+                        const uint32_t acol = F::SEP ? (uint32_t)(s0 / 2) : (uint32_t)((s0 / HW) * HW + (s0 % HW) / 2);
+                        ptx::umma_bf16_ts(acc + (uint32_t)(j * kNeu), xs + acol, wd + (uint64_t)(off >> 4), idesc_m,
+                                          (kc > 0 || kk > 0) ? 1u : 0u);
                     }
+                }
                 ptx::umma_commit(&w_empty[wr.slot]);
-                ptx::umma_commit(&main_done[b]);
+                ptx::umma_commit(F::SEP ? &xs_free[b] : &ds_free[b]);
                 if (kc == KC - 1) ptx::umma_commit(&acc_full[a]);
             }
-            __syncwarp();
+            if (__shfl_sync(0xffffffffu, stalled ? 1 : 0, 0)) break;
             wr.next();
             if (++kc == KC) { kc = 0; ++t; }
         }
@@ -386,33 +404,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         // bw writes unit su = bw % SU of each segment for N-block j = bw / SU: inputs lane and
         // lane + 32. Shared memory is slow to reach while the tensor core streams operands from
         // it, so the work is split over NBW warps whose latency chains overlap, each keeping its
-        // accesses few: its table entries come from a cp.async ring filled D units ahead, and
-        // the offsets to clear when a panel comes round again stay in registers (segments
-        // alternate between two panel pairs). The warps of the first N-block also wait for
-        // their unit's X box, so sk_ready (all NBW warps) means the whole segment is ready.
+        // shared accesses to the stores themselves: its table entries are loaded from global
+        // memory into registers two segments ahead, and the offsets to clear when a panel comes
+        // round again stay in registers (segments alternate between two panel pairs). The warps
+        // of the first N-block also wait for their unit's X box, so sk_ready (all NBW warps)
+        // means the whole segment is ready.
         const int bw = warp == kWarpBuild ? 0 : warp - kFirstBuildExtra + 1;
         const int su = bw % SU, j = bw / SU;
-        constexpr int D = kTabUnits - 1;   // staging lookahead in segments
         const int nseg = G * NSEG;
-        uint16_t* mytab = tab + bw * (kTabUnits * kUnitK);
-        auto seg_src = [&](int g) -> const uint16_t* {   // table entries of (segment g, su, j)
-            const int pu = g * SU + su, i = pu / U, u = pu % U;
-            const int tile = (int)blockIdx.x + (i / KC) * (int)gridDim.x, kc = i % KC;
-            return slot_tab + (size_t)((tile % NG) * Q + j) * K + (size_t)kc * BK + u * kUnitK;
+        auto fetch = [&](int g, uint32_t (&e)[2]) {   // table entries of (segment g, su, j)
+            if (g < nseg) {
+                const int pu = g * SU + su, i = pu / U, u = pu % U;
+                const int tile = (int)blockIdx.x + (i / KC) * (int)gridDim.x, kc = i % KC;
+                const uint16_t* src = slot_tab + (size_t)((tile % NG) * Q + j) * K + (size_t)kc * BK + u * kUnitK;
+                e[0] = __ldg(src + lane);
+                e[1] = __ldg(src + lane + 32);
+            }
         };
-        auto stage = [&](int g) {   // lanes 0..7 copy 16 bytes each; always one group
-            if (g < nseg && lane < 8) ptx::cp_async_ca_16(mytab + (g % kTabUnits) * kUnitK + lane * 8, seg_src(g) + lane * 8);
-            ptx::cp_async_commit();
-        };
-        for (int g = 0; g < D; ++g) stage(g);
         bool ok = true;
         uint32_t held0[2], held1[2];   // offsets written into this warp's panel of pair 0 / 1
-        auto segment = [&](int g, uint32_t (&held)[2]) {
-            stage(g + D);
-            ptx::cp_async_wait<D>();   // segment g's group has landed
-            __syncwarp();
-            const uint16_t* te = mytab + (g % kTabUnits) * kUnitK;
-            const uint16_t e0 = te[lane], e1 = te[lane + 32];
+        uint32_t ent0[2], ent1[2];     // table entries of the next even / odd segment
+        fetch(0, ent0);
+        fetch(1, ent1);
+        auto segment = [&](int g, uint32_t (&held)[2], uint32_t (&ent)[2]) {
+            const uint32_t e0 = ent[0], e1 = ent[1];
+            fetch(g + 2, ent);
             uint8_t* panel = pring + ((g & 1) * SU + su) * F::P_UNIT;
             if (g >= 2) {   // the pair's previous segment (g - 2) has been multiplied
                 if (!warp_wait_spin(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag)) {
@@ -423,8 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint16_t*>(panel + held[0]) = 0;
                 *reinterpret_cast<uint16_t*>(panel + held[1]) = 0;
             }
-            held[0] = sw128_off(j * S + (e0 & kSrcIdxMask), lane);
-            held[1] = sw128_off(j * S + (e1 & kSrcIdxMask), lane + 32);
+            held[0] = sw128_off(j * S + (int)(e0 & kSrcIdxMask), lane);
+            held[1] = sw128_off(j * S + (int)(e1 & kSrcIdxMask), lane + 32);
             *reinterpret_cast<uint16_t*>(panel + held[0]) = (e0 & kSrcNegBit) ? kBf16MinusOne : kBf16One;
             *reinterpret_cast<uint16_t*>(panel + held[1]) = (e1 & kSrcNegBit) ? kBf16MinusOne : kBf16One;
             ptx::fence_proxy_async_smem();
@@ -440,18 +456,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) ptx::mbar_arrive(&sk_ready[g & 1]);
         };
         for (int g = 0; g < nseg && ok; g += 2) {
-            segment(g, held0);
-            if (ok && g + 1 < nseg) segment(g + 1, held1);
+            segment(g, held0, ent0);
+            if (ok && g + 1 < nseg) segment(g + 1, held1, ent1);
         }
-        ptx::cp_async_wait<0>();
     } else if (warp >= kFirstConv && warp < kFirstConv + kConvWarps) {
         // ------------------------------------------------------------------ sketch conversion
-        // Warp (quarter, half) reads fp32 sketch columns [half*HW, half*HW + HW) of D_s for its 32
-        // lanes, releases D_s (ds_free), rounds them to bf16 pairs and writes them to columns
-        // [half*HW/2, half*HW/2 + HW/2) of Xs[b] once the main product of chunk i-2 has read it.
+        // Warp (quarter, half) reads fp32 sketch columns [half*HW, half*HW + HW) of D_s[b] for its
+        // 32 lanes and rounds them to bf16 pairs. SEP: it releases D_s[b] (ds_free) as soon as the
+        // loads are done and writes columns [half*HW/2, +HW/2) of Xs[b] once the main product of
+        // chunk i - 2 has read them. In place: it writes columns [half*HW, +HW/2) of D_s[b], which
+        // only it has read.
         const int quad = warp & 3, half = (warp - kFirstConv) >> 2;
         const uint32_t lanes = (uint32_t)(quad * 32) << 16;
-        const uint32_t src = tm + lanes + (uint32_t)(F::DS_COL + half * HW);
         Ring wr(NW);
         int t = 0, kc = 0;
         for (int i = 0; i < G; ++i) {
@@ -462,34 +478,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             ptx::tc_fence_after();
+            const uint32_t src = tm + lanes + (uint32_t)(F::DS_COL + b * QS + half * HW);
             uint32_t r[HW];
 #pragma unroll
             for (int c0 = 0; c0 < HW; c0 += 16) ptx::tmem_ld_32x32b_x16(src + (uint32_t)c0, r + c0);
             ptx::tmem_ld_wait();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ds_free);
+            if (F::SEP) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&ds_free[b]);
+            }
 #pragma unroll
             for (int p = 0; p < HW / 2; ++p) r[p] = pack_bf16x2(r[2 * p], r[2 * p + 1]);
-            if (i >= 2 && !warp_wait_spin(&main_done[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
-                if (lane == 0) report(status, abort_flag, 10);
-                break;
+            uint32_t dst = src;
+            if (F::SEP) {
+                if (i >= 2 && !warp_wait_spin(&xs_free[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
+                    if (lane == 0) report(status, abort_flag, 10);
+                    break;
+                }
+                ptx::tc_fence_after();
+                dst = tm + lanes + (uint32_t)(F::XS_COL + b * (QS / 2) + half * (HW / 2));
             }
-            ptx::tc_fence_after();
-            const uint32_t dst = tm + lanes + (uint32_t)(F::XS_COL + b * (QS / 2) + half * (HW / 2));
 #pragma unroll
             for (int c = 0; c < HW / 2; c += 8) ptx::tmem_st_32x32b_x8(dst + (uint32_t)c, r + c);
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
-            // the first convert warp also waits for the chunk's Wc and, at a tile's first
-            // chunk, for the epilogue to have read the accumulator
-            if (warp == kFirstConv) {
-                const int a = NACC == 2 ? (t & 1) : 0;
-                if (!warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag) ||
-                    (kc == 0 && !warp_wait(&acc_empty[a], (uint32_t)(((t / NACC) & 1) ^ 1), abort_flag))) {
-                    if (lane == 0) report(status, abort_flag, 9);
-                    break;
-                }
+            // the first convert warp also waits for the chunk's Wc
+            if (warp == kFirstConv && !warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 9);
+                break;
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&mm_ready[b]);
@@ -538,10 +555,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32), ra);
                 ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32 + 32), rb);
                 ptx::tmem_ld_wait();
-                if (q + 2 == 4 * Q) {   // accumulator read: the next tile's MMAs may start
+                if ((q + 2) % 4 == 0) {   // N-block (q / 4) read: the next tile's MMAs into it may start
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&acc_empty[a]);
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[a * Q + q / 4]);
                 }
                 store_block(q, ra);
                 store_block(q + 1, rb);
