@@ -206,6 +206,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) 
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// After tmem_ld_wait: marks registers filled by an earlier tcgen05.ld as written here, so that
+// the compiler cannot move their uses above the wait (the load's outputs are only valid after it).
+template <int N>
+__device__ __forceinline__ void tmem_ld_fence_regs(uint32_t* r) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Warp-collective: one 32-bit column of 32 lanes (lane = thread) at a run-time column.
 __device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
     uint32_t r;

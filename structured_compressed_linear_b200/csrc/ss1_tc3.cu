@@ -483,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c0 = 0; c0 < HW; c0 += 16) ptx::tmem_ld_32x32b_x16(src + (uint32_t)c0, r + c0);
             ptx::tmem_ld_wait();
+            ptx::tmem_ld_fence_regs<HW>(r);
             if (F::SEP) {
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -549,19 +550,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++nst;
             };
+            // two register buffers: the next block's TMEM load is in flight while this block is
+            // staged and stored; N-block j is released right after its last block (4j+3) has landed
+            const uint32_t abase = lane_base + (uint32_t)(a * F::ACC_COLS);
+            uint32_t ra[32], rb[32];
+            ptx::tmem_ld_32x32b_x32(abase, ra);
+            ptx::tmem_ld_wait();
+            ptx::tmem_ld_fence_regs<32>(ra);
 #pragma unroll 1
             for (int q = 0; q < 4 * Q; q += 2) {
-                uint32_t ra[32], rb[32];
-                ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32), ra);
-                ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(a * F::ACC_COLS + q * 32 + 32), rb);
+                ptx::tmem_ld_32x32b_x32(abase + (uint32_t)((q + 1) * 32), rb);
+                store_block(q, ra);
                 ptx::tmem_ld_wait();
-                if ((q + 2) % 4 == 0) {   // N-block (q / 4) read: the next tile's MMAs into it may start
+                ptx::tmem_ld_fence_regs<32>(rb);
+                if ((q + 2) % 4 == 0) {   // N-block q / 4 read: the next tile's MMAs into it may start
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[a * Q + q / 4]);
                 }
-                store_block(q, ra);
+                if (q + 2 < 4 * Q) ptx::tmem_ld_32x32b_x32(abase + (uint32_t)((q + 2) * 32), ra);
                 store_block(q + 1, rb);
+                if (q + 2 < 4 * Q) {
+                    ptx::tmem_ld_wait();
+                    ptx::tmem_ld_fence_regs<32>(ra);
+                }
             }
         }
         if (lane == 0) ptx::tma_store_wait0();
