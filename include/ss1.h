@@ -142,6 +142,45 @@ SS1_API int ss1_device_status(ss1_handle h, int32_t* detail);
 /* ss1_strerror -- static, NUL-terminated text for a status code. */
 SS1_API const char* ss1_strerror(int status);
 
+/* Table entries ((N / BN) * K) that ss1_forward_noalloc accepts at most. */
+#define SS1_NOALLOC_MAX_ENTRIES 983040
+
+/*
+ * ss1_forward_noalloc -- ss1_create + ss1_forward in one call that allocates nothing.
+ * This entry point has no counterpart in the SS1 paper; it only changes where the layer's
+ * hash tables live. It is for callers that must not let a library allocate device memory:
+ * a serving process that reserves all device memory for its own pool up front (an
+ * allocation could fail or fragment that pool mid-run), or code that needs one layer once
+ * and cannot afford ss1_create's allocations and device synchronisation.
+ *
+ *   K, N, c, BK, BN, seed : as for ss1_create (same checks, same tables, same Y).
+ *   X, Wc, Y, M, dtype    : as for ss1_forward.
+ *   device_status : device int32 word owned by the caller, or NULL. The call clears it on
+ *                   `stream` before the launches; a kernel that gives up a bounded wait
+ *                   writes its non-zero code there (read it after synchronising). With
+ *                   NULL the library's own word is used and a time-out is not reported.
+ *   stream        : a cudaStream_t passed as void* (NULL = legacy default stream).
+ *
+ * Every call regenerates the tables on `stream` into one fixed region of device memory
+ * that the library reserves statically (16 MiB per device: 17 bytes per table entry plus
+ * padding), then runs the kernel ss1_forward would choose. Shapes with
+ * (N / BN) * K > SS1_NOALLOC_MAX_ENTRIES are rejected with UNSUPPORTED_SHAPE. No
+ * cudaMalloc, cudaFree, pinned allocation or allocating library routine is called, and
+ * nothing synchronises the device; the region needs no zeroing because the table kernels
+ * write all of it that the forward reads.
+ *
+ * The first call on a device does one-time set-up (it looks up the region's address and
+ * sets kernel attributes); make that first call outside any stream capture.
+ * Calls share the one region: two calls whose work can overlap on the device (different
+ * streams without ordering, or different host threads) race on the tables and give wrong
+ * results. Order them on one stream or with events. Asynchronous: returns after the
+ * launches. Errors: INVALID_ARG, UNSUPPORTED_DEVICE, UNSUPPORTED_SHAPE, MISALIGNED (X, Wc,
+ * Y and device_status must be 16- resp. 4-byte aligned), CUDA.
+ */
+SS1_API int ss1_forward_noalloc(int64_t K, int64_t N, int c, int BK, int BN, uint64_t seed, const void* X,
+                                const void* Wc, void* Y, int64_t M, int dtype, int32_t* device_status,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

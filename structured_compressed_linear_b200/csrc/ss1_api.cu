@@ -42,6 +42,19 @@ int kernel_for(const ss1_layer& L, int64_t M, int dtype) {
 
 }  // namespace
 
+namespace ss1 {
+
+int auto_kernel(const ss1_layer& L, int64_t M, int dtype) { return kernel_for(L, M, dtype); }
+
+bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN) {
+    if (K < 1 || N < 1 || BK < 1 || BN < 1) return false;
+    if (!(c == 1 || c == 2 || c == 4 || c == 8)) return false;
+    if (BK > 256 || BK % c != 0 || K % BK != 0 || N % BN != 0 || BN % 16 != 0) return false;
+    return K <= (int64_t)1 << 30 && N <= (int64_t)1 << 30;
+}
+
+}  // namespace ss1
+
 extern "C" {
 
 SS1_API const char* ss1_strerror(int status) {

@@ -35,6 +35,11 @@ namespace ss1 {
 // Device status codes written by kernels with bounded waits: (kernel id << 8) | wait site.
 enum : int32_t { kStatusKernelTC = 1 };
 
+// The kernel ss1_forward picks for (M, dtype) (SS1_KERNEL_TC, _SIMT or _SMALLM).
+int auto_kernel(const ss1_layer& L, int64_t M, int dtype);
+// The shape checks of ss1_create.
+bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN);
+
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);
 // Derives d_gather from d_src (run after launch_hashgen).
 cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st);

@@ -20,7 +20,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libss1.so")
 
 SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel", "ss1_destroy",
-           "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror")
+           "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc")
+
+#: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
+NOALLOC_MAX_ENTRIES = 983040
 
 
 class Kernel(IntEnum):
@@ -57,6 +60,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.ss1_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     L.ss1_strerror.argtypes = [i32]
+    L.ss1_forward_noalloc.argtypes = [i64, i64, i32, i32, i32, u64, vp, vp, vp, i64, i32, vp, vp]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":
@@ -158,3 +162,33 @@ class SS1Layer:
             self.close()
         except Exception:
             pass
+
+
+def forward_noalloc(X: torch.Tensor, Wc: torch.Tensor, K: int, N: int, c: int, BK: int, BN: int, seed: int,
+                    out: Optional[torch.Tensor] = None, device_status: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Y = SS1(X) through ss1_forward_noalloc: no handle, the tables rebuilt in the library's
+    static device region on `stream`. Calls must not overlap on the device (they share that
+    region). `device_status`, if given, is a CUDA int32 tensor of one element that receives the
+    kernels' bounded-wait status."""
+    if X.dim() != 2 or X.shape[1] != K:
+        raise ValueError(f"X must be [M, {K}]")
+    if Wc.shape != (N, K // c):
+        raise ValueError(f"Wc must be [{N}, {K // c}]")
+    if X.dtype != Wc.dtype or not X.is_cuda or not Wc.is_cuda:
+        raise ValueError("X and Wc must be CUDA tensors of one dtype")
+    if not (X.is_contiguous() and Wc.is_contiguous()):
+        raise ValueError("X and Wc must be contiguous")
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    elif out.shape != (M, N) or out.dtype != X.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [M, N] tensor of X's dtype")
+    if device_status is not None and (device_status.dtype != torch.int32 or not device_status.is_cuda):
+        raise ValueError("device_status must be a CUDA int32 tensor")
+    st = stream if stream is not None else torch.cuda.current_stream(X.device)
+    status_ptr = device_status.data_ptr() if device_status is not None else None
+    _check(lib().ss1_forward_noalloc(K, N, c, BK, BN, seed & 0xFFFFFFFFFFFFFFFF, X.data_ptr(), Wc.data_ptr(),
+                                     out.data_ptr(), M, _dtype_code(X.dtype), status_ptr, st.cuda_stream),
+           "ss1_forward_noalloc")
+    return out

@@ -65,3 +65,10 @@ def test_argument_checks_before_device(lib):
     bogus = ctypes.c_void_p(0x1000)
     assert lib.ss1_get_info(bogus, None, None, None, None, None) == -7
     assert lib.ss1_destroy(bogus) == -7
+    # the allocation-free forward checks its arguments and its table limit first
+    fwd = lib.ss1_forward_noalloc
+    assert fwd(768, 768, 3, 64, 64, 0, None, None, None, 1, 0, None, None) == -1         # c
+    assert fwd(768, 768, 2, 64, 64, 0, None, None, None, -1, 0, None, None) == -1        # M < 0
+    assert fwd(8192, 16384, 2, 128, 128, 0, None, None, None, 1, 0, None, None) == -8    # > table limit
+    assert fwd(768, 768, 2, 64, 64, 0, None, None, None, 0, 0, None, None) == 0          # M == 0: no-op
+    assert fwd(768, 768, 2, 64, 64, 0, None, None, None, 1, 0, None, None) == -1         # null pointers
