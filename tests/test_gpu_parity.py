@@ -92,3 +92,19 @@ def test_workload_parity_sampled(L):
         must = torch.nonzero(X.float().abs().amax(dim=1) > 8.0).flatten().tolist()[:64]
     rows = sample_rows(L.M, 48, seed=L.M + L.K, must=must)
     check_layer(ss1, L, kernel=0, rows=rows, X=X, Wc=Wc)
+
+
+# Multi-wave shapes: more tiles than SMs, not a multiple of them (a partial last wave), ragged M,
+# every BK and a c of each kind; the whole output is compared with the oracle.
+MULTIWAVE = [
+    Layer("multiwave", 8192, 768, 768, 2, 128, 128, "bf16", "normal", "uniform_invsqrtk", 1),
+    Layer("multiwave", 8000, 768, 768, 2, 128, 128, "bf16", "normal", "uniform_invsqrtk", 1),
+    Layer("multiwave", 4096, 1280, 1280, 4, 128, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2),
+    Layer("multiwave", 4096, 4096, 1024, 2, 256, 128, "bf16", "normal", "normal_002", 3),
+    Layer("multiwave", 5000, 3072, 1024, 8, 256, 128, "bf16", "normal", "normal_002", 3),
+]
+
+
+@pytest.mark.parametrize("L", MULTIWAVE, ids=[f"{L.tag}:{L.BK}" for L in MULTIWAVE])
+def test_multiwave_full_parity(L):
+    check_layer(get_ss1(), L, kernel=TC)
