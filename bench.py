@@ -69,7 +69,7 @@ def layer_work(L):
 
 KERNEL_SOURCES = {
     "TC": ["ss1_tc.cu", "ss1_tc2.cu", "ss1_tc3.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
-    "SMALLM": ["ss1_smallm.cu", "ss1_internal.cuh"],
+    "SMALLM": ["ss1_dec.cu", "ss1_smallm.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
     "SIMT": ["ss1_simt.cu", "ss1_internal.cuh"],
 }
 

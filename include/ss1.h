@@ -54,7 +54,7 @@ enum ss1_kernel {
     SS1_KERNEL_AUTO = 0,
     SS1_KERNEL_TC = 1,      /* bf16: TMA + on-chip sketch + tcgen05/TMEM tensor-core GEMM */
     SS1_KERNEL_SIMT = 2,    /* bf16 or fp32: CUDA-core sketch + FMA GEMM, any valid shape */
-    SS1_KERNEL_SMALLM = 3   /* bf16, decode-sized M: streams Wc once at HBM rate */
+    SS1_KERNEL_SMALLM = 3   /* bf16, decode-sized M: streams Wc once (tensor cores for BN = 128) */
 };
 
 enum ss1_status {
@@ -102,8 +102,9 @@ SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, in
  * ss1_forward_with -- ss1_forward with an explicit kernel (enum ss1_kernel). Same arguments,
  * ownership and errors; additionally UNSUPPORTED_SHAPE when the chosen kernel cannot run this
  * (dtype, M, shape): TC needs bf16, S = BK / c a multiple of 16, BN == 128 and K % 8 == 0;
- * SMALLM needs bf16, M <= 64, S = BK / c a power of two >= 8, BN a multiple of 8 and K, K / c
- * multiples of 8; SIMT runs every valid shape.
+ * SMALLM needs bf16, M <= 64 and K, K / c multiples of 8, and either BN == 128 (the
+ * tensor-core decode kernel) or S = BK / c a power of two >= 8 with BN a multiple of 8 (the
+ * CUDA-core one); SIMT runs every valid shape.
  */
 SS1_API int ss1_forward_with(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
                              int kernel, void* stream);
@@ -163,11 +164,13 @@ SS1_API const char* ss1_strerror(int status);
  *
  * Every call regenerates the tables on `stream` into one fixed region of device memory
  * that the library reserves statically (16 MiB per device: 17 bytes per table entry plus
- * padding), then runs the kernel ss1_forward would choose. Shapes with
- * (N / BN) * K > SS1_NOALLOC_MAX_ENTRIES are rejected with UNSUPPORTED_SHAPE. No
+ * padding), then runs the kernel ss1_forward would choose. The decode-sized path (M <= 64)
+ * splits K across CTAs as it does for a handle, with a second static region of 12 MiB for the
+ * fp32 partials and 3 KiB of arrival counters; the call clears those counters on `stream`.
+ * Shapes with (N / BN) * K > SS1_NOALLOC_MAX_ENTRIES are rejected with UNSUPPORTED_SHAPE. No
  * cudaMalloc, cudaFree, pinned allocation or allocating library routine is called, and
- * nothing synchronises the device; the region needs no zeroing because the table kernels
- * write all of it that the forward reads.
+ * nothing synchronises the device; the tables need no zeroing because the table kernels
+ * write all of them that the forward reads.
  *
  * The first call on a device does one-time set-up (it looks up the region's address and
  * sets kernel attributes); make that first call outside any stream capture.

@@ -28,6 +28,8 @@ void release(ss1_layer* L) {
     if (L->d_src) cudaFree(L->d_src);
     if (L->d_gather) cudaFree(L->d_gather);
     if (L->d_slot) cudaFree(L->d_slot);
+    if (L->d_dec_ws) cudaFree(L->d_dec_ws);
+    if (L->d_dec_cnt) cudaFree(L->d_dec_cnt);
     if (L->status_host) cudaFreeHost(L->status_host);
     L->magic = 0;
     delete L;
@@ -106,6 +108,19 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
         return SS1_ERR_OUT_OF_MEMORY;
     }
     *L->status_host = 0;
+    if (ss1::dec_supported(*L, 1) && L->NB <= L->num_sms) {   // K-split partials of the decode kernel
+        if (cudaMalloc(&L->d_dec_ws, ss1::dec_workspace_floats(*L) * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&L->d_dec_cnt, (size_t)L->NB * 4 * sizeof(uint32_t)) != cudaSuccess) {
+            cudaGetLastError();
+            release(L);
+            return SS1_ERR_OUT_OF_MEMORY;
+        }
+        if (cudaMemset(L->d_dec_cnt, 0, (size_t)L->NB * 4 * sizeof(uint32_t)) != cudaSuccess) {
+            cudaGetLastError();
+            release(L);
+            return SS1_ERR_CUDA;
+        }
+    }
     if (cudaHostGetDevicePointer((void**)&L->status_dev, L->status_host, 0) != cudaSuccess) {
         cudaGetLastError();
         release(L);

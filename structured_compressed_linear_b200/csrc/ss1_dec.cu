@@ -1,0 +1,355 @@
+// Tensor-core SS1 forward for decode-sized batches (M <= 64 rows, bf16, N-blocks of 128).
+//
+// "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+// "Approach": the input is sketched (signed hashed additions shrink each K-chunk by c) and the
+// sketch is multiplied with the compressed weights. With a few rows the product is bound by
+// reading Wc (N x K/c bf16) once. Here the 128 neurons of an N-block are the UMMA's M:
+//
+//     D[n, m] += Wc[n, j] * Xs_nb[m, j]      (A = Wc, streamed by TMA; B = the rows' sketch)
+//
+// with UMMA N = the row count rounded up to 16, so the tensor pipe is busy a few percent of the
+// time and the kernel is a TMA stream of Wc.
+//
+// CTA = (N-block nb, K-split s): the split's stages of 64 compressed columns.
+//   warp 0     : TMA loads of Wc stages [128 neurons x 64 columns] (128-byte swizzle) into a ring.
+//   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage.
+//   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
+//                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
+//                stages, warps 4-5 the odd ones); then the epilogue.
+// Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: every warp writes its
+// 32 neurons' fp32 partial to the workspace and counts itself in; the last warp to arrive for
+// those neurons sums all splits' partials in split order (the same bits every call), writes Y
+// and resets its counter.
+// Every wait is bounded; a wait that runs out sets the CTA's abort flag and the status word.
+#include "ss1_internal.cuh"
+#include "ptx_sm100.cuh"
+
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace ss1 {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+namespace {
+
+constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
+constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
+constexpr int kWStage = kNeu * kStageC * 2;   // 16 KB of Wc per stage
+constexpr int kNW = 5;                    // Wc stages in the ring
+constexpr int kNB = 3;                    // sketch stages in the ring
+constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
+constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+template <int MP>
+struct DecCfg {
+    static constexpr int B_STAGE = MP * 128;                    // [MP rows x 64] bf16
+    static constexpr int OFF_W = 0;
+    static constexpr int OFF_B = kNW * kWStage;
+    static constexpr int OFF_BAR = OFF_B + kNB * B_STAGE;
+    static constexpr int NBAR = 2 * kNW + 2 * kNB + 1;
+    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = MP <= 32 ? 32 : 64;
+    static_assert(MP % 16 == 0 && MP >= 16 && MP <= 64, "UMMA N for M = 128");
+    static_assert(B_STAGE % 1024 == 0 && OFF_B % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+__device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
+    *abort_flag = 1;
+    *(volatile int32_t*)status = (kStatusKernelDec << 8) | (0x80 + site);
+    __threadfence_system();
+}
+
+// Lane 0 waits, the warp follows.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, kWaitNs);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+template <int MP, int C>
+__global__ void __launch_bounds__(kThreads, 2)
+    dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ X,
+               __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src, int M, int K, int N, int S, int KC,
+               int splits, float* __restrict__ ws, uint32_t* __restrict__ cnt, int32_t* status) {
+    using F = DecCfg<MP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* wring = smem + F::OFF_W;
+    uint8_t* bring = smem + F::OFF_B;
+    uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
+    uint64_t* w_empty = w_full + kNW;
+    uint64_t* b_full = w_empty + kNW;     // the two build warps of the stage have written it
+    uint64_t* b_empty = b_full + kNB;     // the stage's UMMAs have completed
+    uint64_t* acc_full = b_empty + kNB;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nb = blockIdx.x, split = blockIdx.y;
+    const int Kc = K / C;
+    const int nstg = (Kc + kStageC - 1) / kStageC;
+    const int st0 = (int)((int64_t)nstg * split / splits), st1 = (int)((int64_t)nstg * (split + 1) / splits);
+    const int G = st1 - st0;   // stages of this CTA (>= 1)
+
+    // sketch stages start zeroed: rows past M are never written afterwards
+    for (int i = threadIdx.x; i < kNB * F::B_STAGE / 16; i += kThreads)
+        reinterpret_cast<uint4*>(bring)[i] = make_uint4(0u, 0u, 0u, 0u);
+    ptx::fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
+        for (int i = 0; i < kNB; ++i) { ptx::mbar_init(&b_full[i], kBuildWarps / 2); ptx::mbar_init(&b_empty[i], 1); }
+        ptx::mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(tmem_slot, F::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (warp == kWarpLoad && lane == 0) ptx::prefetch_tmap(&tmap_w);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    if (warp == kWarpLoad) {
+        // ------------------------------------------------------------------ TMA loads of Wc
+        if (lane == 0) {
+            int issued = 0;
+            for (int g = 0; g < G; ++g) {
+                const int slot = g % kNW;
+                if (g >= kNW && !ptx::mbar_wait(&w_empty[slot], (uint32_t)(((g / kNW) - 1) & 1), abort_flag, kWaitNs)) {
+                    report(status, abort_flag, 1);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&w_full[slot], kWStage);
+                ptx::tma_load_2d(wring + slot * kWStage, &tmap_w, &w_full[slot], (st0 + g) * kStageC, nb * kNeu);
+                ++issued;
+            }
+            if (*abort_flag) {   // every issued copy lands before exit
+                volatile int no_abort = 0;
+                for (int g = issued > kNW ? issued - kNW : 0; g < issued; ++g)
+                    ptx::mbar_wait(&w_full[g % kNW], (uint32_t)((g / kNW) & 1), &no_abort, kWaitNs);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------------------ UMMAs
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, MP);
+        const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, 1024, ptx::kLayoutSW128);
+        const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, ptx::kLayoutSW128);
+        bool ok = true;
+        for (int g = 0; g < G && ok; ++g) {
+            const int ws_ = g % kNW, bs = g % kNB;
+            if (!warp_wait(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag) ||
+                !warp_wait(&b_full[bs], (uint32_t)((g / kNB) & 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 2);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                const uint64_t wd = wdesc0 + (uint64_t)((ws_ * kWStage) >> 4);
+                const uint64_t bd = bdesc0 + (uint64_t)((bs * F::B_STAGE) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kStageC / 16; ++kk)
+                    ptx::umma_bf16_ss(tm, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
+                ptx::umma_commit(&w_empty[ws_]);
+                ptx::umma_commit(&b_empty[bs]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            ptx::umma_commit(acc_full);
+            if (*abort_flag) {   // the UMMAs in flight finish before TMEM is released
+                volatile int no_abort = 0;
+                ptx::mbar_wait(acc_full, 0, &no_abort, kWaitNs);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ sketch, then epilogue
+        // Build thread t: column kl = t % 64 of the stages g with g % 2 == t / 64 (two stages are
+        // built at once), all rows. A thread's table entries are loaded one of its stages ahead,
+        // so that a stage waits only for its X gathers, which are all in flight together.
+        const int t = threadIdx.x - kFirstBuild * 32;
+        const int kl = t % kStageC, half = t / kStageC;
+        const int BK = S * C;
+        const uint16_t* tab = src + (size_t)nb * KC * S * C;   // this N-block's entries, column-major order
+        auto fetch = [&](int g, uint16_t (&e)[C]) {
+            const int j = (st0 + g) * kStageC + kl;
+            if (g < G && j < Kc) {
+#pragma unroll
+                for (int q = 0; q < C; ++q) e[q] = __ldg(tab + (size_t)j * C + q);
+            }
+        };
+        uint16_t ent[C];
+        fetch(half, ent);
+        bool ok = true;
+        for (int g = half; g < G; g += 2) {
+            const int bs = g % kNB;
+            uint16_t cur[C];
+#pragma unroll
+            for (int q = 0; q < C; ++q) cur[q] = ent[q];
+            fetch(g + 2, ent);
+            if (g >= kNB && !warp_wait(&b_empty[bs], (uint32_t)(((g / kNB) - 1) & 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 3);
+                ok = false;
+                break;
+            }
+            uint8_t* stage = bring + bs * F::B_STAGE;
+            const int j = (st0 + g) * kStageC + kl;   // compressed column
+            if (j < Kc) {
+                const __nv_bfloat16* xk = X + (size_t)(j / S) * BK;   // the column's K-chunk
+#pragma unroll
+                for (int m = 0; m < MP; ++m) {
+                    if (m < M) {
+                        float v = 0.f;
+#pragma unroll
+                        for (int q = 0; q < C; ++q) {
+                            const float x = __bfloat162float(xk[(size_t)m * K + (cur[q] & kSrcIdxMask)]);
+                            v += (cur[q] & kSrcNegBit) ? -x : x;
+                        }
+                        *reinterpret_cast<__nv_bfloat16*>(stage + m * 128 + (((kl >> 3) ^ (m & 7)) << 4) + (kl & 7) * 2) =
+                            __float2bfloat16_rn(v);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < MP; ++m)
+                    if (m < M)
+                        *reinterpret_cast<uint16_t*>(stage + m * 128 + (((kl >> 3) ^ (m & 7)) << 4) + (kl & 7) * 2) = 0;
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&b_full[bs]);
+        }
+        // epilogue: warp (quad) holds neurons nb * 128 + quad * 32 + lane
+        const int quad = warp & 3;
+        if (ok && warp_wait(acc_full, 0, abort_flag) && !*abort_flag) {
+            ptx::tc_fence_after();
+            const int n = nb * kNeu + quad * 32 + lane;
+            float d[MP];
+#pragma unroll
+            for (int m0 = 0; m0 < MP; m0 += 16) {
+                uint32_t r[16];
+                ptx::tmem_ld_32x32b_x16(tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)m0, r);
+                ptx::tmem_ld_wait();
+                ptx::tmem_ld_fence_regs<16>(r);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) d[m0 + i] = __uint_as_float(r[i]);
+            }
+            if (splits == 1) {
+#pragma unroll
+                for (int m = 0; m < MP; ++m)
+                    if (m < M) Y[(size_t)m * N + n] = __float2bfloat16_rn(d[m]);
+            } else {
+                // workspace: [N-block][split][MP rows][128 neurons] fp32
+                float* mine = ws + ((size_t)(nb * splits + split) * MP) * kNeu + quad * 32 + lane;
+#pragma unroll
+                for (int m = 0; m < MP; ++m)
+                    if (m < M) mine[(size_t)m * kNeu] = d[m];
+                __threadfence();
+                __syncwarp();
+                uint32_t prev = 0;
+                if (lane == 0) prev = atomicAdd(&cnt[nb * 4 + quad], 1u);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == (uint32_t)(splits - 1)) {   // the last split of these neurons: reduce in order
+                    __threadfence();
+                    const float* base = ws + ((size_t)nb * splits * MP) * kNeu + quad * 32 + lane;
+#pragma unroll 1
+                    for (int m = 0; m < M && m < MP; ++m) {
+                        float v = 0.f;
+                        for (int s = 0; s < splits; ++s) v += __ldcg(base + ((size_t)s * MP + m) * kNeu);
+                        Y[(size_t)m * N + n] = __float2bfloat16_rn(v);
+                    }
+                    __syncwarp();
+                    if (lane == 0) cnt[nb * 4 + quad] = 0u;
+                }
+            }
+        } else if (lane == 0 && !*abort_flag) {
+            report(status, abort_flag, 4);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tm, F::TMEM_COLS);
+    }
+}
+
+bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {kStageC, kNeu};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MP, int C>
+cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    using F = DecCfg<MP>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(dec_kernel<MP, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mw;
+    if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N)) return cudaErrorInvalidValue;
+    // K-splits: about two CTAs per SM over all N-blocks, each with at least one stage; a split
+    // needs the layer's workspace
+    const int nstg = (int)((L.K / L.c + kStageC - 1) / kStageC);
+    int splits = 1;
+    if (L.d_dec_ws != nullptr) {
+        splits = (2 * L.num_sms) / L.NB;
+        if (splits > nstg) splits = nstg;
+        if (splits < 1) splits = 1;
+    }
+    const dim3 grid((unsigned)L.NB, (unsigned)splits);
+    dec_kernel<MP, C><<<grid, kThreads, F::SMEM, st>>>(mw, (const __nv_bfloat16*)X, (__nv_bfloat16*)Y, L.d_src, (int)M,
+                                                       (int)L.K, (int)L.N, L.S, L.KC, splits, L.d_dec_ws, L.d_dec_cnt,
+                                                       L.status_dev);
+    return cudaGetLastError();
+}
+
+template <int MP>
+cudaError_t launch_c(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    switch (L.c) {
+        case 1: return launch_cfg<MP, 1>(L, X, Wc, Y, M, st);
+        case 2: return launch_cfg<MP, 2>(L, X, Wc, Y, M, st);
+        case 4: return launch_cfg<MP, 4>(L, X, Wc, Y, M, st);
+        default: return launch_cfg<MP, 8>(L, X, Wc, Y, M, st);
+    }
+}
+
+}  // namespace
+
+bool dec_supported(const ss1_layer& L, int64_t M) {
+    if (M < 1 || M > 64) return false;
+    if (L.BN != kNeu) return false;
+    if (L.K % 8 != 0 || (L.K / L.c) % 8 != 0) return false;
+    return true;
+}
+
+size_t dec_workspace_floats(const ss1_layer& L) {
+    // splits > 1 only where NB <= num_sms, and then NB * splits <= 2 * num_sms slots of 64 x 128
+    return (size_t)(2 * L.num_sms) * 64 * kNeu;
+}
+
+cudaError_t launch_dec(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if (M <= 16) return launch_c<16>(L, X, Wc, Y, M, st);
+    if (M <= 32) return launch_c<32>(L, X, Wc, Y, M, st);
+    return launch_c<64>(L, X, Wc, Y, M, st);
+}
+
+}  // namespace ss1

@@ -26,6 +26,10 @@ struct ss1_layer {
     uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
     uint2* d_gather;     // [NB][KC][BK] per source (slot-major): {k, bf16x2 multiplier (+-1, +-1)}
     uint16_t* d_slot;    // [NB][K] per input: slot inside its chunk (bits 0..7) | kSrcNegBit if the sign is -1
+    // Decode-path workspace (NULL: K is not split): fp32 partials of K-split CTAs, and one arrival
+    // counter per (N-block, 32-neuron quarter), zero between calls.
+    float* d_dec_ws;
+    uint32_t* d_dec_cnt;
     int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
     int32_t* status_dev;   // device alias of status_host
 };
@@ -33,7 +37,7 @@ struct ss1_layer {
 namespace ss1 {
 
 // Device status codes written by kernels with bounded waits: (kernel id << 8) | wait site.
-enum : int32_t { kStatusKernelTC = 1 };
+enum : int32_t { kStatusKernelTC = 1, kStatusKernelDec = 2 };
 
 // The kernel ss1_forward picks for (M, dtype) (SS1_KERNEL_TC, _SIMT or _SMALLM).
 int auto_kernel(const ss1_layer& L, int64_t M, int dtype);
@@ -48,7 +52,11 @@ cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st);
 cudaError_t launch_simt(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
                         cudaStream_t st);
 
-// Decode-sized M (bf16): streams Wc once.
+// Decode-sized M (bf16): streams Wc once. The tensor-core decode kernel takes N-blocks of 128;
+// the CUDA-core one the rest.
+bool dec_supported(const ss1_layer& L, int64_t M);
+size_t dec_workspace_floats(const ss1_layer& L);
+cudaError_t launch_dec(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 bool smallm_supported(const ss1_layer& L, int64_t M);
 cudaError_t launch_smallm(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M,
                           cudaStream_t st);

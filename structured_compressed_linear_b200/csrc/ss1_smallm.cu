@@ -210,6 +210,7 @@ cudaError_t launch_rows(const ss1_layer& L, const void* X, const void* Wc, void*
 
 bool smallm_supported(const ss1_layer& L, int64_t M) {
     if (M < 1 || M > kMaxRows) return false;
+    if (dec_supported(L, M)) return true;
     if (L.BN % 8 != 0) return false;
     const int lgS = log2_exact(L.S);
     if (lgS < 3 || (1 << lgS) > kSegC) return false;          // S a power of two in [8, kSegC]
@@ -218,6 +219,7 @@ bool smallm_supported(const ss1_layer& L, int64_t M) {
 }
 
 cudaError_t launch_smallm(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if (dec_supported(L, M)) return launch_dec(L, X, Wc, Y, M, st);
     if (M <= 1) return launch_rows<1>(L, X, Wc, Y, M, st);
     if (M <= 2) return launch_rows<2>(L, X, Wc, Y, M, st);
     if (M <= 4) return launch_rows<4>(L, X, Wc, Y, M, st);
