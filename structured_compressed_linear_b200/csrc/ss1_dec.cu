@@ -11,11 +11,13 @@
 // time and the kernel is a TMA stream of Wc.
 //
 // CTA = (N-block nb, K-split s): the split's stages of 64 compressed columns.
-//   warp 0     : TMA loads of Wc stages [128 neurons x 64 columns] (128-byte swizzle) into a ring.
+//   warp 0     : TMA loads of Wc stages [128 neurons x 64 columns] (128-byte swizzle) into a ring,
+//                one issuing lane per ring slot.
 //   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage.
 //   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
 //                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
-//                stages, warps 4-5 the odd ones); then the epilogue.
+//                stages, warps 4-5 the odd ones), gathering from a shared-memory copy of the
+//                CTA's X columns where that fits in 20 KB; then the epilogue.
 // Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: every warp writes its
 // 32 neurons' fp32 partial to the workspace and counts itself in; the last warp to arrive for
 // those neurons sums all splits' partials in split order (the same bits every call), writes Y
@@ -38,7 +40,8 @@ namespace {
 constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
 constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
 constexpr int kWStage = kNeu * kStageC * 2;   // 16 KB of Wc per stage
-constexpr int kNW = 5;                    // Wc stages in the ring
+constexpr int kNW = 4;                    // Wc stages in the ring
+constexpr int kXBytes = 20 * 1024;       // X of a CTA's input range, staged when it fits
 constexpr int kNB = 3;                    // sketch stages in the ring
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
@@ -49,7 +52,8 @@ struct DecCfg {
     static constexpr int B_STAGE = MP * 128;                    // [MP rows x 64] bf16
     static constexpr int OFF_W = 0;
     static constexpr int OFF_B = kNW * kWStage;
-    static constexpr int OFF_BAR = OFF_B + kNB * B_STAGE;
+    static constexpr int OFF_X = OFF_B + kNB * B_STAGE;
+    static constexpr int OFF_BAR = OFF_X + kXBytes;
     static constexpr int NBAR = 2 * kNW + 2 * kNB + 1;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = MP <= 32 ? 32 : 64;
@@ -118,10 +122,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kWarpLoad) {
         // ------------------------------------------------------------------ TMA loads of Wc
-        if (lane == 0) {
+        // Lane l owns ring slot l (stages l, l + kNW, ...): the copies of one issuing thread are
+        // served one after another, so kNW threads keep kNW stages coming from HBM at once.
+        if (lane < kNW) {
+            const int slot = lane;
             int issued = 0;
-            for (int g = 0; g < G; ++g) {
-                const int slot = g % kNW;
+            for (int g = slot; g < G; g += kNW) {
                 if (g >= kNW && !ptx::mbar_wait(&w_empty[slot], (uint32_t)(((g / kNW) - 1) & 1), abort_flag, kWaitNs)) {
                     report(status, abort_flag, 1);
                     break;
@@ -130,10 +136,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ptx::tma_load_2d(wring + slot * kWStage, &tmap_w, &w_full[slot], (st0 + g) * kStageC, nb * kNeu);
                 ++issued;
             }
-            if (*abort_flag) {   // every issued copy lands before exit
+            if (*abort_flag && issued > 0) {   // this slot's last copy lands before exit
                 volatile int no_abort = 0;
-                for (int g = issued > kNW ? issued - kNW : 0; g < issued; ++g)
-                    ptx::mbar_wait(&w_full[g % kNW], (uint32_t)((g / kNW) & 1), &no_abort, kWaitNs);
+                ptx::mbar_wait(&w_full[slot], (uint32_t)((issued - 1) & 1), &no_abort, kWaitNs);
             }
         }
     } else if (warp == kWarpMma) {
@@ -186,6 +191,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int q = 0; q < C; ++q) e[q] = __ldg(tab + (size_t)j * C + q);
             }
         };
+        // The X columns of this CTA's chunks, all rows, staged once in shared memory when they fit
+        // (then every gather is a shared-memory read); else the gathers go to L1 / L2.
+        const int kc_lo = (st0 * kStageC) / S;
+        const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
+        const int R = (kc_hi - kc_lo + 1) * BK;   // inputs of the range
+        const bool staged = BK % 8 == 0 && (int64_t)M * R * 2 <= kXBytes;   // 16-byte aligned rows
+        const __nv_bfloat16* xsm = reinterpret_cast<const __nv_bfloat16*>(smem + F::OFF_X);
+        if (staged) {
+            const int r8 = R / 8;
+            for (int i = t; i < M * r8; i += kBuildWarps * 32) {
+                const int m = i / r8, c8 = i - m * r8;
+                *reinterpret_cast<uint4*>(smem + F::OFF_X + ((size_t)m * R + c8 * 8) * 2) =
+                    __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + (size_t)kc_lo * BK + c8 * 8));
+            }
+            ptx::named_barrier_sync(1, kBuildWarps * 32);   // the build warps only
+        }
         uint16_t ent[C];
         fetch(half, ent);
         bool ok = true;
@@ -203,14 +224,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint8_t* stage = bring + bs * F::B_STAGE;
             const int j = (st0 + g) * kStageC + kl;   // compressed column
             if (j < Kc) {
-                const __nv_bfloat16* xk = X + (size_t)(j / S) * BK;   // the column's K-chunk
+                const int kc = j / S;   // the column's K-chunk
+                const __nv_bfloat16* xk = staged ? xsm + (size_t)(kc - kc_lo) * BK : X + (size_t)kc * BK;
+                const size_t row = staged ? (size_t)R : (size_t)K;
 #pragma unroll
                 for (int m = 0; m < MP; ++m) {
                     if (m < M) {
                         float v = 0.f;
 #pragma unroll
                         for (int q = 0; q < C; ++q) {
-                            const float x = __bfloat162float(xk[(size_t)m * K + (cur[q] & kSrcIdxMask)]);
+                            const float x = __bfloat162float(xk[(size_t)m * row + (cur[q] & kSrcIdxMask)]);
                             v += (cur[q] & kSrcNegBit) ? -x : x;
                         }
                         *reinterpret_cast<__nv_bfloat16*>(stage + m * 128 + (((kl >> 3) ^ (m & 7)) << 4) + (kl & 7) * 2) =
