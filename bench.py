@@ -1,6 +1,6 @@
 """Benchmark of the SS1 layer forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID] [--m ROWS]
 
 One step = the forward of every layer of the workload (default: the four GPT-2 Small shaped
 SS1 layers, M = 8192 tokens, c = 2, BK = BN = 128, bf16 with fp32 accumulation) on seeded
@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=None)
+    ap.add_argument("--m", type=int, default=None,
+                    help="time the workload's layers with this row count (default: its largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -282,7 +284,11 @@ def main():
     from structured_compressed_linear_b200.workloads import WORKLOADS, BENCH_WORKLOAD
     wid = args.workload or BENCH_WORKLOAD
     layers = WORKLOADS[wid]
-    if len({L.M for L in layers}) != 1:
+    if args.m is not None:
+        layers = [L for L in layers if L.M == args.m]
+        if not layers:
+            raise SystemExit(f"workload {wid} has no layers with M = {args.m}")
+    elif len({L.M for L in layers}) != 1:
         layers = [L for L in layers if L.M == max(x.M for x in layers)]
 
     if args.impl == "reference":
