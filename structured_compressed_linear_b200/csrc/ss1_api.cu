@@ -4,6 +4,7 @@
 
 #include <mutex>
 #include <new>
+#include <unordered_map>
 #include <unordered_set>
 
 namespace {
@@ -45,6 +46,20 @@ int kernel_for(const ss1_layer& L, int64_t M, int dtype) {
 }  // namespace
 
 namespace ss1 {
+
+cudaError_t smem_attr_once(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::unordered_map<const void*, uint64_t> done;   // kernel -> bit d set once device d has it
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    uint64_t& mask = done[kernel];
+    if (dev < 64 && ((mask >> dev) & 1u)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev < 64) mask |= (uint64_t)1 << dev;
+    return e;
+}
 
 int auto_kernel(const ss1_layer& L, int64_t M, int dtype) { return kernel_for(L, M, dtype); }
 

@@ -321,11 +321,7 @@ bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows
 template <int MP, int C>
 cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     using F = DecCfg<MP>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(dec_kernel<MP, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
-    });
+    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&dec_kernel<MP, C>), F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mw;
     if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N)) return cudaErrorInvalidValue;

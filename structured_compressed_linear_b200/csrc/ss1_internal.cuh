@@ -44,6 +44,10 @@ int auto_kernel(const ss1_layer& L, int64_t M, int dtype);
 // The shape checks of ss1_create.
 bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN);
 
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device. The attribute
+// belongs to a device context, so it is set once per (kernel, device); later calls return at once.
+cudaError_t smem_attr_once(const void* kernel, int bytes);
+
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);
 // Derives d_gather from d_src (run after launch_hashgen).
 cudaError_t launch_gather_tables(const ss1_layer& L, cudaStream_t st);

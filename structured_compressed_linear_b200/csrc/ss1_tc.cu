@@ -326,11 +326,7 @@ template <int BK, int C>
 cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     using F = Cfg<BK, C>;
     constexpr int S = F::S;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(tc_kernel<BK, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
-    });
+    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tc_kernel<BK, C>), F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mx, mw;
     const CUtensorMapSwizzle wsw = S >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B

@@ -495,11 +495,7 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
 template <int BK, int C>
 cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     using F = Cfg<BK, C>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(tc2_kernel<BK, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
-    });
+    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tc2_kernel<BK, C>), F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mx;
     if (!make_map(&mx, X, (uint64_t)L.K, (uint64_t)M, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
