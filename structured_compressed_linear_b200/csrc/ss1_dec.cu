@@ -16,8 +16,10 @@
 //   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage.
 //   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
 //                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
-//                stages, warps 4-5 the odd ones), gathering from a shared-memory copy of the
-//                CTA's X columns where that fits in 20 KB; then the epilogue.
+//                stages, warps 4-5 the odd ones), gathering from shared memory: for up to 16 rows
+//                and K-chunks of whole stages, each chunk's X rows arrive by TMA (one more lane
+//                of warp 0) into a two-chunk ring; otherwise the CTA's X columns are copied in
+//                once where they fit in 20 KB, or the gathers go to L1 / L2. Then the epilogue.
 // Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: every warp writes its
 // 32 neurons' fp32 partial to the workspace and counts itself in; the last warp to arrive for
 // those neurons sums all splits' partials in split order (the same bits every call), writes Y
@@ -41,7 +43,9 @@ constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
 constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
 constexpr int kWStage = kNeu * kStageC * 2;   // 16 KB of Wc per stage
 constexpr int kNW = 4;                    // Wc stages in the ring
-constexpr int kXBytes = 20 * 1024;       // X of a CTA's input range, staged when it fits
+constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
+constexpr int kXChunkRows = 16;          // chunk mode: rows of an X chunk box (M <= 16)
+constexpr int kXChunkBytes = kXChunkRows * 256 * 2;   // one [16 rows x BK <= 256] chunk
 constexpr int kNB = 3;                    // sketch stages in the ring
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
@@ -54,7 +58,7 @@ struct DecCfg {
     static constexpr int OFF_B = kNW * kWStage;
     static constexpr int OFF_X = OFF_B + kNB * B_STAGE;
     static constexpr int OFF_BAR = OFF_X + kXBytes;
-    static constexpr int NBAR = 2 * kNW + 2 * kNB + 1;
+    static constexpr int NBAR = 2 * kNW + 2 * kNB + 1 + 4;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = MP <= 32 ? 32 : 64;
     static_assert(MP % 16 == 0 && MP >= 16 && MP <= 64, "UMMA N for M = 128");
@@ -76,9 +80,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 
 template <int MP, int C>
 __global__ void __launch_bounds__(kThreads, 2)
-    dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __nv_bfloat16* __restrict__ X,
-               __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src, int M, int K, int N, int S, int KC,
-               int splits, float* __restrict__ ws, uint32_t* __restrict__ cnt, int32_t* status) {
+    dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+               const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src,
+               int M, int K, int N, int S, int KC, int splits, int chunked, float* __restrict__ ws,
+               uint32_t* __restrict__ cnt, int32_t* status) {
     using F = DecCfg<MP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,14 +94,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* b_full = w_empty + kNW;     // the two build warps of the stage have written it
     uint64_t* b_empty = b_full + kNB;     // the stage's UMMAs have completed
     uint64_t* acc_full = b_empty + kNB;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* x_full = acc_full + 1;      // [2] chunk mode: an X chunk has landed
+    uint64_t* x_empty = x_full + 2;       // [2] chunk mode: every stage of the chunk has been built
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int nb = blockIdx.x, split = blockIdx.y;
     const int Kc = K / C;
     const int nstg = (Kc + kStageC - 1) / kStageC;
-    const int st0 = (int)((int64_t)nstg * split / splits), st1 = (int)((int64_t)nstg * (split + 1) / splits);
+    // Stages [st0, st1) of this CTA. Chunk mode (M <= 16, S a multiple of 64): whole K-chunks
+    // of S / 64 stages each, so that every chunk a CTA touches is one it uses entirely.
+    const int spc = chunked ? S / kStageC : 1;   // stages per chunk (chunk mode)
+    int st0, st1;
+    if (chunked) {
+        st0 = (int)((int64_t)KC * split / splits) * spc;
+        st1 = (int)((int64_t)KC * (split + 1) / splits) * spc;
+    } else {
+        st0 = (int)((int64_t)nstg * split / splits);
+        st1 = (int)((int64_t)nstg * (split + 1) / splits);
+    }
     const int G = st1 - st0;   // stages of this CTA (>= 1)
 
     // sketch stages start zeroed: rows past M are never written afterwards
@@ -107,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < kNW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
         for (int i = 0; i < kNB; ++i) { ptx::mbar_init(&b_full[i], kBuildWarps / 2); ptx::mbar_init(&b_empty[i], 1); }
         ptx::mbar_init(acc_full, 1);
+        for (int i = 0; i < 2; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -115,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::tmem_relinquish();
     }
     if (warp == kWarpLoad && lane == 0) ptx::prefetch_tmap(&tmap_w);
+    if (warp == kWarpLoad && lane == kNW && chunked) ptx::prefetch_tmap(&tmap_x);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -139,6 +158,26 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (*abort_flag && issued > 0) {   // this slot's last copy lands before exit
                 volatile int no_abort = 0;
                 ptx::mbar_wait(&w_full[slot], (uint32_t)((issued - 1) & 1), &no_abort, kWaitNs);
+            }
+        } else if (lane == kNW && chunked) {
+            // X chunks [16 rows x BK] (rows past M read as zero) into a ring of two
+            const int nch = G / spc, ch0 = st0 / spc;
+            const int BK = S * C;
+            int issued = 0;
+            for (int u = 0; u < nch; ++u) {
+                const int xs = u & 1;
+                if (u >= 2 && !ptx::mbar_wait(&x_empty[xs], (uint32_t)(((u >> 1) - 1) & 1), abort_flag, kWaitNs)) {
+                    report(status, abort_flag, 5);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&x_full[xs], (uint32_t)(kXChunkRows * BK * 2));
+                ptx::tma_load_2d(smem + F::OFF_X + xs * kXChunkBytes, &tmap_x, &x_full[xs], (ch0 + u) * BK, 0);
+                ++issued;
+            }
+            if (*abort_flag) {
+                volatile int no_abort = 0;
+                for (int u = issued > 2 ? issued - 2 : 0; u < issued; ++u)
+                    ptx::mbar_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), &no_abort, kWaitNs);
             }
         }
     } else if (warp == kWarpMma) {
@@ -196,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int kc_lo = (st0 * kStageC) / S;
         const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
         const int R = (kc_hi - kc_lo + 1) * BK;   // inputs of the range
-        const bool staged = BK % 8 == 0 && (int64_t)M * R * 2 <= kXBytes;   // 16-byte aligned rows
+        const bool staged = !chunked && BK % 8 == 0 && (int64_t)M * R * 2 <= kXBytes;   // 16-byte aligned rows
         const __nv_bfloat16* xsm = reinterpret_cast<const __nv_bfloat16*>(smem + F::OFF_X);
         if (staged) {
             const int r8 = R / 8;
@@ -223,10 +262,18 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             uint8_t* stage = bring + bs * F::B_STAGE;
             const int j = (st0 + g) * kStageC + kl;   // compressed column
+            const int u = chunked ? g / spc : 0;      // chunk mode: the stage's chunk in this CTA
+            if (chunked && !warp_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), abort_flag)) {
+                if (lane == 0) report(status, abort_flag, 6);
+                ok = false;
+                break;
+            }
             if (j < Kc) {
                 const int kc = j / S;   // the column's K-chunk
-                const __nv_bfloat16* xk = staged ? xsm + (size_t)(kc - kc_lo) * BK : X + (size_t)kc * BK;
-                const size_t row = staged ? (size_t)R : (size_t)K;
+                const __nv_bfloat16* xk = chunked  ? xsm + (size_t)(u & 1) * (kXChunkBytes / 2)
+                                          : staged ? xsm + (size_t)(kc - kc_lo) * BK
+                                                   : X + (size_t)kc * BK;
+                const size_t row = chunked ? (size_t)BK : staged ? (size_t)R : (size_t)K;
 #pragma unroll
                 for (int m = 0; m < MP; ++m) {
                     if (m < M) {
@@ -248,7 +295,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&b_full[bs]);
+            if (lane == 0) {
+                ptx::mbar_arrive(&b_full[bs]);
+                if (chunked) ptx::mbar_arrive(&x_empty[u & 1]);   // this stage's reads of the chunk are done
+            }
         }
         // epilogue: warp (quad) holds neurons nb * 128 + quad * 32 + lane
         const int quad = warp & 3;
@@ -318,26 +368,48 @@ bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// X as [M rows x K] with [16 rows x BK] boxes, no swizzle (chunk mode; rows past M read as zero).
+bool make_map_x(CUtensorMap* map, const void* base, uint64_t K, uint64_t M, uint32_t BK) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {K, M};
+    cuuint64_t strides[1] = {K * 2};
+    cuuint32_t box[2] = {BK, (cuuint32_t)kXChunkRows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int MP, int C>
 cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     using F = DecCfg<MP>;
     const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&dec_kernel<MP, C>), F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap mw;
+    CUtensorMap mw, mx;
     if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N)) return cudaErrorInvalidValue;
-    // K-splits: about two CTAs per SM over all N-blocks, each with at least one stage; a split
-    // needs the layer's workspace
+    // Chunk mode: up to 16 rows and K-chunks of whole stages; each chunk's X rows then come by
+    // TMA into a two-chunk ring and the sketch gathers read shared memory.
+    const int chunked = (MP == kXChunkRows && L.S % kStageC == 0 && L.BK % 8 == 0 && L.BK <= 256) ? 1 : 0;
+    if (chunked) {
+        if (!make_map_x(&mx, X, (uint64_t)L.K, (uint64_t)M, (uint32_t)L.BK)) return cudaErrorInvalidValue;
+    } else {
+        mx = mw;   // unused
+    }
+    // K-splits: about two CTAs per SM over all N-blocks, each with at least one stage (chunk
+    // mode: one K-chunk); a split needs the layer's workspace
     const int nstg = (int)((L.K / L.c + kStageC - 1) / kStageC);
+    const int units = chunked ? L.KC : nstg;
     int splits = 1;
     if (L.d_dec_ws != nullptr) {
         splits = (2 * L.num_sms) / L.NB;
-        if (splits > nstg) splits = nstg;
+        if (splits > units) splits = units;
         if (splits < 1) splits = 1;
     }
     const dim3 grid((unsigned)L.NB, (unsigned)splits);
-    dec_kernel<MP, C><<<grid, kThreads, F::SMEM, st>>>(mw, (const __nv_bfloat16*)X, (__nv_bfloat16*)Y, L.d_src, (int)M,
-                                                       (int)L.K, (int)L.N, L.S, L.KC, splits, L.d_dec_ws, L.d_dec_cnt,
-                                                       L.status_dev);
+    dec_kernel<MP, C><<<grid, kThreads, F::SMEM, st>>>(mw, mx, (const __nv_bfloat16*)X, (__nv_bfloat16*)Y, L.d_src,
+                                                       (int)M, (int)L.K, (int)L.N, L.S, L.KC, splits, chunked,
+                                                       L.d_dec_ws, L.d_dec_cnt, L.status_dev);
     return cudaGetLastError();
 }
 
