@@ -17,9 +17,10 @@
 //   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
 //                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
 //                stages, warps 4-5 the odd ones), gathering from shared memory: for up to 16 rows
-//                and K-chunks of whole stages, each chunk's X rows arrive by TMA (one more lane
-//                of warp 0) into a two-chunk ring; otherwise the CTA's X columns are copied in
-//                once where they fit in 20 KB, or the gathers go to L1 / L2. Then the epilogue.
+//                the X rows of each unit (one K-chunk of whole stages, or one stage of whole
+//                K-chunks) arrive by TMA (one more lane of warp 0) into a two-unit ring;
+//                otherwise the CTA's X columns are copied in once where they fit in 20 KB, or
+//                the gathers go to L1 / L2. Then the epilogue.
 // Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: every warp writes its
 // 32 neurons' fp32 partial to the workspace and counts itself in; the last warp to arrive for
 // those neurons sums all splits' partials in split order (the same bits every call), writes Y
@@ -44,8 +45,8 @@ constexpr int kStageC = 64;               // compressed columns per stage (one 1
 constexpr int kWStage = kNeu * kStageC * 2;   // 16 KB of Wc per stage
 constexpr int kNW = 4;                    // Wc stages in the ring
 constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
-constexpr int kXChunkRows = 16;          // chunk mode: rows of an X chunk box (M <= 16)
-constexpr int kXChunkBytes = kXChunkRows * 256 * 2;   // one [16 rows x BK <= 256] chunk
+constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
+constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
 constexpr int kNB = 3;                    // sketch stages in the ring
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
@@ -57,7 +58,8 @@ struct DecCfg {
     static constexpr int OFF_W = 0;
     static constexpr int OFF_B = kNW * kWStage;
     static constexpr int OFF_X = OFF_B + kNB * B_STAGE;
-    static constexpr int OFF_BAR = OFF_X + kXBytes;
+    static constexpr int X_BYTES = MP == kXChunkRows ? 2 * kXUnitBytes : kXBytes;   // the ring, or the range
+    static constexpr int OFF_BAR = OFF_X + X_BYTES;
     static constexpr int NBAR = 2 * kNW + 2 * kNB + 1 + 4;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = MP <= 32 ? 32 : 64;
@@ -82,7 +84,7 @@ template <int MP, int C>
 __global__ void __launch_bounds__(kThreads, 2)
     dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src,
-               int M, int K, int N, int S, int KC, int splits, int chunked, float* __restrict__ ws,
+               int M, int K, int N, int S, int KC, int splits, int chunked, int ui, int bi, float* __restrict__ ws,
                uint32_t* __restrict__ cnt, int32_t* status) {
     using F = DecCfg<MP>;
     extern __shared__ uint8_t smem_raw[];
@@ -103,13 +105,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nb = blockIdx.x, split = blockIdx.y;
     const int Kc = K / C;
     const int nstg = (Kc + kStageC - 1) / kStageC;
-    // Stages [st0, st1) of this CTA. Chunk mode (M <= 16, S a multiple of 64): whole K-chunks
-    // of S / 64 stages each, so that every chunk a CTA touches is one it uses entirely.
-    const int spc = chunked ? S / kStageC : 1;   // stages per chunk (chunk mode)
+    // Stages [st0, st1) of this CTA. Chunk mode (M <= 16): whole units, a unit being the X
+    // inputs of one K-chunk of S / 64 stages (S a multiple of 64) or of one stage spanning
+    // 64 / S chunks; so every unit a CTA touches is one it uses entirely. ui = inputs per unit
+    // (contiguous in X), bi = inputs per TMA box (ui or 256).
+    const int spc = chunked ? (S >= kStageC ? S / kStageC : 1) : 1;   // stages per unit
     int st0, st1;
     if (chunked) {
-        st0 = (int)((int64_t)KC * split / splits) * spc;
-        st1 = (int)((int64_t)KC * (split + 1) / splits) * spc;
+        const int nu = S >= kStageC ? KC : nstg;
+        st0 = (int)((int64_t)nu * split / splits) * spc;
+        st1 = (int)((int64_t)nu * (split + 1) / splits) * spc;
     } else {
         st0 = (int)((int64_t)nstg * split / splits);
         st1 = (int)((int64_t)nstg * (split + 1) / splits);
@@ -160,18 +165,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ptx::mbar_wait(&w_full[slot], (uint32_t)((issued - 1) & 1), &no_abort, kWaitNs);
             }
         } else if (lane == kNW && chunked) {
-            // X chunks [16 rows x BK] (rows past M read as zero) into a ring of two
-            const int nch = G / spc, ch0 = st0 / spc;
-            const int BK = S * C;
+            // X units [16 rows x ui] (rows past M read as zero) into a ring of two, as boxes of
+            // [16 x bi] stored one after another
+            const int nun = G / spc, un0 = st0 / spc;
             int issued = 0;
-            for (int u = 0; u < nch; ++u) {
+            for (int u = 0; u < nun; ++u) {
                 const int xs = u & 1;
                 if (u >= 2 && !ptx::mbar_wait(&x_empty[xs], (uint32_t)(((u >> 1) - 1) & 1), abort_flag, kWaitNs)) {
                     report(status, abort_flag, 5);
                     break;
                 }
-                ptx::mbar_arrive_expect_tx(&x_full[xs], (uint32_t)(kXChunkRows * BK * 2));
-                ptx::tma_load_2d(smem + F::OFF_X + xs * kXChunkBytes, &tmap_x, &x_full[xs], (ch0 + u) * BK, 0);
+                ptx::mbar_arrive_expect_tx(&x_full[xs], (uint32_t)(kXChunkRows * ui * 2));
+                for (int b = 0; b < ui / bi; ++b)
+                    ptx::tma_load_2d(smem + F::OFF_X + xs * kXUnitBytes + b * (kXChunkRows * bi * 2), &tmap_x,
+                                     &x_full[xs], (un0 + u) * ui + b * bi, 0);
                 ++issued;
             }
             if (*abort_flag) {
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int kc_lo = (st0 * kStageC) / S;
         const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
         const int R = (kc_hi - kc_lo + 1) * BK;   // inputs of the range
-        const bool staged = !chunked && BK % 8 == 0 && (int64_t)M * R * 2 <= kXBytes;   // 16-byte aligned rows
+        const bool staged = !chunked && BK % 8 == 0 && (int64_t)M * R * 2 <= F::X_BYTES;   // 16-byte aligned rows
         const __nv_bfloat16* xsm = reinterpret_cast<const __nv_bfloat16*>(smem + F::OFF_X);
         if (staged) {
             const int r8 = R / 8;
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             uint8_t* stage = bring + bs * F::B_STAGE;
             const int j = (st0 + g) * kStageC + kl;   // compressed column
-            const int u = chunked ? g / spc : 0;      // chunk mode: the stage's chunk in this CTA
+            const int u = chunked ? g / spc : 0;      // chunk mode: the stage's unit in this CTA
             if (chunked && !warp_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 6);
                 ok = false;
@@ -270,10 +277,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (j < Kc) {
                 const int kc = j / S;   // the column's K-chunk
-                const __nv_bfloat16* xk = chunked  ? xsm + (size_t)(u & 1) * (kXChunkBytes / 2)
+                // chunk mode: the chunk's inputs start at ii0 within its unit, inside one box
+                const int ii0 = chunked ? kc * BK - (st0 / spc + u) * ui : 0;
+                const __nv_bfloat16* xk = chunked  ? xsm + (size_t)(u & 1) * (kXUnitBytes / 2) +
+                                                         (size_t)(ii0 / bi) * (kXChunkRows * bi) + (ii0 % bi)
                                           : staged ? xsm + (size_t)(kc - kc_lo) * BK
                                                    : X + (size_t)kc * BK;
-                const size_t row = chunked ? (size_t)BK : staged ? (size_t)R : (size_t)K;
+                const size_t row = chunked ? (size_t)bi : staged ? (size_t)R : (size_t)K;
 #pragma unroll
                 for (int m = 0; m < MP; ++m) {
                     if (m < M) {
@@ -297,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(&b_full[bs]);
-                if (chunked) ptx::mbar_arrive(&x_empty[u & 1]);   // this stage's reads of the chunk are done
+                if (chunked) ptx::mbar_arrive(&x_empty[u & 1]);   // this stage's reads of the unit are done
             }
         }
         // epilogue: warp (quad) holds neurons nb * 128 + quad * 32 + lane
@@ -369,12 +379,12 @@ bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows
 }
 
 // X as [M rows x K] with [16 rows x BK] boxes, no swizzle (chunk mode; rows past M read as zero).
-bool make_map_x(CUtensorMap* map, const void* base, uint64_t K, uint64_t M, uint32_t BK) {
+bool make_map_x(CUtensorMap* map, const void* base, uint64_t K, uint64_t M, uint32_t bi) {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {K, M};
     cuuint64_t strides[1] = {K * 2};
-    cuuint32_t box[2] = {BK, (cuuint32_t)kXChunkRows};
+    cuuint32_t box[2] = {bi, (cuuint32_t)kXChunkRows};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -390,16 +400,28 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N)) return cudaErrorInvalidValue;
     // Chunk mode: up to 16 rows and K-chunks of whole stages; each chunk's X rows then come by
     // TMA into a two-chunk ring and the sketch gathers read shared memory.
-    const int chunked = (MP == kXChunkRows && L.S % kStageC == 0 && L.BK % 8 == 0 && L.BK <= 256) ? 1 : 0;
+    const int Kc = (int)(L.K / L.c);
+    const bool whole_chunks = L.S % kStageC == 0;                          // a unit = one K-chunk
+    const bool whole_stages = kStageC % L.S == 0 && Kc % kStageC == 0;     // a unit = one stage
+    const int ui = whole_chunks ? L.BK : kStageC * L.c;                    // inputs per unit
+    const int bi = ui < 256 ? ui : 256;                                    // inputs per TMA box
+    // The one-time copy of a CTA's X columns is cheaper where it fits; the ring is for the rest.
+    const int nstg0 = (Kc + kStageC - 1) / kStageC;
+    int splits0 = L.d_dec_ws != nullptr ? (2 * L.num_sms) / L.NB : 1;
+    splits0 = splits0 < 1 ? 1 : (splits0 > nstg0 ? nstg0 : splits0);
+    const int64_t range_max = ((int64_t)(nstg0 + splits0 - 1) / splits0 * kStageC / L.S + 2) * L.BK;   // inputs
+    const bool range_fits = L.BK % 8 == 0 && M * range_max * 2 <= F::X_BYTES;
+    const int chunked = (MP == kXChunkRows && !range_fits && L.BK % 8 == 0 && (whole_chunks || whole_stages) &&
+                         ui <= 512 && ui % bi == 0) ? 1 : 0;
     if (chunked) {
-        if (!make_map_x(&mx, X, (uint64_t)L.K, (uint64_t)M, (uint32_t)L.BK)) return cudaErrorInvalidValue;
+        if (!make_map_x(&mx, X, (uint64_t)L.K, (uint64_t)M, (uint32_t)bi)) return cudaErrorInvalidValue;
     } else {
         mx = mw;   // unused
     }
     // K-splits: about two CTAs per SM over all N-blocks, each with at least one stage (chunk
     // mode: one K-chunk); a split needs the layer's workspace
     const int nstg = (int)((L.K / L.c + kStageC - 1) / kStageC);
-    const int units = chunked ? L.KC : nstg;
+    const int units = chunked ? (whole_chunks ? L.KC : nstg) : nstg;
     int splits = 1;
     if (L.d_dec_ws != nullptr) {
         splits = (2 * L.num_sms) / L.NB;
@@ -408,7 +430,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     }
     const dim3 grid((unsigned)L.NB, (unsigned)splits);
     dec_kernel<MP, C><<<grid, kThreads, F::SMEM, st>>>(mw, mx, (const __nv_bfloat16*)X, (__nv_bfloat16*)Y, L.d_src,
-                                                       (int)M, (int)L.K, (int)L.N, L.S, L.KC, splits, chunked,
+                                                       (int)M, (int)L.K, (int)L.N, L.S, L.KC, splits, chunked, ui, bi,
                                                        L.d_dec_ws, L.d_dec_cnt, L.status_dev);
     return cudaGetLastError();
 }
