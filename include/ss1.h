@@ -136,7 +136,9 @@ SS1_API int ss1_get_info(ss1_handle h, int64_t* K, int64_t* N, int* c, int* BK, 
  * synchronising. Kernels with bounded waits write a non-zero code there instead of
  * trapping when a wait runs out; the word lives in pinned host memory. Returns SS1_OK or
  * SS1_ERR_DEVICE_TIMEOUT; *detail (may be NULL) receives the raw code (kernel id and wait site).
- * Call after synchronising the stream to see the result of the work enqueued so far.
+ * Call after synchronising the stream to see the result of the work enqueued so far. When it
+ * reports a time-out it also synchronises the device and resets the decode kernel's K-split
+ * counters, which a launch that gave up may have left non-zero.
  */
 SS1_API int ss1_device_status(ss1_handle h, int32_t* detail);
 

@@ -200,6 +200,15 @@ SS1_API int ss1_device_status(ss1_handle h, int32_t* detail) {
     if (!live(h)) return SS1_ERR_BAD_HANDLE;
     const int32_t v = __atomic_exchange_n(h->status_host, 0, __ATOMIC_ACQ_REL);
     if (detail) *detail = v;
+    if (v != 0 && h->d_dec_cnt) {   // a launch that gave up may have left split counters behind
+        int prev = -1;
+        cudaGetDevice(&prev);
+        if (prev != h->device) cudaSetDevice(h->device);
+        cudaDeviceSynchronize();
+        cudaMemset(h->d_dec_cnt, 0, (size_t)h->NB * 4 * sizeof(uint32_t));
+        cudaGetLastError();
+        if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+    }
     return v == 0 ? SS1_OK : SS1_ERR_DEVICE_TIMEOUT;
 }
 
