@@ -275,21 +275,27 @@ def workload_config(layers, wid, world):
     }
 
 
+def select_layers(workload, m):
+    """The layers one bench step runs: the workload's layers at row count m, or at its largest."""
+    from structured_compressed_linear_b200.workloads import WORKLOADS, BENCH_WORKLOAD
+    wid = workload or BENCH_WORKLOAD
+    layers = WORKLOADS[wid]
+    if m is not None:
+        layers = [L for L in layers if L.M == m]
+        if not layers:
+            raise SystemExit(f"workload {wid} has no layers with M = {m}")
+    elif len({L.M for L in layers}) != 1:
+        layers = [L for L in layers if L.M == max(x.M for x in layers)]
+    return wid, layers
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    from structured_compressed_linear_b200.workloads import WORKLOADS, BENCH_WORKLOAD
-    wid = args.workload or BENCH_WORKLOAD
-    layers = WORKLOADS[wid]
-    if args.m is not None:
-        layers = [L for L in layers if L.M == args.m]
-        if not layers:
-            raise SystemExit(f"workload {wid} has no layers with M = {args.m}")
-    elif len({L.M for L in layers}) != 1:
-        layers = [L for L in layers if L.M == max(x.M for x in layers)]
+    wid, layers = select_layers(args.workload, args.m)
 
     if args.impl == "reference":
         run_reference(args, layers, wid, rank, world)

@@ -72,3 +72,6 @@ def test_argument_checks_before_device(lib):
     assert fwd(8192, 16384, 2, 128, 128, 0, None, None, None, 1, 0, None, None) == -8    # > table limit
     assert fwd(768, 768, 2, 64, 64, 0, None, None, None, 0, 0, None, None) == 0          # M == 0: no-op
     assert fwd(768, 768, 2, 64, 64, 0, None, None, None, 1, 0, None, None) == -1         # null pointers
+    # misaligned pointers are rejected before any device call (the addresses are never touched)
+    assert fwd(768, 768, 2, 64, 64, 0, 0x1008, 0x2000, 0x3000, 1, 0, None, None) == -5   # X
+    assert fwd(768, 768, 2, 64, 64, 0, 0x1000, 0x2000, 0x3000, 1, 0, 0x4002, None) == -5  # status word

@@ -1,6 +1,7 @@
 """Host-side checks of the seeded workloads and of the parity metric (no GPU)."""
 
 import numpy as np
+import pytest
 import torch
 
 from structured_compressed_linear_b200.workloads import WORKLOADS, make_inputs, instance_seed
@@ -41,3 +42,21 @@ def test_parity_metric():
     y[1, 2] += 1.0
     assert abs(row_normalised_max_err(y, ref) - 0.01) < 1e-12
     assert row_normalised_max_err(ref, ref) == 0.0
+
+
+def test_bench_layer_selection():
+    """bench.py runs a workload's largest row count by default and any of its row counts on request."""
+    import importlib.util
+    import os
+    from tests.conftest import ROOT
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    wid, layers = bench.select_layers(None, None)
+    assert wid == 2 and len(layers) == 4 and {L.M for L in layers} == {8192}
+    _, layers = bench.select_layers(4, None)
+    assert {L.M for L in layers} == {4096} and len(layers) == 8
+    _, layers = bench.select_layers(4, 1)
+    assert {L.M for L in layers} == {1} and len(layers) == 8
+    with pytest.raises(SystemExit):
+        bench.select_layers(4, 3)
