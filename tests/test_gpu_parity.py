@@ -108,3 +108,17 @@ MULTIWAVE = [
 @pytest.mark.parametrize("L", MULTIWAVE, ids=[f"{L.tag}:{L.BK}" for L in MULTIWAVE])
 def test_multiwave_full_parity(L):
     check_layer(get_ss1(), L, kernel=TC)
+
+
+# Decode rows whose X range per CTA is too large to copy once, so the decode kernel's unit mode
+# runs (each unit's X rows by TMA, boxes of 16 rows with the rows past M read as zero): fewer
+# than 16 rows, a K-chunk of whole stages (c = 2) and a stage of whole K-chunks (c = 8).
+UNITMODE = [
+    Layer("unitmode", M, 4096, 14336, c, 256, 128, "bf16", "normal", "normal_002", 3)
+    for c in (2, 8) for M in (8, 13)
+]
+
+
+@pytest.mark.parametrize("L", UNITMODE, ids=[L.tag for L in UNITMODE])
+def test_decode_unit_mode_parity(L):
+    check_layer(get_ss1(), L, kernel=SMALLM)
