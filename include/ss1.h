@@ -76,9 +76,12 @@ enum ss1_status {
  *   BK, BN : K-chunk and N-block sizes; K % BK == 0, N % BN == 0, BK % c == 0, BK <= 256.
  *   seed   : table seed (any 64-bit value).
  *   out    : receives the handle (host pointer to a handle variable).
- * Allocates device memory (tables) and one pinned host word (device status), launches the
- * table generator and synchronises. Errors: INVALID_ARG, UNSUPPORTED_DEVICE, OUT_OF_MEMORY,
- * CUDA. On error *out is set to NULL and nothing is leaked.
+ * Allocates device memory and one pinned host word (device status), launches the table
+ * generator and synchronises. The device memory is the tables (17 bytes per (N / BN) * K
+ * entry). Where BN == 128 and N / BN is at most the SM count, it is also the decode kernel's
+ * K-split scratch: 2 x SMs x 32 KiB of fp32 partials plus 16 bytes per N-block of counters.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, OUT_OF_MEMORY, CUDA. On error *out is set to NULL
+ * and nothing is leaked.
  */
 SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t seed, ss1_handle* out);
 
@@ -93,7 +96,10 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
  * Asynchronous: returns after the launch. Errors: BAD_HANDLE, INVALID_ARG, MISALIGNED
  * (X, Wc, Y must be 16-byte aligned), CUDA (launch failure), DEVICE_TIMEOUT (an earlier
  * launch on this handle reported a bounded-wait time-out; see ss1_device_status).
- * Re-entrant: the handle is read-only here, so calls may run concurrently on any streams.
+ * Decode calls (the SMALLM kernel, which AUTO picks for M <= 16) on a handle with N-blocks of
+ * 128 pass partial sums through the handle's K-split scratch: such calls on one handle must not
+ * overlap on the device (order them on one stream or with events). Every other call only reads
+ * the handle, so those may run concurrently on any streams.
  */
 SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
                         void* stream);
