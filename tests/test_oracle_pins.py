@@ -71,11 +71,27 @@ def test_fisher_yates_positions_uniform_bk128():
         assert chi2 < 30.0  # 7 dof
 
 
-def test_signs_balanced_and_independent_of_perm():
+def test_signs_balanced():
     g = O.block_signs(O.block_key(99, np.arange(2000)), 64).astype(np.int64)
     frac = (g == 1).mean()
     assert abs(frac - 0.5) < 0.01
     assert set(np.unique(g).tolist()) == {-1, 1}
+
+
+def test_signs_independent_of_permutation():
+    """A block's signs are drawn apart from its shuffle. With BK = 4 the first shuffle step
+    puts its pick j (in [0, 3]) at position 3 and no later step moves it, so perm[3] is that
+    draw's result; (perm[3], g[0]) must be uniform over its 8 cells. Signs that reuse the
+    shuffle's draws (g from draw k instead of draw BK - 1 + k) tie g[0] to j and fail."""
+    n = 40000
+    keys = O.block_key(31, np.arange(n))
+    perm = O.block_permutation(keys, 4)
+    g = O.block_signs(keys, 4)
+    cell = perm[:, 3] * 2 + (g[:, 0] > 0)
+    hist = np.bincount(cell, minlength=8)
+    exp = n / 8
+    chi2 = float(((hist - exp) ** 2 / exp).sum())
+    assert chi2 < 30.0  # 7 dof: P(chi2 > 30) ~ 1e-4
 
 
 # ---------------------------------------------------------------------------- tables
