@@ -123,11 +123,13 @@ class SS1Layer:
             raise ValueError("X and Wc must be CUDA tensors of one dtype")
         if not (X.is_contiguous() and Wc.is_contiguous()):
             raise ValueError("X and Wc must be contiguous")
+        if X.device.index != self.device or Wc.device.index != self.device:
+            raise ValueError(f"X and Wc must be on cuda:{self.device}, where the layer's tables are")
         M = X.shape[0]
         if out is None:
             out = torch.empty((M, self.N), dtype=X.dtype, device=X.device)
-        elif out.shape != (M, self.N) or out.dtype != X.dtype or not out.is_contiguous():
-            raise ValueError("out must be a contiguous [M, N] tensor of X's dtype")
+        elif out.shape != (M, self.N) or out.dtype != X.dtype or not out.is_contiguous() or out.device != X.device:
+            raise ValueError("out must be a contiguous [M, N] tensor of X's dtype on X's device")
         st = stream if stream is not None else torch.cuda.current_stream(X.device)
         _check(lib().ss1_forward_with(self.handle, X.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
                                       _dtype_code(X.dtype), int(kernel), st.cuda_stream), "ss1_forward")
@@ -179,13 +181,16 @@ def forward_noalloc(X: torch.Tensor, Wc: torch.Tensor, K: int, N: int, c: int, B
         raise ValueError("X and Wc must be CUDA tensors of one dtype")
     if not (X.is_contiguous() and Wc.is_contiguous()):
         raise ValueError("X and Wc must be contiguous")
+    if X.device != Wc.device or X.device.index != torch.cuda.current_device():
+        raise ValueError("X and Wc must be on the current CUDA device (the library runs there)")
     M = X.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=X.dtype, device=X.device)
-    elif out.shape != (M, N) or out.dtype != X.dtype or not out.is_contiguous():
-        raise ValueError("out must be a contiguous [M, N] tensor of X's dtype")
-    if device_status is not None and (device_status.dtype != torch.int32 or not device_status.is_cuda):
-        raise ValueError("device_status must be a CUDA int32 tensor")
+    elif out.shape != (M, N) or out.dtype != X.dtype or not out.is_contiguous() or out.device != X.device:
+        raise ValueError("out must be a contiguous [M, N] tensor of X's dtype on X's device")
+    if device_status is not None and (device_status.dtype != torch.int32 or device_status.device != X.device
+                                      or device_status.numel() < 1):
+        raise ValueError("device_status must be an int32 tensor on X's device")
     st = stream if stream is not None else torch.cuda.current_stream(X.device)
     status_ptr = device_status.data_ptr() if device_status is not None else None
     _check(lib().ss1_forward_noalloc(K, N, c, BK, BN, seed & 0xFFFFFFFFFFFFFFFF, X.data_ptr(), Wc.data_ptr(),
