@@ -60,3 +60,38 @@ def test_bench_layer_selection():
     assert {L.M for L in layers} == {1} and len(layers) == 8
     with pytest.raises(SystemExit):
         bench.select_layers(4, 3)
+
+
+def test_bench_work_matches_hand_values():
+    """The benchmark's per-layer work against values worked out by hand from the metric's
+    definition: actual flops = 2 M N K / c plus the M (N / BN) K (1 - 1/c) sketch additions,
+    bytes = 2 (M K + N K / c + M N) for bf16 (GFLOP and MB, rounded as written)."""
+    import importlib.util
+    import os
+    from structured_compressed_linear_b200.workloads import Layer
+    from tests.conftest import ROOT
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    cases = [  # (M, K, N, c, BK, GFLOP, MB)
+        (16384, 1280, 3840, 4, 128, 40.7, 170.2),
+        (16384, 1280, 1280, 4, 128, 13.6, 84.7),
+        (16384, 1280, 5120, 4, 128, 54.3, 213.0),
+        (4096, 4096, 4096, 2, 256, 69.0, 83.9),
+        (4096, 4096, 1024, 2, 256, 17.2, 46.1),
+        (4096, 4096, 14336, 2, 256, 241.5, 209.7),
+        (4096, 4096, 4096, 8, 256, 17.65, 71.3),
+        (4096, 4096, 1024, 8, 256, 4.4, 43.0),
+    ]
+    for M, K, N, c, BK, gflop, mb in cases:
+        L = Layer("hand", M, K, N, c, BK, 128, "bf16", "normal", "normal_002", 0)
+        dense, actual, byts = bench.layer_work(L)
+        assert dense == 2.0 * M * N * K
+        assert abs(actual / 1e9 - gflop) <= 0.05, (M, K, N, c, actual)
+        assert abs(byts / 1e6 - mb) <= 0.05, (M, K, N, c, byts)
+    # exactly, in powers of two: Llama 4096 x 4096 at M = 4096, c = 8, BK = 256 (32 N-blocks):
+    # 2 * 2^36 / 8 = 2^34 products, 2^12 * 32 * 2^12 * 7/8 = 7 * 2^26 additions;
+    # bytes 2 * (2^24 + 2^21 + 2^24)
+    L = Layer("hand", 4096, 4096, 4096, 8, 256, 128, "bf16", "normal", "normal_002", 0)
+    _, actual, byts = bench.layer_work(L)
+    assert actual == 2 ** 34 + 7 * 2 ** 26 and byts == 2 * (2 ** 24 + 2 ** 21 + 2 ** 24)
