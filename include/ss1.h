@@ -100,6 +100,10 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
  * 128 pass partial sums through the handle's K-split scratch: such calls on one handle must not
  * overlap on the device (order them on one stream or with events). Every other call only reads
  * the handle, so those may run concurrently on any streams.
+ * The tensor-core decode kernel is launched with programmatic dependent launch: it may start
+ * while the previous kernel on the stream is still running, but before that kernel completes it
+ * only prefetches Wc into L2. It reads X and the tables and writes Y only afterwards, so stream
+ * order holds as for any launch.
  */
 SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype,
                         void* stream);

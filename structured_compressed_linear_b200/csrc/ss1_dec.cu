@@ -48,9 +48,25 @@ constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input 
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
 constexpr int kNB = 3;                    // sketch stages in the ring
+constexpr int kPrefetchStages = 16;       // Wc stages asked of L2 before the previous kernel ends
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
 constexpr uint64_t kWaitNs = 2000000000ull;
+
+// L2 prefetch of one 2D tile of a tensor map: no shared memory, no completion to wait for.
+// c0 * 2 bytes must be a multiple of 16, as for a tiled load.
+__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+// Programmatic dependent launch. pdl_wait blocks until the grids this one depends on have
+// completed and their memory is visible; for a launch without the attribute it returns at once.
+// pdl_launch_dependents lets a dependent grid be scheduled once every CTA of this grid has
+// issued it or exited (the dependent still waits for this grid's completion in pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 template <int MP>
 struct DecCfg {
@@ -143,6 +159,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tm = *tmem_slot;
+
+    // The launch may overlap the end of the previous kernel on the stream (programmatic
+    // dependent launch). Until that kernel has completed, this CTA only asks L2 for the first
+    // Wc stages it will stream: a prefetch goes through L2, so it cannot return data older than
+    // what that kernel writes. Every global read and write below comes after the wait.
+    if (warp == kWarpLoad && lane == 0) {
+        for (int g = 0; g < G && g < kPrefetchStages; ++g)
+            prefetch_l2_2d(&tmap_w, (st0 + g) * kStageC, nb * kNeu);
+    }
+    if (threadIdx.x == 0) pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == kWarpLoad) {
         // ------------------------------------------------------------------ TMA loads of Wc
@@ -428,11 +455,22 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
         if (splits > units) splits = units;
         if (splits < 1) splits = 1;
     }
-    const dim3 grid((unsigned)L.NB, (unsigned)splits);
-    dec_kernel<MP, C><<<grid, kThreads, F::SMEM, st>>>(mw, mx, (const __nv_bfloat16*)X, (__nv_bfloat16*)Y, L.d_src,
-                                                       (int)M, (int)L.K, (int)L.N, L.S, L.KC, splits, chunked, ui, bi,
-                                                       L.d_dec_ws, L.d_dec_cnt, L.status_dev);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may start while the previous kernel finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)L.NB, (unsigned)splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = F::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_kernel<MP, C>, mw, mx, (const __nv_bfloat16*)X,
+                                             (__nv_bfloat16*)Y, (const uint16_t*)L.d_src, (int)M, (int)L.K, (int)L.N,
+                                             L.S, L.KC, splits, chunked, ui, bi, L.d_dec_ws, L.d_dec_cnt,
+                                             L.status_dev);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int MP>
