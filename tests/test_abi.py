@@ -75,3 +75,16 @@ def test_argument_checks_before_device(lib):
     # misaligned pointers are rejected before any device call (the addresses are never touched)
     assert fwd(768, 768, 2, 64, 64, 0, 0x1008, 0x2000, 0x3000, 1, 0, None, None) == -5   # X
     assert fwd(768, 768, 2, 64, 64, 0, 0x1000, 0x2000, 0x3000, 1, 0, 0x4002, None) == -5  # status word
+
+
+def test_binding_constants_match_header():
+    """The binding's enums and limits are the header's (a drift would mis-marshal arguments)."""
+    from structured_compressed_linear_b200 import ss1
+    text = open(os.path.join(ROOT, "include", "ss1.h")).read()
+    consts = {k: int(v) for k, v in re.findall(r"\b(SS1_\w+)\s*=\s*(-?\d+)", text)}
+    for k in ss1.Kernel:
+        assert consts[f"SS1_KERNEL_{k.name}"] == int(k)
+    for d in ss1.DType:
+        assert consts[f"SS1_DTYPE_{d.name}"] == int(d)
+    m = re.search(r"#define\s+SS1_NOALLOC_MAX_ENTRIES\s+(\d+)", text)
+    assert m and int(m.group(1)) == ss1.NOALLOC_MAX_ENTRIES
