@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -76,13 +77,23 @@ KERNEL_SOURCES = {
 }
 
 
+_COMMENT_OR_STRING = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
+
+
+def code_only(text):
+    """C++ / CUDA source without its comments and blank lines (string literals kept)."""
+    text = _COMMENT_OR_STRING.sub(lambda m: m.group(0) if m.group(0).startswith('"') else "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel_name):
-    """Hash of the sources a kernel is built from; a traffic record holds only for the same hash."""
+    """Hash of the code (comments excluded) a kernel is built from; a traffic record holds only
+    for the same hash."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "structured_compressed_linear_b200", "csrc")
     for name in KERNEL_SOURCES.get(kernel_name, []):
-        with open(os.path.join(pkg, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(pkg, name), encoding="utf-8") as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

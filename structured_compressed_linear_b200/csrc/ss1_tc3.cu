@@ -11,29 +11,33 @@
 // result is exact in the fp32 accumulator (c signed bf16 terms), rounded once to bf16. Both
 // products run on the tensor cores; the CUDA cores only build P and convert the sketch.
 //
-// Tile: 128 rows of X (UMMA M) x Q N-blocks (Q = 2 for most shapes). Per K-chunk:
-//   * X-load warp : X[m0:+128, chunk] as [128 x 64] TMA boxes (128B swizzle) into a ring.
-//   * W-load warp : the Q N-blocks' Wc[nb*128:+128, kc*S:+S] as TMA boxes into a second ring.
-//   * build warp  : writes the Q sketch matrices of the chunk, stacked as the [Q*S x BK] K-major
-//                   B operand, into a ring of zeroed panels: only the BK*Q non-zeros are written,
-//                   and cleared again before a panel is reused. Its table entries arrive through
-//                   a cp.async ring several units ahead. Once a segment's panels are written and
-//                   its X boxes have landed it raises sk_ready.
-//   * MMA warp    : sketch  D_s[128 rows x Q*S] (fp32, TMEM) = X_chunk * P^T  (BK/16 UMMAs)
-//                   main    D_j[128 rows x 128] += Xs_j (A operand from TMEM) * Wc_j^T  (S/16 UMMAs
-//                   per N-block j). The sketch of chunk i+1 is issued before the main product of
-//                   chunk i, so the tensor pipe stays busy while chunk i is converted. This warp
-//                   waits on two kinds of barrier only (sk_ready, mm_ready): an mbarrier wait
-//                   costs about as much as two N = 128 UMMAs and the tensor pipe's queue is
-//                   short, so every wait in the issuing thread is a bubble in the pipe.
+// Tile: 128 rows of X (UMMA M) x Q N-blocks (Q = 2 for most shapes); one persistent CTA per SM
+// takes tiles N-block-pair fastest. Per K-chunk:
+//   * X-load warp  : X[m0:+128, chunk] as [128 x 64] TMA boxes (128B swizzle) into a ring.
+//   * W-load warp  : the Q N-blocks' Wc[nb*128:+128, kc*S:+S] as TMA boxes into a 2-stage ring.
+//   * build warps  : one per (64-input unit, N-block) of a sketch segment (up to four). Each
+//                    writes its unit's non-zeros into the stacked [Q*S x 64] K-major panel of
+//                    the B operand (two entries per lane) and clears the previous use's entries,
+//                    whose offsets it keeps in registers. Its table entries are loaded two
+//                    segments ahead. The first N-block's warps also wait for their X box, and
+//                    all of them raise sk_ready.
+//   * sketch warp  : D_s[128 rows x Q*S] (fp32, TMEM, double-buffered) = X_chunk * P^T, BK/16
+//                    UMMAs, one commit (seg_done) per segment; every consumer derives from that
+//                    one barrier what it has freed.
 //   * 8 convert warps (two per TMEM lane quarter, one per half of the sketch columns): fp32 ->
-//                   bf16 in place in TMEM (the A-operand layout: lane = row, two consecutive slots
-//                   per 32-bit column). D_s is double-buffered. The first convert warp also waits
-//                   for the chunk's Wc (and for the accumulator at a tile's first chunk) and then
-//                   all eight raise mm_ready.
+//                    bf16 in the A-operand layout (lane = row, two consecutive slots per 32-bit
+//                    column), in place in D_s or into a separate buffer where TMEM has room. The
+//                    first also waits for the chunk's Wc. All raise mm_ready.
+//   * main warp    : D_j[128 rows x 128] += Xs_j (A operand from TMEM) * Wc_j^T, S/16 UMMAs per
+//                    N-block j. At a tile's first chunk it waits per N-block for the epilogue to
+//                    have read the accumulator. It commits the Wc stage and the sketch buffer
+//                    back. Sketch and main products come from two warps, so that one warp's
+//                    barrier waits overlap the other's UMMAs: a wait in the issuing thread drains
+//                    the tensor pipe's short queue.
 //   * 4 epilogue warps: accumulators -> bf16 (round to nearest even) -> swizzled shared-memory
-//                   staging -> TMA bulk stores of [32 rows x 32 neurons] boxes (rows past M are
-//                   clipped by the tensor map).
+//                    staging -> TMA bulk stores of [32 rows x 32 neurons] boxes (rows past M are
+//                    clipped by the tensor map); each N-block's accumulator is released as soon
+//                    as it has been read.
 // Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
 // handle's status word, drains the copies and MMAs in flight and returns (no trap).
 #include "ss1_internal.cuh"
