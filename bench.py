@@ -70,13 +70,6 @@ def layer_work(L):
     return dense, actual, byts
 
 
-KERNEL_SOURCES = {
-    "TC": ["ss1_tc.cu", "ss1_tc2.cu", "ss1_tc3.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
-    "SMALLM": ["ss1_dec.cu", "ss1_smallm.cu", "ptx_sm100.cuh", "ss1_internal.cuh"],
-    "SIMT": ["ss1_simt.cu", "ss1_internal.cuh"],
-}
-
-
 _COMMENT_OR_STRING = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
 
 
@@ -86,26 +79,34 @@ def code_only(text):
     return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
 
 
-def kernel_source_hash(kernel_name):
-    """Hash of the code (comments excluded) a kernel is built from; a traffic record holds only
-    for the same hash."""
+def source_hash(names):
+    """Hash of the code (comments and blank lines excluded) of the named files under csrc/."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "structured_compressed_linear_b200", "csrc")
-    for name in KERNEL_SOURCES.get(kernel_name, []):
+    for name in names:
         with open(os.path.join(pkg, name), encoding="utf-8") as f:
             h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel_name):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+def layer_key(L):
+    return [L.M, L.K, L.N, L.c, L.BK, L.BN]
+
+
+def traffic_record(kernel_name, layers):
+    """ncu DRAM bytes of one step of `kernel_name` over `layers`, from profiles/dram_traffic.json.
+
+    The record holds only for the layers it was taken on and for the code it was taken on: its
+    `sources` (the kernel's own files) must hash as they did then. Otherwise None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     rec = d.get(kernel_name)
-    if not rec or rec.get("source_hash") != kernel_source_hash(kernel_name):
+    if not rec or rec.get("layers") != [layer_key(L) for L in layers]:
+        return None
+    if rec.get("source_hash") != source_hash(rec.get("sources", [])):
         return None
     return rec
 
@@ -458,7 +459,7 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} (burst figure; MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    rec = traffic_record(dom)
+    rec = traffic_record(dom, [L for L, _ in dom_layers])
     roof["traffic"] = rec["dram_bytes_per_step"] if rec else None
     roof["kernel"] = dom
     roof["launches_per_step"] = kernels.count(dom)

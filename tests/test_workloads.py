@@ -95,3 +95,32 @@ def test_bench_work_matches_hand_values():
     L = Layer("hand", 4096, 4096, 4096, 8, 256, 128, "bf16", "normal", "normal_002", 0)
     _, actual, byts = bench.layer_work(L)
     assert actual == 2 ** 34 + 7 * 2 ** 26 and byts == 2 * (2 ** 24 + 2 ** 21 + 2 ** 24)
+
+
+def _bench_module():
+    import importlib.util
+    import os
+    from tests.conftest import ROOT
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    return bench
+
+
+def test_traffic_record_only_for_its_layers():
+    """The committed DRAM counters are reported for the layers they were taken on and no others."""
+    bench = _bench_module()
+    assert bench.traffic_record("TC", WORKLOADS[2]) is not None
+    assert bench.traffic_record("TC", WORKLOADS[3]) is None
+    assert bench.traffic_record("TC", [L.with_M(4096) for L in WORKLOADS[2]]) is None
+    assert bench.traffic_record("SMALLM", WORKLOADS[2]) is None
+
+
+def test_source_hash_ignores_comments_only():
+    bench = _bench_module()
+    a = 'int f() { return 1; }  // one\n/* block\n comment */\nconst char* s = "a // b /* c */";\n'
+    b = '// header\nint f() { return 1; }\n\nconst char* s = "a // b /* c */";  /* tail */\n'
+    c = 'int f() { return 2; }\nconst char* s = "a // b /* c */";\n'
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(c)
+    assert '"a // b /* c */"' in bench.code_only(a)
