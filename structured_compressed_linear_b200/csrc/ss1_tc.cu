@@ -1,22 +1,19 @@
-// Tensor-core SS1 forward for sm_100a: TMA -> on-chip sketch -> tcgen05.mma (TMEM accumulator).
+// Tensor-core SS1 forward for sm_100a at c = 1: TMA -> tcgen05.mma (TMEM accumulator) -> Y.
 //
 // "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
 // "Approach": the input is sketched (signed hashed additions shrink it by the compression
-// factor c) and then multiplied with the compressed weights; after the sketch the work is a
-// dense contraction, so it runs on the 5th-generation tensor cores.
+// factor c) and then multiplied with the compressed weights. At c = 1 the hash is the identity
+// with all signs +1, so the layer is the dense product Y = X Wc^T and the X tile itself is the
+// A operand. (c >= 2 runs in ss1_tc3.cu, or in ss1_tc2.cu for the shapes tc3 does not take;
+// launch_tc below chooses.)
 //
 // One CTA computes a 128-row x 128-column output tile = rows [m0, m0+128) of N-block nb
-// (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs, S = BK / c compressed columns):
+// (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs):
 //   * TMA warp      : X[m0:+128, kc*BK:+BK] -> smem (128B-swizzled, 64-column panels) and
-//                     Wc[nb*128:+128, kc*S:+S] -> smem (K-major, swizzle chosen by S).
-//   * sketch warps  : thread = row; Xs[row, s] = sum_j sign_j * X[row, kc*BK + k_j] in fp32,
-//                     rounded once to bf16 and written as the UMMA A operand (K-major,
-//                     same swizzle as the Wc tile). The sketch never leaves shared memory.
-//   * MMA thread    : S/16 x tcgen05.mma.kind::f16 (M=128, N=128, K=16) into one TMEM
+//                     Wc[nb*128:+128, kc*BK:+BK] -> smem (K-major, 128B swizzle).
+//   * MMA thread    : BK/16 x tcgen05.mma.kind::f16 (M=128, N=128, K=16) into one TMEM
 //                     accumulator; tcgen05.commit releases the stage.
-//   * epilogue      : the sketch warps read the fp32 accumulator with tcgen05.ld, round to
-//                     bf16 and store Y.
-// c = 1 skips the sketch: the X tile is the A operand (a plain GEMM, identity hash).
+//   * epilogue warps: read the fp32 accumulator with tcgen05.ld, round to bf16 and store Y.
 // Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the
 // handle's status word, drains the copies and MMAs in flight and returns (no trap).
 #include "ss1_internal.cuh"
@@ -35,16 +32,15 @@ namespace {
 
 constexpr int kBM = 128;         // rows per tile (UMMA M)
 constexpr int kBN = 128;         // N-block size handled (UMMA N)
-constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 sketch + epilogue
+constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kSmemBudget = 200 * 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <int BK, int C>
+template <int BK>
 struct Cfg {
-    static constexpr int S = BK / C;
+    static constexpr int S = BK;                        // c = 1: one compressed column per input
     static constexpr int X_BYTES = kBM * BK * 2;
     static constexpr int W_BYTES = kBN * S * 2;
-    static constexpr int A_BYTES = (C == 1) ? 0 : kBM * S * 2;
     static constexpr int RB = S >= 64 ? 128 : 2 * S;   // bytes per row inside one swizzle panel
     static constexpr int PANEL = 128 * RB;              // bytes of one 128-row panel
     static constexpr uint32_t LAYOUT = S >= 64 ? ptx::kLayoutSW128 : (S == 32 ? ptx::kLayoutSW64 : ptx::kLayoutSW32);
@@ -54,7 +50,7 @@ struct Cfg {
         int best_x = 1, best_w = 1, best_score = -1;
         for (int nx = 1; nx <= 4; ++nx)
             for (int nw = 1; nw <= 4; ++nw) {
-                const int bytes = nx * X_BYTES + nw * (W_BYTES + A_BYTES);
+                const int bytes = nx * X_BYTES + nw * W_BYTES;
                 if (bytes > kSmemBudget) continue;
                 const int score = (nx < nw ? nx : nw) * 16 + nx + nw;
                 if (score > best_score) { best_score = score; best_x = nx; best_w = nw; }
@@ -63,8 +59,8 @@ struct Cfg {
     }
     static constexpr int NX = stage_pick(true);
     static constexpr int NW = stage_pick(false);
-    static constexpr int NBAR = 2 * NX + 3 * NW + 1;
-    static constexpr int SMEM = NX * X_BYTES + NW * (W_BYTES + A_BYTES) + NBAR * 8 + 16 + 1024;
+    static constexpr int NBAR = 2 * NX + 2 * NW + 1;
+    static constexpr int SMEM = NX * X_BYTES + NW * W_BYTES + NBAR * 8 + 16 + 1024;
     static_assert(S % 16 == 0 && S >= 16, "UMMA K-steps of 16");
     static_assert(BK % 64 == 0, "X panels of 64 columns");
 };
@@ -75,35 +71,21 @@ __device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag
     __threadfence_system();
 }
 
-// Byte offset of element (row, col) in a K-major tile of `cols` columns stored as 128-row
-// panels of RB bytes per row with the matching TMA / UMMA swizzle.
-template <int RB>
-__device__ __forceinline__ uint32_t kmajor_offset(int row, int col) {
-    constexpr int per_panel = RB / 2;
-    const int p = col / per_panel;
-    const int cin = col % per_panel;
-    const uint32_t chunk = (uint32_t)(cin >> 3) ^ (uint32_t)(((row * RB) >> 7) & (RB / 16 - 1));
-    return (uint32_t)(p * 128 * RB + row * RB) + (chunk << 4) + (uint32_t)(cin & 7) * 2u;
-}
-
-template <int BK, int C>
+template <int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-              __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src, int M, int N, int KC,
-              int32_t* status) {
-    using F = Cfg<BK, C>;
+              __nv_bfloat16* __restrict__ Y, int M, int N, int KC, int32_t* status) {
+    using F = Cfg<BK>;
     constexpr int S = F::S, NX = F::NX, NW = F::NW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* xs = smem;
     uint8_t* ws = xs + NX * F::X_BYTES;
-    uint8_t* as = ws + NW * F::W_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(as + NW * F::A_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ws + NW * F::W_BYTES);
     uint64_t* x_full = bars;
     uint64_t* x_empty = x_full + NX;
     uint64_t* w_full = x_empty + NX;
-    uint64_t* a_full = w_full + NW;
-    uint64_t* aw_empty = a_full + NW;
+    uint64_t* aw_empty = w_full + NW;
     uint64_t* acc_full = aw_empty + NW;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -115,11 +97,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < NX; ++i) {
             ptx::mbar_init(&x_full[i], 1);
-            ptx::mbar_init(&x_empty[i], C == 1 ? 1 : 128);
+            ptx::mbar_init(&x_empty[i], 1);
         }
         for (int i = 0; i < NW; ++i) {
             ptx::mbar_init(&w_full[i], 1);
-            ptx::mbar_init(&a_full[i], 128);
             ptx::mbar_init(&aw_empty[i], 1);
         }
         ptx::mbar_init(acc_full, 1);
@@ -182,17 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int wi = kc % NW;
                 const uint32_t ph = (kc / NW) & 1;
                 if (!ptx::mbar_wait(&w_full[wi], ph, abort_flag, kWaitLimitNs)) { report(status, abort_flag, 3); break; }
-                const uint8_t* a_tile;
-                if constexpr (C == 1) {
-                    if (!ptx::mbar_wait(&x_full[kc % NX], (kc / NX) & 1, abort_flag, kWaitLimitNs)) {
-                        report(status, abort_flag, 4);
-                        break;
-                    }
-                    a_tile = xs + (kc % NX) * F::X_BYTES;
-                } else {
-                    if (!ptx::mbar_wait(&a_full[wi], ph, abort_flag, kWaitLimitNs)) { report(status, abort_flag, 4); break; }
-                    a_tile = as + wi * F::A_BYTES;
+                if (!ptx::mbar_wait(&x_full[kc % NX], (kc / NX) & 1, abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 4);
+                    break;
                 }
+                const uint8_t* a_tile = xs + (kc % NX) * F::X_BYTES;
                 ptx::tc_fence_after();
                 const uint32_t a_base = ptx::smem_u32(a_tile);
                 const uint32_t b_base = ptx::smem_u32(ws + wi * F::W_BYTES);
@@ -205,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::umma_bf16_ss(tmem_acc, ad, bd, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
                 }
                 ptx::umma_commit(&aw_empty[wi]);
-                if constexpr (C == 1) ptx::umma_commit(&x_empty[kc % NX]);
+                ptx::umma_commit(&x_empty[kc % NX]);
             }
             ptx::umma_commit(acc_full);
             if (*abort_flag) {
@@ -214,60 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------------ sketch + epilogue
+        // ------------------------------------------------------------------ epilogue
         const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
         const int row = quad * 32 + lane;       // row of the tile owned by this thread
-        if constexpr (C > 1) {
-            for (int kc = 0; kc < KC; ++kc) {
-                const int xi = kc % NX, wi = kc % NW;
-                if (!ptx::mbar_wait(&x_full[xi], (kc / NX) & 1, abort_flag, kWaitLimitNs)) {
-                    report(status, abort_flag, 5);
-                    break;
-                }
-                if (!ptx::mbar_wait(&aw_empty[wi], ((kc / NW) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
-                    report(status, abort_flag, 6);
-                    break;
-                }
-                const uint8_t* xt = xs + xi * F::X_BYTES;
-                uint8_t* at = as + wi * F::A_BYTES;
-                const uint4* tab = reinterpret_cast<const uint4*>(src + ((size_t)nb * KC + kc) * (size_t)(S * C));
-#pragma unroll 1
-                for (int s8 = 0; s8 < S / 8; ++s8) {
-                    uint4 e[C];
-#pragma unroll
-                    for (int j = 0; j < C; ++j) e[j] = __ldg(tab + s8 * C + j);
-                    const uint16_t* ent = reinterpret_cast<const uint16_t*>(e);
-                    float v[8];
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        float acc = 0.f;
-#pragma unroll
-                        for (int j = 0; j < C; ++j) {
-                            const uint16_t en = ent[t * C + j];
-                            const int k = en & kSrcIdxMask;
-                            const uint32_t off = (uint32_t)((k >> 6) * 128 * 128) + kmajor_offset<128>(row, k & 63);
-                            const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(xt + off));
-                            acc += (en & kSrcNegBit) ? -x : x;
-                        }
-                        v[t] = acc;
-                    }
-                    uint4 packed;
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]);
-                    __nv_bfloat162 p1 = __floats2bfloat162_rn(v[2], v[3]);
-                    __nv_bfloat162 p2 = __floats2bfloat162_rn(v[4], v[5]);
-                    __nv_bfloat162 p3 = __floats2bfloat162_rn(v[6], v[7]);
-                    packed.x = *reinterpret_cast<uint32_t*>(&p0);
-                    packed.y = *reinterpret_cast<uint32_t*>(&p1);
-                    packed.z = *reinterpret_cast<uint32_t*>(&p2);
-                    packed.w = *reinterpret_cast<uint32_t*>(&p3);
-                    *reinterpret_cast<uint4*>(at + kmajor_offset<F::RB>(row, s8 * 8)) = packed;
-                }
-                ptx::fence_proxy_async_smem();
-                ptx::mbar_arrive(&x_empty[xi]);
-                ptx::mbar_arrive(&a_full[wi]);
-            }
-        }
-        // epilogue
         bool ok = ptx::mbar_wait(acc_full, 0, abort_flag, kWaitLimitNs);
         if (!ok) report(status, abort_flag, 7);
         ptx::tc_fence_after();
@@ -322,11 +246,11 @@ bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
     return r == CUDA_SUCCESS;
 }
 
-template <int BK, int C>
+template <int BK>
 cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    using F = Cfg<BK, C>;
+    using F = Cfg<BK>;
     constexpr int S = F::S;
-    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tc_kernel<BK, C>), F::SMEM);
+    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tc_kernel<BK>), F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mx, mw;
     const CUtensorMapSwizzle wsw = S >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -335,8 +259,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     if (!make_map_2d(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kBN, wsw))
         return cudaErrorInvalidValue;
     dim3 grid((unsigned)L.NB, (unsigned)((M + kBM - 1) / kBM));
-    tc_kernel<BK, C><<<grid, kThreads, F::SMEM, st>>>(mx, mw, (__nv_bfloat16*)Y, L.d_src, (int)M, (int)L.N, L.KC,
-                                                      L.status_dev);
+    tc_kernel<BK><<<grid, kThreads, F::SMEM, st>>>(mx, mw, (__nv_bfloat16*)Y, (int)M, (int)L.N, L.KC, L.status_dev);
     return cudaGetLastError();
 }
 
@@ -366,21 +289,11 @@ bool tc_supported(const ss1_layer& L) {
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     if (tc3_supported(L)) return launch_tc3(L, X, Wc, Y, M, st);
     if (tc2_supported(L)) return launch_tc2(L, X, Wc, Y, M, st);
-    if ((M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
-#define SS1_TC_CASE(bk, cc) \
-    if (L.BK == bk && L.c == cc) return launch_cfg<bk, cc>(L, X, Wc, Y, M, st);
-    SS1_TC_CASE(64, 1)
-    SS1_TC_CASE(64, 2)
-    SS1_TC_CASE(64, 4)
-    SS1_TC_CASE(128, 1)
-    SS1_TC_CASE(128, 2)
-    SS1_TC_CASE(128, 4)
-    SS1_TC_CASE(128, 8)
-    SS1_TC_CASE(256, 1)
-    SS1_TC_CASE(256, 2)
-    SS1_TC_CASE(256, 4)
-    SS1_TC_CASE(256, 8)
-#undef SS1_TC_CASE
+    // c >= 2 shapes that tc_supported accepts are all taken above (tc2_supported covers them)
+    if (L.c != 1 || (M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
+    if (L.BK == 64) return launch_cfg<64>(L, X, Wc, Y, M, st);
+    if (L.BK == 128) return launch_cfg<128>(L, X, Wc, Y, M, st);
+    if (L.BK == 256) return launch_cfg<256>(L, X, Wc, Y, M, st);
     return cudaErrorInvalidValue;
 }
 
