@@ -111,7 +111,8 @@ SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, in
 /*
  * ss1_forward_with -- ss1_forward with an explicit kernel (enum ss1_kernel). Same arguments,
  * ownership and errors; additionally UNSUPPORTED_SHAPE when the chosen kernel cannot run this
- * (dtype, M, shape): TC needs bf16, S = BK / c a multiple of 16, BN == 128 and K % 8 == 0;
+ * (dtype, M, shape): TC needs bf16, BK one of 64, 128, 256, S = BK / c a multiple of 16,
+ * BN == 128, and K, K / c multiples of 8;
  * SMALLM needs bf16, M <= 64 and K, K / c multiples of 8, and either BN == 128 (the
  * tensor-core decode kernel) or S = BK / c a power of two >= 8 with BN a multiple of 8 (the
  * CUDA-core one); SIMT runs every valid shape.
