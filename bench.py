@@ -1,6 +1,7 @@
 """Benchmark of the SS1 layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID] [--m ROWS]
+    python bench.py --decode-block C [--m ROWS] [--steps K]   (one Llama-3-8B block's decode latency)
 
 One step = the forward of every layer of the workload (default: the four GPT-2 Small shaped
 SS1 layers, M = 8192 tokens, c = 2, BK = BN = 128, bf16 with fp32 accumulation) on seeded
@@ -46,6 +47,9 @@ def parse():
     ap.add_argument("--workload", type=int, default=None)
     ap.add_argument("--m", type=int, default=None,
                     help="time the workload's layers with this row count (default: its largest)")
+    ap.add_argument("--decode-block", type=int, choices=[2, 8], default=None, metavar="C",
+                    help="time one Llama-3-8B block's seven projections back to back at compression C "
+                         "(rows: --m, default 1) instead of the workload step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -223,6 +227,62 @@ def oracle_sample_rate(prepared, budget_s, rows_per_layer=None):
     return dense / dt / 1e12, dt, rows_per_layer
 
 
+# One Llama-3-8B transformer block's projections, in order: q, k, v, o, gate, up, down (K, N).
+LLAMA_BLOCK = [(4096, 4096), (4096, 1024), (4096, 1024), (4096, 4096), (4096, 14336), (4096, 14336), (14336, 4096)]
+
+
+def run_decode_block(args, peaks, peak_src, dev):
+    """Decode latency of one Llama-3-8B block: its seven projections back to back at M rows,
+    through the public API, as a model's decode step runs them. Wc is rotated over enough
+    copies that they exceed L2, so no flush runs between blocks, and one event pair brackets
+    all timed blocks. The roofline is the block's bytes (X + Wc + Y) at the HBM copy rate."""
+    import torch
+    from structured_compressed_linear_b200 import ss1
+    M, c = args.m or 1, args.decode_block
+    layers = [ss1.SS1Layer(K, N, c, 256, 128, 3) for K, N in LLAMA_BLOCK]
+    wc_bytes = sum(N * (K // c) * 2 for K, N in LLAMA_BLOCK)
+    ncopy = max(2, -(-300_000_000 // wc_bytes))
+    gen = torch.Generator(device=dev).manual_seed(3)
+    Ws = [[(torch.randn(N, K // c, device=dev, generator=gen) * 0.02).to(torch.bfloat16) for K, N in LLAMA_BLOCK]
+          for _ in range(ncopy)]
+    Xs = [torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16) for K, _ in LLAMA_BLOCK]
+    Ys = [torch.empty(M, N, device=dev, dtype=torch.bfloat16) for _, N in LLAMA_BLOCK]
+    kernels = sorted({layer.select_kernel(M).name for layer in layers})
+
+    def block(cp):
+        for i, layer in enumerate(layers):
+            layer.forward(Xs[i], Ws[cp][i], out=Ys[i])
+
+    for s in range(max(3, args.warmup) * ncopy):
+        block(s % ncopy)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.steps):
+        block(s % ncopy)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    for layer in layers:
+        st, detail = layer.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {detail:#x} after the decode block")
+    byts = wc_bytes + sum(2 * (M * K + M * N) for K, N in LLAMA_BLOCK)
+    achieved = byts / (us * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "SS1 decode block latency (Llama-3-8B q, k, v, o, gate, up, down back to back)",
+        "value": us, "unit": "us per block", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"llama-3-8b block at M={M}, c={c}, BK=256, BN=128", "kernels": kernels,
+                   "l2": f"Wc rotated over {ncopy} copies ({ncopy * wc_bytes / 1e6:.0f} MB), no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes": byts,
+                     "peak_source": peak_src},
+    }), flush=True)
+    for layer in layers:
+        layer.close()
+
+
 def run_reference(args, layers, wid, rank, world):
     if rank != 0:
         return
@@ -306,6 +366,17 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.decode_block is not None:   # a latency measurement on one GPU, not the workload step
+        if rank != 0:
+            return
+        import torch
+        from structured_compressed_linear_b200 import build
+        build.build()
+        torch.cuda.set_device(local)
+        peaks, peak_src = load_peaks()
+        run_decode_block(args, peaks, peak_src, torch.device("cuda", local))
+        return
 
     wid, layers = select_layers(args.workload, args.m)
 
