@@ -162,13 +162,14 @@ SS1_API int ss1_destroy(ss1_handle h) {
         if (!g_live.count(h) || h->magic != kMagic) return SS1_ERR_BAD_HANDLE;
         g_live.erase(h);
     }
+    const int dev = h->device;   // read before release() frees the handle
     int prev = -1;
     cudaGetDevice(&prev);
-    if (prev != h->device) cudaSetDevice(h->device);
+    if (prev != dev) cudaSetDevice(dev);
     cudaDeviceSynchronize();
     cudaGetLastError();
     release(h);
-    if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+    if (prev >= 0 && prev != dev) cudaSetDevice(prev);
     return SS1_OK;
 }
 
