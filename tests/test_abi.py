@@ -58,6 +58,7 @@ def test_argument_checks_before_device(lib):
     assert lib.ss1_create(770, 768, 2, 64, 64, 0, ctypes.byref(h)) == -1      # K % BK
     assert lib.ss1_create(768, 760, 2, 64, 40, 0, ctypes.byref(h)) == -1      # BN % 16
     assert lib.ss1_create(768, 768, 2, 64, 64, 0, None) == -1
+    assert lib.ss1_create(1 << 30, 1 << 20, 1, 256, 16, 0, ctypes.byref(h)) == -1   # > 2^31 table entries
     assert h.value is None
     # null / unknown handles
     assert lib.ss1_forward(None, None, None, None, 1, 0, None) == -7
