@@ -74,7 +74,7 @@ enum ss1_status {
  *   K, N   : input and output features, K >= 1, N >= 1.
  *   c      : compression factor, one of 1, 2, 4, 8. Wc has K / c columns.
  *   BK, BN : K-chunk and N-block sizes; K % BK == 0, N % BN == 0, BK % c == 0, BK <= 256,
- *            BN % 16 == 0, and (N / BN) * K <= 2^31 table entries.
+ *            BN % 16 == 0, and (N / BN) * K < 2^31 table entries.
  *   seed   : table seed (any 64-bit value).
  *   out    : receives the handle (host pointer to a handle variable).
  * Allocates device memory and one pinned host word (device status), launches the table

@@ -96,7 +96,7 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
     if (!(c == 1 || c == 2 || c == 4 || c == 8)) return SS1_ERR_INVALID_ARG;
     if (BK > 256 || BK % c != 0 || K % BK != 0 || N % BN != 0 || BN % 16 != 0) return SS1_ERR_INVALID_ARG;
     if (K > (int64_t)1 << 30 || N > (int64_t)1 << 30) return SS1_ERR_INVALID_ARG;
-    if ((N / BN) * K > (int64_t)1 << 31) return SS1_ERR_INVALID_ARG;   // table entries, indexed in 32 bits
+    if ((N / BN) * K >= (int64_t)1 << 31) return SS1_ERR_INVALID_ARG;   // table entries, indexed in 32 bits
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
