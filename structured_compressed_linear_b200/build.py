@@ -1,6 +1,6 @@
 """Builds the in-tree CUDA library `libss1.so` for sm_100a with nvcc.
 
-    python -m structured_compressed_linear_b200.build [--force] [--debug]
+    python -m structured_compressed_linear_b200.build [--force] [-v]
 
 Every .cu under csrc/ is compiled separately (in parallel) for sm_100a and linked into one
 shared library next to this file. The CUDA runtime is linked statically; the driver API
@@ -52,16 +52,15 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
-    if not force and not debug and up_to_date():
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
     cc = nvcc()
-    extra = ["-DSS1_DEBUG=1"] if debug else []
 
     def compile_one(src):
         obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [cc, *ARCH, *COMMON, *extra, "-c", src, "-o", obj]
+        cmd = [cc, *ARCH, *COMMON, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -85,10 +84,9 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
-    ap.add_argument("--debug", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true", help="print ptxas register/smem usage")
     a = ap.parse_args()
-    print(build(force=a.force, debug=a.debug, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose))
 
 
 if __name__ == "__main__":
