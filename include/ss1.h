@@ -198,6 +198,18 @@ SS1_API int ss1_forward_noalloc(int64_t K, int64_t N, int c, int BK, int BN, uin
                                 const void* Wc, void* Y, int64_t M, int dtype, int32_t* device_status,
                                 void* stream);
 
+/*
+ * ss1_test_device_timeout -- exercises the bounded-wait error path without a fault, for tests of
+ * failure handling (the SS1 pages have no counterpart). Launches one thread on `stream` that
+ * waits on a barrier nothing completes, with the forward kernels' bounded wait cut to
+ * limit_ns nanoseconds (1 .. 2e9). When the limit passes, the thread writes the handle's status
+ * word as a stalled forward kernel would: kernel id 3, site 1, that is (3 << 8) | 0x81. Then it
+ * returns, and the context stays usable. Afterwards ss1_forward on this handle returns
+ * SS1_ERR_DEVICE_TIMEOUT until ss1_device_status has read and cleared the word.
+ * Asynchronous. Errors: BAD_HANDLE, INVALID_ARG (limit_ns out of range), CUDA (launch failure).
+ */
+SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,8 @@ int kernel_for(const ss1_layer& L, int64_t M, int dtype) {
 
 namespace ss1 {
 
+bool handle_live(const ss1_layer* h) { return live(h); }
+
 cudaError_t smem_attr_once(const void* kernel, int bytes) {
     static std::mutex mu;
     static std::unordered_map<const void*, uint64_t> done;   // kernel -> bit d set once device d has it

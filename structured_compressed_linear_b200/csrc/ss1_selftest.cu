@@ -1,0 +1,44 @@
+// ss1_test_device_timeout: the bounded-wait error path, exercised without a fault. The SS1
+// pages have no counterpart; the entry point is specified in include/ss1.h.
+//
+// One thread waits on an mbarrier that nothing arrives on, through the same bounded wait the
+// forward kernels use, and writes the handle's status word the way a stalled forward kernel
+// does once the limit has passed. Nothing traps; the kernel returns and the context stays usable.
+#include "ss1_internal.cuh"
+#include "ptx_sm100.cuh"
+
+namespace ss1 {
+bool handle_live(const ss1_layer* h);   // ss1_api.cu: a handle from ss1_create, not yet destroyed
+}
+
+namespace {
+
+constexpr int32_t kStatusKernelSelftest = 3;   // kernel id in the status word (forward kernels use 1 and 2)
+constexpr int32_t kSiteUnsatisfiedWait = 1;
+
+__global__ void unsatisfied_wait_kernel(int32_t* status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    abort_flag = 0;
+    ss1::ptx::mbar_init(&bar, 1);   // one arrival would complete phase 0; none comes
+    ss1::ptx::fence_mbar_init();
+    if (!ss1::ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns)) {
+        *(volatile int32_t*)status = (kStatusKernelSelftest << 8) | (0x80 + kSiteUnsatisfiedWait);
+        __threadfence_system();
+    }
+}
+
+}  // namespace
+
+extern "C" SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, void* stream) {
+    if (!ss1::handle_live(h)) return SS1_ERR_BAD_HANDLE;
+    if (limit_ns < 1 || limit_ns > 2000000000) return SS1_ERR_INVALID_ARG;
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    unsatisfied_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->status_dev, (uint64_t)limit_ns);
+    const cudaError_t e = cudaGetLastError();
+    if (prev != h->device) cudaSetDevice(prev);
+    return e == cudaSuccess ? SS1_OK : SS1_ERR_CUDA;
+}

@@ -20,7 +20,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libss1.so")
 
 SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel", "ss1_destroy",
-           "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc")
+           "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc",
+           "ss1_test_device_timeout")
 
 #: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
 NOALLOC_MAX_ENTRIES = 983040
@@ -61,6 +62,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ss1_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     L.ss1_strerror.argtypes = [i32]
     L.ss1_forward_noalloc.argtypes = [i64, i64, i32, i32, i32, u64, vp, vp, vp, i64, i32, vp, vp]
+    L.ss1_test_device_timeout.argtypes = [vp, i64, vp]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":

@@ -66,6 +66,8 @@ def test_argument_checks_before_device(lib):
     bogus = ctypes.c_void_p(0x1000)
     assert lib.ss1_get_info(bogus, None, None, None, None, None) == -7
     assert lib.ss1_destroy(bogus) == -7
+    assert lib.ss1_test_device_timeout(None, 1000000, None) == -7
+    assert lib.ss1_test_device_timeout(bogus, 1000000, None) == -7
     # the allocation-free forward checks its arguments and its table limit first
     fwd = lib.ss1_forward_noalloc
     assert fwd(768, 768, 3, 64, 64, 0, None, None, None, 1, 0, None, None) == -1         # c
