@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--decode-block", type=int, choices=[2, 8], default=None, metavar="C",
                     help="time one Llama-3-8B block's seven projections back to back at compression C "
                          "(rows: --m, default 1) instead of the workload step")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="name each layer launch with an NVTX range (for profilers that filter on them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -413,11 +415,15 @@ def main():
 
     def step(evs=None):
         for i, (L, layer, Xd, Wd, Yd, _) in enumerate(objs):
+            if args.nvtx:
+                torch.cuda.nvtx.range_push(f"ss1_forward {L.K}x{L.N} M={L.M} c={L.c}")
             if evs is not None:
                 evs[i][0].record(stream)
             layer.forward(Xd, Wd, out=Yd)
             if evs is not None:
                 evs[i][1].record(stream)
+            if args.nvtx:
+                torch.cuda.nvtx.range_pop()
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
