@@ -226,17 +226,15 @@ def ss1_forward(X, Wc, h, g, BN: int):
     return Y
 
 
-def ss1_forward_rows(X, Wc, h, g, BN: int, rows, cols=None):
-    """The definition evaluated only at the given rows (and optionally columns) of Y.
+def ss1_forward_rows(X, Wc, h, g, BN: int, rows):
+    """The definition evaluated only at the given rows of Y.
 
     Rows of Y are independent, so a sample of rows is exact for those rows.
-    Returns float64 [len(rows), len(cols) or N].
+    Returns float64 [len(rows), N].
     """
     X = np.asarray(X, dtype=np.float64)
     rows = np.asarray(rows, dtype=np.int64)
     Ys = ss1_forward(X[rows], Wc, h, g, BN)
-    if cols is not None:
-        Ys = Ys[:, np.asarray(cols, dtype=np.int64)]
     return Ys
 
 

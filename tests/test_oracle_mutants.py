@@ -90,6 +90,7 @@ def _pins(golden_dir):
         ("one_hot_probe_structure", P.test_one_hot_probe_structure),
         ("linearity_and_sign_symmetry", P.test_linearity_and_sign_symmetry),
         ("rows_sample_matches_full", P.test_rows_sample_matches_full),
+        ("projection_at_c1_is_identity", P.test_projection_at_c1_is_identity),
         ("projection_recovers_tied_weights", P.test_projection_recovers_tied_weights),
     ]
     for args in [(768, 768, 2, 64, 64, 0), (1280, 512, 4, 128, 128, 2), (1024, 256, 8, 256, 128, 3),

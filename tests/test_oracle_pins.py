@@ -261,6 +261,15 @@ def test_rows_sample_matches_full():
 
 # ---------------------------------------------------------------------------- projection
 
+def test_projection_at_c1_is_identity():
+    """c = 1: every slot holds one input with sign +1, so projecting W returns W itself."""
+    rng = np.random.default_rng(8)
+    K, N, BK, BN = 256, 64, 64, 32
+    h, g = O.ss1_tables(K, N, 1, BK, BN, 4)
+    W = rng.standard_normal((N, K))
+    assert np.array_equal(O.project_dense(W, h, g, BN, 1), W)
+
+
 def test_projection_recovers_tied_weights():
     """Projecting an SS1 tied weight returns its Wc; the residual of a dense W is
     orthogonal to the SS1 subspace (least squares, from S^T S = c I)."""
