@@ -66,6 +66,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The CUDA-core FP32 peak that the fp32 (SIMT) path is held to: 148 SMs x 128 FP32 lanes x
+# 2 flops per FMA x 1.965 GHz, the B200's maximum SM clock.
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def compute_peak_tflops(L, peaks):
+    """Arithmetic peak for a layer's kernel: the bf16 tensor peak, or the FP32 ALU peak for fp32 data."""
+    return FP32_ALU_TFLOPS if L.dtype == "fp32" else peaks["bf16_tflops"]
+
+
 def layer_work(L):
     """Algorithmic work of one layer: dense-equivalent flops, actual flops, bytes moved."""
     e = 2 if L.dtype == "bf16" else 4
@@ -520,22 +530,29 @@ def main():
     value = whole_job_value(dense_step, step_ms, world)
 
     # roofline of the dominant kernel over the step (sum over its launches, one per layer)
-    tc_peak = peaks["bf16_tflops"] * 1e12
     hbm_peak = peaks["hbm_gbs"] * 1e9
     dom = max(set(kernels), key=kernels.count)
     dom_layers = [(L, ms) for L, k, ms in zip(layers, kernels, layer_ms) if k == dom]
-    t_tc = sum(layer_work(L)[1] / tc_peak for L, _ in dom_layers)
+
+    def t_compute(L):
+        return layer_work(L)[1] / (compute_peak_tflops(L, peaks) * 1e12)
+
+    t_tc = sum(t_compute(L) for L, _ in dom_layers)
     t_hbm = sum(layer_work(L)[2] / hbm_peak for L, _ in dom_layers)
     t_kernel = sum(ms for _, ms in dom_layers) * 1e-3
-    ns_frac = sum(max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) for L in layers) / (step_ms * 1e-3)
+    ns_frac = sum(max(t_compute(L), layer_work(L)[2] / hbm_peak) for L in layers) / (step_ms * 1e-3)
+    alu = all(L.dtype == "fp32" for L, _ in dom_layers)
     if t_tc >= t_hbm:
         achieved = sum(layer_work(L)[1] for L, _ in dom_layers) / t_kernel / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof = {"bound": "alu" if alu else "tensor", "achieved": achieved,
+                "peak": FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"], "unit": "TFLOP/s"}
     else:
         achieved = sum(layer_work(L)[2] for L, _ in dom_layers) / t_kernel / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} (burst figure; MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    if roof["bound"] == "alu":
+        roof["peak_source"] = "derived: 148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz"
     rec = traffic_record(dom, [L for L, _ in dom_layers])
     roof["traffic"] = rec["dram_bytes_per_step"] if rec else None
     roof["kernel"] = dom
@@ -554,7 +571,7 @@ def main():
                     "dense_tflops": layer_work(L)[0] / (ms * 1e-3) / 1e12,
                     "actual_tflops": layer_work(L)[1] / (ms * 1e-3) / 1e12,
                     "gbs": layer_work(L)[2] / (ms * 1e-3) / 1e9,
-                    "roofline_frac": max(layer_work(L)[1] / tc_peak, layer_work(L)[2] / hbm_peak) / (ms * 1e-3)}
+                    "roofline_frac": max(t_compute(L), layer_work(L)[2] / hbm_peak) / (ms * 1e-3)}
                    for L, k, ms in zip(layers, kernels, layer_ms)],
         "roofline": roof,
         "gpu_launches": K * len(objs),

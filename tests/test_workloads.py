@@ -124,3 +124,12 @@ def test_source_hash_ignores_comments_only():
     assert bench.code_only(a) == bench.code_only(b)
     assert bench.code_only(a) != bench.code_only(c)
     assert '"a // b /* c */"' in bench.code_only(a)
+
+
+def test_fp32_layers_use_the_alu_peak():
+    """The fp32 workload runs on the CUDA cores: its roofline is the FP32 ALU peak, not the bf16
+    tensor peak (148 SMs x 128 lanes x 2 flops x 1.965 GHz = 74.4 TFLOP/s)."""
+    bench = _bench_module()
+    peaks = {"bf16_tflops": 1628.3, "hbm_gbs": 6542.7}
+    assert abs(bench.compute_peak_tflops(WORKLOADS[1][0], peaks) - 74.4) < 0.05
+    assert bench.compute_peak_tflops(WORKLOADS[2][0], peaks) == 1628.3
