@@ -91,3 +91,28 @@ def test_binding_constants_match_header():
         assert consts[f"SS1_DTYPE_{d.name}"] == int(d)
     m = re.search(r"#define\s+SS1_NOALLOC_MAX_ENTRIES\s+(\d+)", text)
     assert m and int(m.group(1)) == ss1.NOALLOC_MAX_ENTRIES
+
+
+def test_plain_c_program_uses_the_abi(lib, tmp_path):
+    """The header is plain C99 and a C program links against the library and calls it (no
+    torch, no C++): status strings and argument checks, neither of which touches a device."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_ss1.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <string.h>\n#include "ss1.h"\n'
+        "int main(void) {\n"
+        "  ss1_handle h = 0;\n"
+        '  if (strcmp(ss1_strerror(SS1_OK), "ok") != 0) return 1;\n'
+        "  if (ss1_create(770, 768, 2, 64, 64, 0, &h) != SS1_ERR_INVALID_ARG || h != 0) return 2;\n"
+        "  if (ss1_forward(0, 0, 0, 0, 1, SS1_DTYPE_BF16, 0) != SS1_ERR_BAD_HANDLE) return 3;\n"
+        '  puts("c-abi ok");\n  return 0;\n}\n')
+    exe = tmp_path / "use_ss1"
+    libdir = os.path.join(ROOT, "structured_compressed_linear_b200")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-L", libdir, "-lss1", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "c-abi ok", (out.returncode, out.stdout, out.stderr)
