@@ -82,8 +82,9 @@ def _workloads() -> Dict[int, List[Layer]]:
 
 WORKLOADS: Dict[int, List[Layer]] = _workloads()
 
-#: The workload the benchmark times by default: the four GPT-2 Small shaped layers.
-BENCH_WORKLOAD = 2
+#: The workload the benchmark times by default: the eight Llama-3-8B shaped projections at
+#: M = 4096 (c = 2 and c = 8), the largest single-GPU configuration.
+BENCH_WORKLOAD = 4
 
 
 def make_inputs(layer: Layer, device: str = "cpu") -> Tuple[torch.Tensor, torch.Tensor]:

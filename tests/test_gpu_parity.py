@@ -125,11 +125,10 @@ def test_decode_unit_mode_parity(L):
 
 
 # BK = 64 on the tensor-core kernels (the dense kernel at c = 1, the gathering kernel at c = 2
-# and 4): no workload uses it, and these cases have not yet run on a GPU.
+# and 4): no workload uses it, but the automatic choice sends such layers there.
 BK64 = [Layer("bk64", M, 1024, 384, c, 64, 128, "bf16", "normal", "normal_002", 12) for c in (1, 2, 4) for M in (130, 333)]
 
 
-@pytest.mark.skip(reason="written, not yet run on a GPU: enable after its first run")
 @pytest.mark.parametrize("L", BK64, ids=[f"{L.tag}:c{L.c}:M{L.M}" for L in BK64])
 def test_bk64_tensor_core_parity(L):
     check_layer(get_ss1(), L, kernel=TC)

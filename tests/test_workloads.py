@@ -52,8 +52,11 @@ def test_bench_layer_selection():
     spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
     bench = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(bench)
+    # default: the Llama-3-8B projections at the prefill row count, both compressions
     wid, layers = bench.select_layers(None, None)
-    assert wid == 2 and len(layers) == 4 and {L.M for L in layers} == {8192}
+    assert wid == 4 and len(layers) == 8 and {L.M for L in layers} == {4096} and {L.c for L in layers} == {2, 8}
+    _, layers = bench.select_layers(2, None)
+    assert len(layers) == 4 and {L.M for L in layers} == {8192}
     _, layers = bench.select_layers(4, None)
     assert {L.M for L in layers} == {4096} and len(layers) == 8
     _, layers = bench.select_layers(4, 1)
@@ -107,13 +110,22 @@ def _bench_module():
     return bench
 
 
-def test_traffic_record_only_for_its_layers():
-    """The committed DRAM counters are reported for the layers they were taken on and no others."""
+def test_traffic_record_only_for_its_layers_and_code(tmp_path):
+    """DRAM counters are reported for the layers and the kernel code they were taken on, no others."""
+    import json
     bench = _bench_module()
-    assert bench.traffic_record("TC", WORKLOADS[2]) is not None
-    assert bench.traffic_record("TC", WORKLOADS[3]) is None
-    assert bench.traffic_record("TC", [L.with_M(4096) for L in WORKLOADS[2]]) is None
-    assert bench.traffic_record("SMALLM", WORKLOADS[2]) is None
+    sources = ["ss1_tc3.cu", "ptx_sm100.cuh", "ss1_internal.cuh"]
+    rec = {"TC": {"layers": [bench.layer_key(L) for L in WORKLOADS[2]], "dram_bytes_per_step": 1,
+                  "sources": sources, "source_hash": bench.source_hash(sources)}}
+    p = tmp_path / "dram_traffic.json"
+    p.write_text(json.dumps(rec))
+    assert bench.traffic_record("TC", WORKLOADS[2], str(p)) is not None
+    assert bench.traffic_record("TC", WORKLOADS[3], str(p)) is None
+    assert bench.traffic_record("TC", [L.with_M(4096) for L in WORKLOADS[2]], str(p)) is None
+    assert bench.traffic_record("SMALLM", WORKLOADS[2], str(p)) is None
+    rec["TC"]["source_hash"] = "0" * 16          # the kernel's code changed since the capture
+    p.write_text(json.dumps(rec))
+    assert bench.traffic_record("TC", WORKLOADS[2], str(p)) is None
 
 
 def test_source_hash_ignores_comments_only():
