@@ -72,6 +72,8 @@ __all__ = [
     "ss1_forward_rows",
     "ss1_forward_sketch",
     "project_dense",
+    "ss1_backward_input",
+    "ss1_backward_weight",
 ]
 
 _U64 = np.uint64
@@ -277,3 +279,42 @@ def project_dense(W, h, g, BN: int, c: int):
         Sk = sketch_matrix(h, g, nb, K, Kc)
         Wc[nb * BN:(nb + 1) * BN] = (W[nb * BN:(nb + 1) * BN] @ Sk) / c
     return Wc
+
+
+def ss1_backward_input(dY, Wc, h, g, BN: int):
+    """Gradient of a loss with respect to X, given dY = dLoss/dY: since Y = X W_full^T,
+    dX = dY W_full, computed in float64 one N-block of W_full at a time.
+
+    The pages say the SS1 backward pass is not made cheaper ("Limitations") and give no
+    formula; this is plain matrix calculus on the tied weight. dY: [M, N]; returns [M, K].
+    """
+    dY = np.asarray(dY, dtype=np.float64)
+    Wc = np.asarray(Wc, dtype=np.float64)
+    M, N = dY.shape
+    K = h.shape[1]
+    NB = N // BN
+    dX = np.zeros((M, K), dtype=np.float64)
+    for nb in range(NB):
+        Wf = expand_weight(Wc, h, g, BN, nb)                   # [BN, K]
+        dX += dY[:, nb * BN:(nb + 1) * BN] @ Wf
+    return dX
+
+
+def ss1_backward_weight(X, dY, h, g, BN: int, Kc: int):
+    """Gradient with respect to the compressed weights. The gradient of the dense weight is
+    dW_full = dY^T X; every W_full[n, k] is g_nb(k) * Wc[n, h_nb(k)], so by the chain rule
+        dWc[n, j] = sum over k with h_nb(k) == j of g_nb(k) * dW_full[n, k].
+    float64; X: [M, K], dY: [M, N]; returns [N, Kc].
+    """
+    X = np.asarray(X, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    N = dY.shape[1]
+    NB = N // BN
+    dWfull = dY.T @ X                                          # [N, K]
+    dWc = np.zeros((N, Kc), dtype=np.float64)
+    for nb in range(NB):
+        rows = slice(nb * BN, (nb + 1) * BN)
+        signed = dWfull[rows] * g[nb].astype(np.float64)[None, :]
+        for k in range(h.shape[1]):                            # collect every input's term in its column
+            dWc[rows, h[nb, k]] += signed[:, k]
+    return dWc

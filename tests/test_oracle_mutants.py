@@ -59,6 +59,16 @@ MUTANTS = [
     ("projection_without_1_over_c", "(W[nb * BN:(nb + 1) * BN] @ Sk) / c", "(W[nb * BN:(nb + 1) * BN] @ Sk)", "pinned"),
     ("rows_sample_ignores_rows", "Ys = ss1_forward(X[rows], Wc, h, g, BN)", "Ys = ss1_forward(X[:len(rows)], Wc, h, g, BN)",
      "pinned"),
+    ("backward_input_transposed_block", "dX += dY[:, nb * BN:(nb + 1) * BN] @ Wf",
+     "dX += dY[:, nb * BN:(nb + 1) * BN] @ Wf[::-1]", "pinned"),
+    ("backward_input_uses_block0_weights", "Wf = expand_weight(Wc, h, g, BN, nb)                   # [BN, K]",
+     "Wf = expand_weight(Wc, h, g, BN, 0)                   # [BN, K]", "pinned"),
+    ("backward_weight_drops_sign", "signed = dWfull[rows] * g[nb].astype(np.float64)[None, :]",
+     "signed = dWfull[rows] * 1.0", "pinned"),
+    ("backward_weight_overwrites_collisions", "dWc[rows, h[nb, k]] += signed[:, k]", "dWc[rows, h[nb, k]] = signed[:, k]",
+     "pinned"),
+    ("backward_weight_block0_tables", "dWc[rows, h[nb, k]] += signed[:, k]", "dWc[rows, h[0, k]] += signed[:, k]",
+     "pinned"),
     ("sign_from_low_bit", "np.where((r >> _U64(63)) != 0, -1, 1)", "np.where((r & _U64(1)) != 0, -1, 1)", "convention"),
     ("block_key_without_offset", "^ mix64(ids + _U64(1))", "^ mix64(ids)", "convention"),
 ]
@@ -101,6 +111,11 @@ def _pins(golden_dir):
         pins.append((f"frobenius_identity[{c}]", lambda c=c: P.test_frobenius_identity(c)))
     for args in [(64, 32, 2, 16, 8), (256, 256, 4, 64, 64), (512, 256, 8, 256, 128), (768, 768, 2, 64, 64)]:
         pins.append((f"two_routes_agree{args}", lambda a=args: P.test_two_routes_agree(*a)))
+    for args in [(2, 8, 4), (4, 8, 8), (1, 4, 4), (8, 16, 4)]:
+        pins.append((f"backward_input_fd{args}", lambda a=args: P.test_backward_input_finite_differences(*a)))
+        pins.append((f"backward_weight_fd{args}", lambda a=args: P.test_backward_weight_finite_differences(*a)))
+    pins.append(("backward_c1", P.test_backward_c1_is_plain_matrix_calculus))
+    pins.append(("backward_weight_vs_projection", P.test_backward_weight_is_c_times_projection_of_dense_gradient))
     return pins
 
 

@@ -286,3 +286,67 @@ def test_projection_recovers_tied_weights():
     # residual is orthogonal to every tied direction: projecting it gives zero
     np.testing.assert_allclose(O.project_dense(R, h, g, BN, c), 0.0, atol=1e-12)
     assert math.isclose((W * W).sum(), (Wp * Wp).sum() + (R * R).sum(), rel_tol=1e-12)
+
+
+# ---------------------------------------------------------------------------- backward
+
+def _loss_pieces(seed, M=3, K=16, N=8, c=2, BK=8, BN=4):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, K))
+    Wc = rng.standard_normal((N, K // c))
+    R = rng.standard_normal((M, N))          # loss L = sum(R * Y), so dL/dY = R
+    h, g = O.ss1_tables(K, N, c, BK, BN, seed)
+    return X, Wc, R, h, g
+
+
+@pytest.mark.parametrize("c,BK,BN", [(2, 8, 4), (4, 8, 8), (1, 4, 4), (8, 16, 4)])
+def test_backward_input_finite_differences(c, BK, BN):
+    """dX from the oracle against central differences of L(X) = sum(R * Y(X)) in float64. L is
+    linear in X, so the central difference is exact up to rounding; a transposed operand, a
+    missing sign or the wrong N-block's tables all change dX by O(1)."""
+    X, Wc, R, h, g = _loss_pieces(7 + c, c=c, BK=BK, BN=BN)
+    dX = O.ss1_backward_input(R, Wc, h, g, BN)
+    eps = 0.5
+    num = np.empty_like(X)
+    for m in range(X.shape[0]):
+        for k in range(X.shape[1]):
+            E = np.zeros_like(X)
+            E[m, k] = eps
+            num[m, k] = (np.sum(R * O.ss1_forward(X + E, Wc, h, g, BN)) -
+                         np.sum(R * O.ss1_forward(X - E, Wc, h, g, BN))) / (2 * eps)
+    assert np.allclose(dX, num, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("c,BK,BN", [(2, 8, 4), (4, 8, 8), (1, 4, 4), (8, 16, 4)])
+def test_backward_weight_finite_differences(c, BK, BN):
+    """dWc against central differences of L(Wc) = sum(R * Y(Wc)): the chain rule through the
+    tying must collect every input k of a slot with its sign, in the slot's own N-block."""
+    X, Wc, R, h, g = _loss_pieces(11 + c, c=c, BK=BK, BN=BN)
+    dWc = O.ss1_backward_weight(X, R, h, g, BN, Wc.shape[1])
+    eps = 0.5
+    num = np.empty_like(Wc)
+    for n in range(Wc.shape[0]):
+        for j in range(Wc.shape[1]):
+            E = np.zeros_like(Wc)
+            E[n, j] = eps
+            num[n, j] = (np.sum(R * O.ss1_forward(X, Wc + E, h, g, BN)) -
+                         np.sum(R * O.ss1_forward(X, Wc - E, h, g, BN))) / (2 * eps)
+    assert np.allclose(dWc, num, rtol=0, atol=1e-12)
+
+
+def test_backward_c1_is_plain_matrix_calculus():
+    """With the identity hash the layer is Y = X Wc^T, so dX = dY Wc and dWc = dY^T X."""
+    rng = np.random.default_rng(3)
+    M, K, N = 5, 12, 8
+    X, Wc, dY = rng.standard_normal((M, K)), rng.standard_normal((N, K)), rng.standard_normal((M, N))
+    h, g = O.ss1_tables(K, N, 1, 4, 4, 9)
+    assert np.allclose(O.ss1_backward_input(dY, Wc, h, g, 4), dY @ Wc, atol=1e-12)
+    assert np.allclose(O.ss1_backward_weight(X, dY, h, g, 4, K), dY.T @ X, atol=1e-12)
+
+
+def test_backward_weight_is_c_times_projection_of_dense_gradient():
+    """The tied-sum of the dense gradient equals c times the least-squares projection of it
+    (the projection divides the same signed sum by c): ties the two oracle functions together."""
+    X, Wc, R, h, g = _loss_pieces(5, M=6, K=32, N=8, c=4, BK=16, BN=4)
+    dWc = O.ss1_backward_weight(X, R, h, g, 4, Wc.shape[1])
+    assert np.allclose(dWc, 4 * O.project_dense(R.T @ X, h, g, 4, 4), atol=1e-12)
