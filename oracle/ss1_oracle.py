@@ -74,6 +74,10 @@ __all__ = [
     "project_dense",
     "ss1_backward_input",
     "ss1_backward_weight",
+    "e4m3_decode",
+    "e4m3_encode",
+    "quantize_rows_e4m3",
+    "ss1_forward_fp8",
 ]
 
 _U64 = np.uint64
@@ -318,3 +322,58 @@ def ss1_backward_weight(X, dY, h, g, BN: int, Kc: int):
         for k in range(h.shape[1]):                            # collect every input's term in its column
             dWc[rows, h[nb, k]] += signed[:, k]
     return dWc
+
+
+# ---------------------------------------------------------------------------- FP8 weights
+#
+# The SS1 page ("Limitations") lists quantised SS1 kernels as not built, and ("Measured
+# effects") reports post-training quantisation of SS1 models. This reading stores Wc as FP8
+# E4M3 codes with one float32 scale per output neuron: Wc_deq[n, j] = scale[n] * e4m3(Wq[n, j]).
+# E4M3 (the OCP 8-bit floating point format): 1 sign bit, 4 exponent bits with bias 7, 3
+# mantissa bits; exponent field 0 holds subnormals m/8 * 2^-6; S.1111.111 is NaN; there are no
+# infinities, so the largest finite magnitude is 1.75 * 2^8 = 448.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes):
+    """Exact float64 value of each E4M3 code (uint8 array); NaN for 0x7F and 0xFF."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(x):
+    """The E4M3 code nearest to each float (ties to the even code), magnitudes above 448
+    saturated to +-448 (the conversion's 'satfinite' behaviour). x: finite floats."""
+    x = np.asarray(x, dtype=np.float64)
+    values = e4m3_decode(np.arange(0x7F))          # the 127 non-negative finite codes, increasing
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.searchsorted(values, a, side="left")   # first code with value >= a
+    hi = np.minimum(hi, 0x7E)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - values[lo], values[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))   # an even code has an even mantissa
+    code = np.where(a == values[hi], hi, np.where(pick_hi, hi, lo)).astype(np.int64)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def quantize_rows_e4m3(Wc):
+    """Per-row FP8 quantisation: scale[n] = max_j |Wc[n, j]| / 448 computed in float32 (1 for an
+    all-zero row), then codes = e4m3_encode(Wc / scale) with the quotient rounded to float32.
+    Returns (codes uint8 [N, Kc], scale float32 [N])."""
+    W32 = np.asarray(Wc, dtype=np.float32)
+    amax = np.abs(W32).max(axis=1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = (W32 / scale[:, None]).astype(np.float32)
+    return e4m3_encode(q), scale
+
+
+def ss1_forward_fp8(X, Wq, scale, h, g, BN: int):
+    """The layer with FP8 weights: the definition applied to Wc_deq = scale[n] * e4m3(Wq[n, j])."""
+    Wd = e4m3_decode(Wq) * np.asarray(scale, dtype=np.float64)[:, None]
+    return ss1_forward(X, Wd, h, g, BN)

@@ -69,6 +69,15 @@ MUTANTS = [
      "pinned"),
     ("backward_weight_block0_tables", "dWc[rows, h[nb, k]] += signed[:, k]", "dWc[rows, h[0, k]] += signed[:, k]",
      "pinned"),
+    ("e4m3_bias_8", "(1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0)",
+     "(1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 8.0)", "pinned"),
+    ("e4m3_subnormal_scale", "np.where(e == 0, m / 8.0 * 2.0 ** -6", "np.where(e == 0, m / 8.0 * 2.0 ** -7", "pinned"),
+    ("e4m3_ties_to_odd", "((d_hi == d_lo) & (hi % 2 == 0))", "((d_hi == d_lo) & (hi % 2 == 1))", "pinned"),
+    ("e4m3_encode_drops_sign", "return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)",
+     "return code.astype(np.uint8)", "pinned"),
+    ("quantize_scale_not_448", "amax / np.float32(E4M3_MAX)", "amax / np.float32(240.0)", "pinned"),
+    ("fp8_forward_drops_scale", "Wd = e4m3_decode(Wq) * np.asarray(scale, dtype=np.float64)[:, None]",
+     "Wd = e4m3_decode(Wq)", "pinned"),
     ("sign_from_low_bit", "np.where((r >> _U64(63)) != 0, -1, 1)", "np.where((r & _U64(1)) != 0, -1, 1)", "convention"),
     ("block_key_without_offset", "^ mix64(ids + _U64(1))", "^ mix64(ids)", "convention"),
 ]
@@ -115,6 +124,9 @@ def _pins(golden_dir):
         pins.append((f"backward_input_fd{args}", lambda a=args: P.test_backward_input_finite_differences(*a)))
         pins.append((f"backward_weight_fd{args}", lambda a=args: P.test_backward_weight_finite_differences(*a)))
     pins.append(("backward_c1", P.test_backward_c1_is_plain_matrix_calculus))
+    pins.append(("e4m3_decode", P.test_e4m3_decode_matches_library_and_closed_forms))
+    pins.append(("e4m3_encode", P.test_e4m3_encode_round_trip_ties_and_saturation))
+    pins.append(("quantize_rows_fp8_forward", P.test_quantize_rows_and_fp8_forward))
     pins.append(("backward_weight_vs_projection", P.test_backward_weight_is_c_times_projection_of_dense_gradient))
     return pins
 

@@ -350,3 +350,64 @@ def test_backward_weight_is_c_times_projection_of_dense_gradient():
     X, Wc, R, h, g = _loss_pieces(5, M=6, K=32, N=8, c=4, BK=16, BN=4)
     dWc = O.ss1_backward_weight(X, R, h, g, 4, Wc.shape[1])
     assert np.allclose(dWc, 4 * O.project_dense(R.T @ X, h, g, 4, 4), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------- FP8 (E4M3)
+
+def test_e4m3_decode_matches_library_and_closed_forms():
+    """All 256 codes against torch's float8_e4m3fn (an independent implementation of the OCP
+    E4M3 format), plus closed forms: 2^-9 (smallest subnormal), 7 * 2^-9, 2^-6 (smallest
+    normal), 1.0 = 0x38, 448 = 0x7E (largest), NaN at 0x7F and 0xFF, sign symmetry."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = O.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    assert np.array_equal(ours[ok], lib[ok])
+    assert ours[0x01] == 2.0 ** -9 and ours[0x07] == 7 * 2.0 ** -9 and ours[0x08] == 2.0 ** -6
+    assert ours[0x38] == 1.0 and ours[0x7E] == 448.0 and ours[0xFE] == -448.0
+    assert np.isnan(ours[0x7F]) and np.isnan(ours[0xFF]) and np.sum(np.isnan(ours)) == 2
+    assert np.array_equal(ours[0x80:0xFF], -ours[0x00:0x7F])
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    """encode(decode(c)) == c for every finite code; halfway values go to the even mantissa;
+    magnitudes past 448 saturate; random values agree with torch's round-to-nearest-even cast."""
+    import torch
+    codes = np.arange(256)
+    v = O.e4m3_decode(codes)
+    ok = ~np.isnan(v)
+    assert np.array_equal(O.e4m3_encode(v[ok]), codes[ok].astype(np.uint8))
+    # 1.0 (0x38) and 1.125 (0x39): the midpoint 1.0625 goes to 0x38; 1.1875 (between 0x39 and
+    # 0x3A) goes to 0x3A; 2^-10 (between 0 and the smallest subnormal) goes to 0
+    assert O.e4m3_encode(1.0625) == 0x38 and O.e4m3_encode(1.1875) == 0x3A and O.e4m3_encode(2.0 ** -10) == 0
+    assert O.e4m3_encode(1000.0) == 0x7E and O.e4m3_encode(-449.0) == 0xFE
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(20000) * np.exp2(rng.uniform(-12, 8, 20000))).clip(-448, 448).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x), lib)
+
+
+def test_quantize_rows_and_fp8_forward():
+    """Each row's largest |Wc| maps to +-448 (code 0x7E / 0xFE); the dequantised weight is within
+    half an E4M3 step (2^-4 relative) of Wc; the FP8 forward with scale 1 on codes of exactly
+    representable weights is the plain forward."""
+    rng = np.random.default_rng(1)
+    Wc = rng.standard_normal((16, 24)).astype(np.float32) * 0.02
+    Wq, scale = O.quantize_rows_e4m3(Wc)
+    assert scale.dtype == np.float32 and Wq.dtype == np.uint8
+    big = np.argmax(np.abs(Wc), axis=1)
+    assert all((Wq[n, big[n]] & 0x7F) == 0x7E for n in range(16))
+    deq = O.e4m3_decode(Wq) * scale[:, None].astype(np.float64)
+    assert (np.abs(deq - Wc) <= 2.0 ** -4 * np.abs(Wc) + 2.0 ** -10 * scale[:, None]).all()
+    h, g = O.ss1_tables(48, 16, 2, 16, 8, 4)
+    X = rng.standard_normal((3, 48))
+    W_exact = O.e4m3_decode(rng.integers(0, 0x7E, size=(16, 24)))
+    Y8 = O.ss1_forward_fp8(X, O.e4m3_encode(W_exact), np.ones(16, np.float32), h, g, 8)
+    assert np.array_equal(Y8, O.ss1_forward(X, W_exact, h, g, 8))
+    # the scale of neuron n multiplies output column n alone, linearly
+    one_hot = np.zeros(16, np.float32)
+    one_hot[5] = 4.0
+    Ys = O.ss1_forward_fp8(X, O.e4m3_encode(W_exact), one_hot, h, g, 8)
+    assert np.array_equal(Ys[:, 5], 4.0 * Y8[:, 5]) and np.count_nonzero(np.delete(Ys, 5, axis=1)) == 0
