@@ -78,6 +78,12 @@ __all__ = [
     "e4m3_encode",
     "quantize_rows_e4m3",
     "ss1_forward_fp8",
+    "ACT_NONE",
+    "ACT_RELU",
+    "ACT_GELU",
+    "activation",
+    "ss1_forward_bias_act",
+    "ss1_chain_forward",
 ]
 
 _U64 = np.uint64
@@ -377,3 +383,45 @@ def ss1_forward_fp8(X, Wq, scale, h, g, BN: int):
     """The layer with FP8 weights: the definition applied to Wc_deq = scale[n] * e4m3(Wq[n, j])."""
     Wd = e4m3_decode(Wq) * np.asarray(scale, dtype=np.float64)[:, None]
     return ss1_forward(X, Wd, h, g, BN)
+
+
+# ---------------------------------------------------------------------------- epilogue, chain
+#
+# The SS1 page ("Measured effects") replaces the DLRM MLPerf top MLP's layers by SS1 layers. The
+# layer itself has no bias or activation; an MLP adds both between layers. This reading: a
+# per-neuron bias added to the fp64 sum, then the activation, ReLU (max(v, 0)) or GELU in its
+# exact form v * Phi(v) = 0.5 v (1 + erf(v / sqrt(2))), written with the library erf.
+
+ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
+
+
+def activation(v, act: int):
+    """The activation of the epilogue on float64 values."""
+    v = np.asarray(v, dtype=np.float64)
+    if act == ACT_NONE:
+        return v
+    if act == ACT_RELU:
+        return np.maximum(v, 0.0)
+    if act == ACT_GELU:
+        from math import erf, sqrt
+        return 0.5 * v * (1.0 + np.vectorize(erf)(v / sqrt(2.0)))
+    raise ValueError(act)
+
+
+def ss1_forward_bias_act(X, Wc, h, g, BN: int, bias=None, act: int = ACT_NONE):
+    """act(SS1(X) + bias) in float64; bias: [N] or None."""
+    Y = ss1_forward(X, Wc, h, g, BN)
+    if bias is not None:
+        Y = Y + np.asarray(bias, dtype=np.float64)[None, :]
+    return activation(Y, act)
+
+
+def ss1_chain_forward(X, layers):
+    """A chain of SS1 layers, each the input of the next: layers is a list of
+    (Wc, h, g, BN, bias, act). Returns every layer's output (float64, no intermediate rounding)."""
+    outs = []
+    cur = np.asarray(X, dtype=np.float64)
+    for Wc, h, g, BN, bias, act in layers:
+        cur = ss1_forward_bias_act(cur, Wc, h, g, BN, bias, act)
+        outs.append(cur)
+    return outs

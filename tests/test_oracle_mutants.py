@@ -78,6 +78,12 @@ MUTANTS = [
     ("quantize_scale_not_448", "amax / np.float32(E4M3_MAX)", "amax / np.float32(240.0)", "pinned"),
     ("fp8_forward_drops_scale", "Wd = e4m3_decode(Wq) * np.asarray(scale, dtype=np.float64)[:, None]",
      "Wd = e4m3_decode(Wq)", "pinned"),
+    ("relu_is_identity", "return np.maximum(v, 0.0)", "return v", "pinned"),
+    ("gelu_without_sqrt2", "return 0.5 * v * (1.0 + np.vectorize(erf)(v / sqrt(2.0)))",
+     "return 0.5 * v * (1.0 + np.vectorize(erf)(v))", "pinned"),
+    ("bias_dropped", "Y = Y + np.asarray(bias, dtype=np.float64)[None, :]", "Y = Y + 0.0", "pinned"),
+    ("chain_drops_activation", "cur = ss1_forward_bias_act(cur, Wc, h, g, BN, bias, act)",
+     "cur = ss1_forward_bias_act(cur, Wc, h, g, BN, bias, ACT_NONE)", "pinned"),
     ("sign_from_low_bit", "np.where((r >> _U64(63)) != 0, -1, 1)", "np.where((r & _U64(1)) != 0, -1, 1)", "convention"),
     ("block_key_without_offset", "^ mix64(ids + _U64(1))", "^ mix64(ids)", "convention"),
 ]
@@ -127,6 +133,9 @@ def _pins(golden_dir):
     pins.append(("e4m3_decode", P.test_e4m3_decode_matches_library_and_closed_forms))
     pins.append(("e4m3_encode", P.test_e4m3_encode_round_trip_ties_and_saturation))
     pins.append(("quantize_rows_fp8_forward", P.test_quantize_rows_and_fp8_forward))
+    pins.append(("activations", P.test_activations_closed_forms))
+    pins.append(("bias_act_layer", P.test_bias_act_layer))
+    pins.append(("chain_composition", P.test_chain_is_composition))
     pins.append(("backward_weight_vs_projection", P.test_backward_weight_is_c_times_projection_of_dense_gradient))
     return pins
 

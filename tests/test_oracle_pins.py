@@ -411,3 +411,56 @@ def test_quantize_rows_and_fp8_forward():
     one_hot[5] = 4.0
     Ys = O.ss1_forward_fp8(X, O.e4m3_encode(W_exact), one_hot, h, g, 8)
     assert np.array_equal(Ys[:, 5], 4.0 * Y8[:, 5]) and np.count_nonzero(np.delete(Ys, 5, axis=1)) == 0
+
+
+# ---------------------------------------------------------------------------- bias, activation, chain
+
+def test_activations_closed_forms():
+    """ReLU clamps at zero; GELU(0) = 0, GELU(x) -> x for large x and -> 0 for very negative x,
+    GELU(1) = Phi(1) = 0.8413447460685429 (the normal distribution function at 1, a tabulated
+    value), and GELU(x) - GELU(-x) = x (Phi(x) + Phi(-x) = 1)."""
+    v = np.array([-3.0, -0.5, 0.0, 0.25, 2.0])
+    assert np.array_equal(O.activation(v, O.ACT_RELU), [0.0, 0.0, 0.0, 0.25, 2.0])
+    assert np.array_equal(O.activation(v, O.ACT_NONE), v)
+    gl = O.activation(np.array([0.0, 1.0, 12.0, -12.0]), O.ACT_GELU)
+    assert gl[0] == 0.0 and abs(gl[1] - 0.8413447460685429) < 1e-15
+    assert abs(gl[2] - 12.0) < 1e-12 and abs(gl[3]) < 1e-12
+    x = np.linspace(-4, 4, 41)
+    assert np.allclose(O.activation(x, O.ACT_GELU) - O.activation(-x, O.ACT_GELU), x, atol=1e-14)
+
+
+def test_bias_act_layer():
+    """With X = 0 the layer gives act(bias) exactly; with zero bias and no activation it is the
+    plain forward; the bias of neuron n shifts column n alone."""
+    rng = np.random.default_rng(2)
+    K, N, c, BK, BN = 32, 16, 2, 16, 8
+    h, g = O.ss1_tables(K, N, c, BK, BN, 3)
+    Wc = rng.standard_normal((N, K // c))
+    X = rng.standard_normal((5, K))
+    b = rng.standard_normal(N)
+    for act in (O.ACT_NONE, O.ACT_RELU, O.ACT_GELU):
+        Y0 = O.ss1_forward_bias_act(np.zeros((2, K)), Wc, h, g, BN, b, act)
+        assert np.array_equal(Y0, np.tile(O.activation(b, act), (2, 1)))
+    assert np.array_equal(O.ss1_forward_bias_act(X, Wc, h, g, BN, None, O.ACT_NONE), O.ss1_forward(X, Wc, h, g, BN))
+    e = np.zeros(N)
+    e[3] = 1.5
+    d = O.ss1_forward_bias_act(X, Wc, h, g, BN, e, O.ACT_NONE) - O.ss1_forward(X, Wc, h, g, BN)
+    assert np.allclose(d[:, 3], 1.5, atol=1e-14) and np.count_nonzero(np.delete(d, 3, axis=1)) == 0
+
+
+def test_chain_is_composition():
+    """Each output of the chain is the next layer's input: layer 2 of the chain equals one layer
+    applied to layer 1's output."""
+    rng = np.random.default_rng(4)
+    dims = [32, 16, 16, 8]
+    layers = []
+    for i in range(3):
+        h, g = O.ss1_tables(dims[i], dims[i + 1], 2, 16, 8, 4)
+        layers.append((rng.standard_normal((dims[i + 1], dims[i] // 2)), h, g, 8, rng.standard_normal(dims[i + 1]),
+                       O.ACT_RELU if i < 2 else O.ACT_NONE))
+    X = rng.standard_normal((6, 32))
+    outs = O.ss1_chain_forward(X, layers)
+    assert [o.shape for o in outs] == [(6, 16), (6, 16), (6, 8)]
+    W, h, g, BN, b, act = layers[1]
+    assert np.array_equal(outs[1], O.ss1_forward_bias_act(outs[0], W, h, g, BN, b, act))
+    assert (outs[0] >= 0).all() and (outs[1] >= 0).all()
