@@ -50,6 +50,11 @@ def parse():
     ap.add_argument("--decode-block", type=int, choices=[2, 8], default=None, metavar="C",
                     help="time one Llama-3-8B block's seven projections back to back at compression C "
                          "(rows: --m, default 1) instead of the workload step")
+    ap.add_argument("--op", choices=["forward", "project", "backward"], default="forward",
+                    help="project: time ss1_project (dense W[N, K] -> Wc[N, K/c]) on the workload's layer shapes; "
+                         "backward: time ss1_backward_input + ss1_backward_weight on the workload's layers")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 (E4M3) weights with per-neuron scales (ss1_forward_fp8; decode-sized rows only)")
     ap.add_argument("--nvtx", action="store_true",
                     help="name each layer launch with an NVTX range (for profilers that filter on them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -76,13 +81,15 @@ def compute_peak_tflops(L, peaks):
     return FP32_ALU_TFLOPS if L.dtype == "fp32" else peaks["bf16_tflops"]
 
 
-def layer_work(L):
-    """Algorithmic work of one layer: dense-equivalent flops, actual flops, bytes moved."""
+def layer_work(L, fp8=False):
+    """Algorithmic work of one layer: dense-equivalent flops, actual flops, bytes moved. With FP8
+    weights Wc is one byte per weight plus one float scale per neuron."""
     e = 2 if L.dtype == "bf16" else 4
     dense = 2.0 * L.M * L.N * L.K
     adds = float(L.M) * (L.N // L.BN) * L.K * (1.0 - 1.0 / L.c)
     actual = 2.0 * L.M * L.N * L.K / L.c + adds
-    byts = float(e) * (L.M * L.K + L.N * L.K // L.c + L.M * L.N)
+    wbytes = (L.N * L.K // L.c + 4.0 * L.N) if fp8 else float(e) * (L.N * L.K // L.c)
+    byts = float(e) * (L.M * L.K + L.M * L.N) + wbytes
     return dense, actual, byts
 
 
@@ -252,18 +259,23 @@ def run_decode_block(args, peaks, peak_src, dev):
     from structured_compressed_linear_b200 import ss1
     M, c = args.m or 1, args.decode_block
     layers = [ss1.SS1Layer(K, N, c, 256, 128, 3) for K, N in LLAMA_BLOCK]
-    wc_bytes = sum(N * (K // c) * 2 for K, N in LLAMA_BLOCK)
+    wc_bytes = sum(N * (K // c) * (1 if args.fp8 else 2) + (4 * N if args.fp8 else 0) for K, N in LLAMA_BLOCK)
     ncopy = max(2, -(-300_000_000 // wc_bytes))
     gen = torch.Generator(device=dev).manual_seed(3)
     Ws = [[(torch.randn(N, K // c, device=dev, generator=gen) * 0.02).to(torch.bfloat16) for K, N in LLAMA_BLOCK]
           for _ in range(ncopy)]
+    if args.fp8:
+        Ws = [[ss1.quantize_fp8(w) for w in copy] for copy in Ws]
     Xs = [torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16) for K, _ in LLAMA_BLOCK]
     Ys = [torch.empty(M, N, device=dev, dtype=torch.bfloat16) for _, N in LLAMA_BLOCK]
-    kernels = sorted({layer.select_kernel(M).name for layer in layers})
+    kernels = ["SMALLM-FP8"] if args.fp8 else sorted({layer.select_kernel(M).name for layer in layers})
 
     def block(cp):
         for i, layer in enumerate(layers):
-            layer.forward(Xs[i], Ws[cp][i], out=Ys[i])
+            if args.fp8:
+                layer.forward_fp8(Xs[i], Ws[cp][i][0], Ws[cp][i][1], out=Ys[i])
+            else:
+                layer.forward(Xs[i], Ws[cp][i], out=Ys[i])
 
     for s in range(max(3, args.warmup) * ncopy):
         block(s % ncopy)
@@ -282,9 +294,11 @@ def run_decode_block(args, peaks, peak_src, dev):
     byts = wc_bytes + sum(2 * (M * K + M * N) for K, N in LLAMA_BLOCK)
     achieved = byts / (us * 1e-6) / 1e9
     print(json.dumps({
-        "metric": "SS1 decode block latency (Llama-3-8B q, k, v, o, gate, up, down back to back)",
+        "metric": "SS1 decode block latency (Llama-3-8B q, k, v, o, gate, up, down back to back)"
+                  + (", FP8 weights" if args.fp8 else ""),
         "value": us, "unit": "us per block", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
-        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "higher_is_better": False, "dtype": "bf16 activations, " + ("e4m3 weights" if args.fp8 else "bf16 weights"),
+        "data": "synthetic",
         "config": {"workload": f"llama-3-8b block at M={M}, c={c}, BK=256, BN=128", "kernels": kernels,
                    "l2": f"Wc rotated over {ncopy} copies ({ncopy * wc_bytes / 1e6:.0f} MB), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -293,6 +307,150 @@ def run_decode_block(args, peaks, peak_src, dev):
     }), flush=True)
     for layer in layers:
         layer.close()
+
+
+def run_project(args, layers, wid, peaks, peak_src, dev):
+    """ss1_project on every distinct layer shape of the workload: W[N, K] (seeded, N(0, 0.02^2))
+    -> Wc[N, K/c]. HBM-bound: the algorithmic bytes are W read once and Wc written once. L2 is
+    flushed before every timed step; each launch is bracketed by CUDA events."""
+    import torch
+    from structured_compressed_linear_b200 import ss1
+    shapes = []
+    for L in layers:
+        key = (L.K, L.N, L.c, L.BK, L.BN, L.dtype)
+        if key not in [x[0] for x in shapes]:
+            shapes.append((key, L))
+    objs = []
+    gen = torch.Generator(device=dev).manual_seed(7)
+    for (K, N, c, BK, BN, dt), L in shapes:
+        dtype = torch.bfloat16 if dt == "bf16" else torch.float32
+        W = (torch.randn(N, K, device=dev, generator=gen) * 0.02).to(dtype)
+        layer = ss1.SS1Layer(K, N, c, BK, BN, L.seed)
+        objs.append((L, layer, W, torch.empty((N, K // c), dtype=dtype, device=dev)))
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        for _L, layer, W, Wc in objs:
+            layer.project(W, out=Wc)
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in objs]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index or 0)
+    with sampler:
+        for s_ in range(args.steps):
+            flush.zero_()
+            for i, (_L, layer, W, Wc) in enumerate(objs):
+                evs[s_][i][0].record(stream)
+                layer.project(W, out=Wc)
+                evs[s_][i][1].record(stream)
+        torch.cuda.synchronize()
+    per = []
+    total_bytes, total_ms = 0.0, 0.0
+    for i, (L, layer, W, Wc) in enumerate(objs):
+        ms = statistics.mean(evs[s_][i][0].elapsed_time(evs[s_][i][1]) for s_ in range(args.steps))
+        e = W.element_size()
+        byts = float(e) * (L.N * L.K + L.N * (L.K // L.c))
+        total_bytes += byts
+        total_ms += ms
+        per.append({"K": L.K, "N": L.N, "c": L.c, "BK": L.BK, "BN": L.BN, "us": ms * 1e3,
+                    "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+        layer.close()
+    achieved = total_bytes / (total_ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "SS1 dense -> SS1 projection (ss1_project) GB/s on 1 B200; achieved fraction of HBM roofline",
+        "value": achieved, "unit": "GB/s (W read + Wc written, algorithmic)", "n_gpus": 1, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms, "higher_is_better": True, "dtype": layers[0].dtype,
+        "data": "synthetic (seeded)", "config": {"workload": f"workload {wid} layer shapes", "l2": "flushed before every step"},
+        "layers": per,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src, "kernel": "project_kernel",
+                     "algorithmic_bytes": total_bytes},
+        "gpu_launches": args.steps * len(objs), "clocks": sampler.summary(),
+    }), flush=True)
+
+
+def backward_work(L):
+    """Algorithmic work of one layer's backward pass (both gradients): dense-equivalent flops
+    2 * 2 M N K; the method's own flops: the two compressed products 2 * 2 M N K / c, the
+    un-sketch adds of dX (M K NB) and the sketch adds of dWc (M NB K (1 - 1/c))."""
+    NB = L.N // L.BN
+    dense = 4.0 * L.M * L.N * L.K
+    actual = 4.0 * L.M * L.N * L.K / L.c + float(L.M) * L.K * NB + float(L.M) * NB * L.K * (1.0 - 1.0 / L.c)
+    return dense, actual
+
+
+def run_backward(args, layers, wid, peaks, peak_src, dev):
+    """ss1_backward_input + ss1_backward_weight on every layer of the workload, seeded dY and
+    X, workspaces allocated once. L2 flushed before every step; CUDA events around each call."""
+    import torch
+    from structured_compressed_linear_b200 import ss1
+    from structured_compressed_linear_b200.workloads import make_inputs
+    objs = []
+    for L in layers:
+        X, Wc = make_inputs(L)
+        gen = torch.Generator().manual_seed(L.M + L.N)
+        dY = torch.randn(L.M, L.N, generator=gen).to(X.dtype)
+        layer = ss1.SS1Layer(L.K, L.N, L.c, L.BK, L.BN, L.seed)
+        wi, ww = layer.backward_workspace(L.M, X.dtype)
+        objs.append((L, layer, X.to(dev), Wc.to(dev), dY.to(dev), torch.empty(L.M, L.K, dtype=X.dtype, device=dev),
+                     torch.empty(L.N, L.K // L.c, dtype=X.dtype, device=dev),
+                     torch.empty(max(wi, ww, 1), dtype=torch.uint8, device=dev)))
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        for i, (L, layer, X, Wc, dY, dX, dWc, ws) in enumerate(objs):
+            if evs is not None:
+                evs[i][0].record(stream)
+            layer.backward_input(dY, Wc, out=dX, workspace=ws)
+            if evs is not None:
+                evs[i][1].record(stream)
+            layer.backward_weight(X, dY, out=dWc, workspace=ws)
+            if evs is not None:
+                evs[i][2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in objs] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index or 0)
+    with sampler:
+        for s_ in range(args.steps):
+            flush.zero_()
+            step(evs[s_])
+        torch.cuda.synchronize()
+    per, tot_ms, tot_dense, tot_actual = [], 0.0, 0.0, 0.0
+    for i, (L, layer, *_r) in enumerate(objs):
+        ms_in = statistics.mean(evs[s_][i][0].elapsed_time(evs[s_][i][1]) for s_ in range(args.steps))
+        ms_w = statistics.mean(evs[s_][i][1].elapsed_time(evs[s_][i][2]) for s_ in range(args.steps))
+        dense, actual = backward_work(L)
+        ms = ms_in + ms_w
+        tot_ms += ms
+        tot_dense += dense
+        tot_actual += actual
+        per.append({"K": L.K, "N": L.N, "M": L.M, "c": L.c, "dX_us": ms_in * 1e3, "dWc_us": ms_w * 1e3,
+                    "dense_tflops": dense / (ms * 1e-3) / 1e12,
+                    "roofline_frac": actual / (peaks["bf16_tflops"] * 1e12) / (ms * 1e-3)})
+        st, detail = layer.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {detail:#x}")
+        layer.close()
+    achieved = tot_actual / (tot_ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "SS1 backward (dX and dWc) dense-equiv TFLOP/s on 1 B200; achieved fraction of roofline",
+        "value": tot_dense / (tot_ms * 1e-3) / 1e12, "unit": "TFLOP/s (dense-equivalent 4*M*N*K per layer)",
+        "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": tot_ms,
+        "higher_is_better": True, "dtype": layers[0].dtype, "data": "synthetic (seeded)",
+        "config": {"workload": f"workload {wid} layers at M = {layers[0].M}", "l2": "flushed before every step"},
+        "layers": per,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "peak_source": peak_src,
+                     "note": "algorithmic flops: the compressed products and the sketch adds; the kernels run the "
+                             "dense products (the pages: the backward pass is not made cheaper)"},
+        "gpu_launches": None, "clocks": sampler.summary(),
+    }), flush=True)
 
 
 def run_reference(args, layers, wid, rank, world):
@@ -397,6 +555,18 @@ def main():
 
     wid, layers = select_layers(args.workload, args.m)
 
+    if args.op in ("project", "backward"):   # one GPU: the projection or the backward kernels
+        if rank != 0:
+            return
+        import torch
+        from structured_compressed_linear_b200 import build
+        build.build()
+        torch.cuda.set_device(local)
+        peaks, peak_src = load_peaks()
+        run = run_project if args.op == "project" else run_backward
+        run(args, layers, wid, peaks, peak_src, torch.device("cuda", local))
+        return
+
     if args.impl == "reference":
         run_reference(args, layers, wid, rank, world)
         return
@@ -425,6 +595,12 @@ def main():
         Yd = torch.empty((L.M, L.N), dtype=Xd.dtype, device=dev)
         objs.append((L, layer, Xd, Wd, Yd, X))
     kernels = [ss1.Kernel(layer.select_kernel(L.M, Xd.dtype)).name for (L, layer, Xd, *_r) in objs]
+    fp8 = None
+    if args.fp8:   # per-neuron FP8 weights for the decode kernel
+        if any(L.M > 64 or L.BN != 128 for L in layers):
+            raise SystemExit("--fp8 runs decode-sized layers (M <= 64, BN = 128)")
+        fp8 = [ss1.quantize_fp8(Wd) for (_L, _l, _X, Wd, *_r) in objs]
+        kernels = ["SMALLM-FP8"] * len(objs)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -434,7 +610,10 @@ def main():
                 torch.cuda.nvtx.range_push(f"ss1_forward {L.K}x{L.N} M={L.M} c={L.c}")
             if evs is not None:
                 evs[i][0].record(stream)
-            layer.forward(Xd, Wd, out=Yd)
+            if fp8 is not None:
+                layer.forward_fp8(Xd, fp8[i][0], fp8[i][1], out=Yd)
+            else:
+                layer.forward(Xd, Wd, out=Yd)
             if evs is not None:
                 evs[i][1].record(stream)
             if args.nvtx:
@@ -474,7 +653,7 @@ def main():
     # so that a step's inputs travel to the device while the previous step's results travel back
     # (PCIe carries both directions at once) and the forwards run in between.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and fp8 is None:
         hostX = [x.pin_memory() for (*_r, x) in objs]
         hostY = [torch.empty((L.M, L.N), dtype=Xd.dtype).pin_memory() for (L, _l, Xd, *_r) in objs]
         h2d = sum(x.numel() * x.element_size() for x in hostX)
@@ -531,7 +710,8 @@ def main():
         te = max_over_ranks(torch.tensor([e0.elapsed_time(e1) / ke], dtype=torch.float64, device=dev), world)
         e2e = (float(te[0]), h2d, d2h)
 
-    dense_step = sum(layer_work(L)[0] for L in layers)
+    isfp8 = fp8 is not None
+    dense_step = sum(layer_work(L, isfp8)[0] for L in layers)
     value = whole_job_value(dense_step, step_ms, world)
 
     # roofline of the dominant kernel over the step (sum over its launches, one per layer)
@@ -543,16 +723,16 @@ def main():
         return layer_work(L)[1] / (compute_peak_tflops(L, peaks) * 1e12)
 
     t_tc = sum(t_compute(L) for L, _ in dom_layers)
-    t_hbm = sum(layer_work(L)[2] / hbm_peak for L, _ in dom_layers)
+    t_hbm = sum(layer_work(L, isfp8)[2] / hbm_peak for L, _ in dom_layers)
     t_kernel = sum(ms for _, ms in dom_layers) * 1e-3
-    ns_frac = sum(max(t_compute(L), layer_work(L)[2] / hbm_peak) for L in layers) / (step_ms * 1e-3)
+    ns_frac = sum(max(t_compute(L), layer_work(L, isfp8)[2] / hbm_peak) for L in layers) / (step_ms * 1e-3)
     alu = all(L.dtype == "fp32" for L, _ in dom_layers)
     if t_tc >= t_hbm:
         achieved = sum(layer_work(L)[1] for L, _ in dom_layers) / t_kernel / 1e12
         roof = {"bound": "alu" if alu else "tensor", "achieved": achieved,
                 "peak": FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"], "unit": "TFLOP/s"}
     else:
-        achieved = sum(layer_work(L)[2] for L, _ in dom_layers) / t_kernel / 1e9
+        achieved = sum(layer_work(L, isfp8)[2] for L, _ in dom_layers) / t_kernel / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} (burst figure; MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
@@ -563,20 +743,21 @@ def main():
     roof["kernel"] = dom
     roof["launches_per_step"] = kernels.count(dom)
     roof["per"] = "one step: the sum over that kernel's launches (one per layer)"
-    roof["algorithmic_bytes"] = sum(layer_work(L)[2] for L, k in zip(layers, kernels) if k == dom)
+    roof["algorithmic_bytes"] = sum(layer_work(L, isfp8)[2] for L, k in zip(layers, kernels) if k == dom)
     roof["algorithmic_flops"] = sum(layer_work(L)[1] for L, k in zip(layers, kernels) if k == dom)
     roof["frac_slower_of_tensor_and_hbm"] = ns_frac
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if layers[0].dtype == "bf16" else "fp32", "data": "synthetic (seeded, shapes of the workload)",
+        "dtype": ("bf16 activations, e4m3 weights" if isfp8 else "bf16") if layers[0].dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded, shapes of the workload)",
         "config": workload_config(layers, wid, world),
         "layers": [{"K": L.K, "N": L.N, "M": L.M, "c": L.c, "kernel": k, "ms": ms,
                     "dense_tflops": layer_work(L)[0] / (ms * 1e-3) / 1e12,
                     "actual_tflops": layer_work(L)[1] / (ms * 1e-3) / 1e12,
-                    "gbs": layer_work(L)[2] / (ms * 1e-3) / 1e9,
-                    "roofline_frac": max(t_compute(L), layer_work(L)[2] / hbm_peak) / (ms * 1e-3)}
+                    "gbs": layer_work(L, isfp8)[2] / (ms * 1e-3) / 1e9,
+                    "roofline_frac": max(t_compute(L), layer_work(L, isfp8)[2] / hbm_peak) / (ms * 1e-3)}
                    for L, k, ms in zip(layers, kernels, layer_ms)],
         "roofline": roof,
         "gpu_launches": K * len(objs),

@@ -31,6 +31,7 @@
 #ifndef SS1_H
 #define SS1_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -79,8 +80,7 @@ enum ss1_status {
  *   out    : receives the handle (host pointer to a handle variable).
  * Allocates device memory and one pinned host word (device status), launches the table
  * generator and synchronises. The device memory is the tables (17 bytes per (N / BN) * K
- * entry). Where BN == 128 and N / BN is at most the SM count, it is also the decode kernel's
- * K-split scratch: 2 x SMs x 32 KiB of fp32 partials plus 16 bytes per N-block of counters.
+ * entry); after this call the handle is only read.
  * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, OUT_OF_MEMORY, CUDA. On error *out is set to NULL
  * and nothing is leaked.
  */
@@ -97,10 +97,9 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
  * Asynchronous: returns after the launch. Errors: BAD_HANDLE, INVALID_ARG, MISALIGNED
  * (X, Wc, Y must be 16-byte aligned), CUDA (launch failure), DEVICE_TIMEOUT (an earlier
  * launch on this handle reported a bounded-wait time-out; see ss1_device_status).
- * Decode calls (the SMALLM kernel, which AUTO picks for M <= 16) on a handle with N-blocks of
- * 128 pass partial sums through the handle's K-split scratch: such calls on one handle must not
- * overlap on the device (order them on one stream or with events). Every other call only reads
- * the handle, so those may run concurrently on any streams.
+ * Re-entrant: every kernel only reads the handle and writes nothing but Y (the decode kernel's
+ * K-split partial sums stay in the shared memory of one thread-block cluster), so calls on one
+ * handle may run concurrently on any streams and threads.
  * The tensor-core decode kernel is launched with programmatic dependent launch: it may start
  * while the previous kernel on the stream is still running, but before that kernel completes it
  * only prefetches Wc into L2. It reads X and the tables and writes Y only afterwards, so stream
@@ -148,14 +147,116 @@ SS1_API int ss1_get_info(ss1_handle h, int64_t* K, int64_t* N, int* c, int* BK, 
  * synchronising. Kernels with bounded waits write a non-zero code there instead of
  * trapping when a wait runs out; the word lives in pinned host memory. Returns SS1_OK or
  * SS1_ERR_DEVICE_TIMEOUT; *detail (may be NULL) receives the raw code (kernel id and wait site).
- * Call after synchronising the stream to see the result of the work enqueued so far. When it
- * reports a time-out it also synchronises the device and resets the decode kernel's K-split
- * counters, which a launch that gave up may have left non-zero.
+ * Call after synchronising the stream to see the result of the work enqueued so far.
  */
 SS1_API int ss1_device_status(ss1_handle h, int32_t* detail);
 
 /* ss1_strerror -- static, NUL-terminated text for a status code. */
 SS1_API const char* ss1_strerror(int status);
+
+/*
+ * ss1_project -- the SS1 weights closest to a dense weight: Wc = argmin || W_full(Wc) - W ||_F.
+ * "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+ * "Key results": pre-trained dense layers (BERT-Base, Llama-3-8B) are projected onto SS1. The
+ * pages give no formula; this is the orthogonal projection onto the tied weights of this
+ * handle's tables. Every slot of every (N-block, K-chunk) holds exactly c inputs with signs
+ * +-1, so the projection is the sketch of each weight row, divided by c:
+ *
+ *     Wc[n, j] = (1 / c) * sum over k with h_nb(k) == j of g_nb(k) * W[n, k],   nb = n / BN.
+ *
+ * Projecting a tied weight (W = W_full(Wc0)) returns Wc0 exactly.
+ *   W     : device, [N, K] of `dtype` (torch.nn.Linear layout: one row per output neuron).
+ *   Wc    : device, [N, K / c] of `dtype`, written in full; must not overlap W.
+ *   dtype : SS1_DTYPE_BF16 or SS1_DTYPE_FP32; the c terms are summed in fp32 and rounded once.
+ *   stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ * The caller owns W and Wc. Asynchronous; reads the handle only, so calls may run concurrently.
+ * Rows and chunks that are multiples of 16 bytes with 16-byte-aligned W and Wc take the fast
+ * kernel; any other shape a plain one. Errors: BAD_HANDLE, INVALID_ARG (NULL pointer, dtype),
+ * MISALIGNED (W or Wc not aligned to its element size), CUDA (launch failure).
+ */
+SS1_API int ss1_project(ss1_handle h, const void* W, void* Wc, int dtype, void* stream);
+
+/*
+ * Backward pass. "SS1: Accelerating Inference with Fast and Expressive Sketch Structured
+ * Transform", section "Limitations": SS1 does not make the backward pass cheaper. The pages give
+ * no formula; on the tied weight W_full[n, k] = g_nb(k) Wc[n, h_nb(k)] matrix calculus gives, for
+ * dY = dLoss/dY [M, N],
+ *
+ *     dX[m, k]  = sum_n dY[m, n] W_full[n, k]                                     [M, K]
+ *     dWc[n, j] = sum over k with h_nb(k) == j of g_nb(k) * sum_m dY[m, n] X[m, k]   [N, K / c]
+ *
+ * Both run at the dense layer's cost (as the pages describe): W_full^T, or dY^T and X^T, are
+ * written into a caller-provided workspace and multiplied on the tensor cores (bf16 shapes with
+ * K a multiple of 128 and, for dX, N a multiple of 64) or the CUDA cores (fp32, other shapes),
+ * accumulating in fp32. The workspace is device memory of at least the size that
+ * ss1_backward_workspace gives, 256-byte aligned, owned by the caller, not read before it is
+ * written; calls that share one workspace must be ordered on the device. Both calls are
+ * asynchronous and only read the handle.
+ */
+
+/*
+ * ss1_backward_workspace -- workspace bytes of ss1_backward_input (independent of M) and of
+ * ss1_backward_weight for M rows; either output pointer may be NULL. Errors: BAD_HANDLE,
+ * INVALID_ARG (M < 0, dtype).
+ */
+SS1_API int ss1_backward_workspace(ss1_handle h, int64_t M, int dtype, size_t* input_bytes, size_t* weight_bytes);
+
+/*
+ * ss1_backward_input -- dX = dY W_full.
+ *   dY : device, [M, N] of `dtype`.     Wc : device, [N, K / c].     dX : device, [M, K], written.
+ *   workspace, workspace_bytes : see above (W_full^T, K * N elements).
+ * M == 0 is a no-op. Errors: BAD_HANDLE, INVALID_ARG (sizes, dtype, NULL pointer, workspace too
+ * small), MISALIGNED (dY, Wc, dX not 16-byte or workspace not 256-byte aligned), CUDA,
+ * DEVICE_TIMEOUT (as for ss1_forward).
+ */
+SS1_API int ss1_backward_input(ss1_handle h, const void* dY, const void* Wc, void* dX, int64_t M, int dtype,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ss1_backward_weight -- dWc, the gradient with respect to the compressed weights.
+ *   X  : device, [M, K] of `dtype` (the forward's input).   dY : device, [M, N].
+ *   dWc: device, [N, K / c], written (overwritten, not accumulated); zero when M == 0.
+ *   workspace, workspace_bytes : see above (dY^T and X^T padded to a multiple of 64 rows, and
+ *   the dense gradient dY^T X).
+ * Errors: as ss1_backward_input (X, dY, dWc 16-byte aligned).
+ */
+SS1_API int ss1_backward_weight(ss1_handle h, const void* X, const void* dY, void* dWc, int64_t M, int dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * FP8 weights. "SS1: Accelerating Inference with Fast and Expressive Sketch Structured
+ * Transform", section "Limitations": quantised SS1 kernels were not built; section "Measured
+ * effects": post-training quantisation of SS1 models. The pages fix no format; this library
+ * stores the compressed weights as OCP FP8 E4M3 codes (1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits, largest magnitude 448, no infinities) with one float scale per output neuron:
+ *
+ *     Wc_deq[n, j] = scale[n] * e4m3(Wq[n, j]),   Y = SS1(X) computed with Wc_deq.
+ */
+
+/*
+ * ss1_quantize_fp8 -- per-neuron FP8 quantisation of compressed weights (no handle needed).
+ *   Wc    : device, [N, Kc] of `dtype` (bf16 or fp32).
+ *   Wq    : device, [N, Kc] bytes, written: E4M3 codes of Wc[n, j] / scale[n], rounded to nearest
+ *           even, magnitudes past 448 saturated to 448.
+ *   scale : device, [N] float, written: max_j |Wc[n, j]| / 448 (correctly rounded float32
+ *           division), or 1 for an all-zero row.
+ * Asynchronous. Errors: INVALID_ARG (sizes, dtype, NULL), MISALIGNED (Wc not aligned to its
+ * element, scale to 4 bytes), CUDA.
+ */
+SS1_API int ss1_quantize_fp8(const void* Wc, int dtype, int64_t N, int64_t Kc, void* Wq, float* scale, void* stream);
+
+/*
+ * ss1_forward_fp8 -- Y = SS1(X) with FP8 weights (Wq, scale), for decode-sized batches.
+ *   X : device, bf16 [M, K].   Wq : device, [N, K / c] E4M3 codes.   scale : device, float [N].
+ *   Y : device, bf16 [M, N], written.   M : 0 .. 64 (M == 0 is a no-op).
+ * Runs the tensor-core decode kernel: Wc streams as one byte per weight, each stage is widened
+ * to bf16 on chip (exactly), the sketch is as in ss1_forward, products accumulate in fp32, and
+ * Y[m, n] = bf16(scale[n] * sum). Re-entrant like ss1_forward.
+ * Errors: BAD_HANDLE, INVALID_ARG, MISALIGNED (X, Wq, Y 16-byte, scale 4-byte aligned),
+ * UNSUPPORTED_SHAPE (M > 64, BN != 128, K / c not a multiple of 16), CUDA, DEVICE_TIMEOUT.
+ */
+SS1_API int ss1_forward_fp8(ss1_handle h, const void* X, const void* Wq, const float* scale, void* Y, int64_t M,
+                            void* stream);
 
 /* Table entries ((N / BN) * K) that ss1_forward_noalloc accepts at most. */
 #define SS1_NOALLOC_MAX_ENTRIES 983040
@@ -178,16 +279,16 @@ SS1_API const char* ss1_strerror(int status);
  *
  * Every call regenerates the tables on `stream` into one fixed region of device memory
  * that the library reserves statically (16 MiB per device: 17 bytes per table entry plus
- * padding), then runs the kernel ss1_forward would choose. The decode-sized path (M <= 64)
- * splits K across CTAs as it does for a handle, with a second static region of 12 MiB for the
- * fp32 partials and 3 KiB of arrival counters; the call clears those counters on `stream`.
+ * padding), then runs the kernel ss1_forward would choose, with the same results bit for bit.
  * Shapes with (N / BN) * K > SS1_NOALLOC_MAX_ENTRIES are rejected with UNSUPPORTED_SHAPE. No
  * cudaMalloc, cudaFree, pinned allocation or allocating library routine is called, and
  * nothing synchronises the device; the tables need no zeroing because the table kernels
  * write all of them that the forward reads.
  *
  * The first call on a device does one-time set-up (it looks up the region's address and
- * sets kernel attributes); make that first call outside any stream capture.
+ * sets kernel attributes); make that first call outside any stream capture. The set-up belongs
+ * to the device's CUDA context: after cudaDeviceReset the next call on that device runs it
+ * again in the new context (so that call, too, should come before any stream capture).
  * Calls share the one region: two calls whose work can overlap on the device (different
  * streams without ordering, or different host threads) race on the tables and give wrong
  * results. Order them on one stream or with events. Asynchronous: returns after the

@@ -2,8 +2,12 @@
 // The operation and every entry point are specified in include/ss1.h.
 #include "ss1_internal.cuh"
 
+#include <cuda.h>
+
+#include <functional>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <unordered_map>
 #include <unordered_set>
 
@@ -20,6 +24,12 @@ bool live(const ss1_layer* h) {
     return h != nullptr && g_live.count(h) != 0 && h->magic == kMagic;
 }
 
+struct PairHash {
+    size_t operator()(const std::pair<const void*, uint64_t>& k) const {
+        return std::hash<const void*>()(k.first) ^ (std::hash<uint64_t>()(k.second) * 0x9E3779B97F4A7C15ull);
+    }
+};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 void release(ss1_layer* L) {
@@ -29,8 +39,6 @@ void release(ss1_layer* L) {
     if (L->d_src) cudaFree(L->d_src);
     if (L->d_gather) cudaFree(L->d_gather);
     if (L->d_slot) cudaFree(L->d_slot);
-    if (L->d_dec_ws) cudaFree(L->d_dec_ws);
-    if (L->d_dec_cnt) cudaFree(L->d_dec_cnt);
     if (L->status_host) cudaFreeHost(L->status_host);
     L->magic = 0;
     delete L;
@@ -49,17 +57,42 @@ namespace ss1 {
 
 bool handle_live(const ss1_layer* h) { return live(h); }
 
+uint64_t current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+        cudaGetLastError();
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return (uint64_t)id;
+}
+
 cudaError_t smem_attr_once(const void* kernel, int bytes) {
     static std::mutex mu;
-    static std::unordered_map<const void*, uint64_t> done;   // kernel -> bit d set once device d has it
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
+    static std::unordered_set<std::pair<const void*, uint64_t>, PairHash> done;   // (kernel, context id)
+    const uint64_t ctx = current_context_id();
     std::lock_guard<std::mutex> lk(mu);
-    uint64_t& mask = done[kernel];
-    if (dev < 64 && ((mask >> dev) & 1u)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev < 64) mask |= (uint64_t)1 << dev;
+    if (ctx != 0 && done.count({kernel, ctx})) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // the attribute call makes the device's context current, so its id is known from here on
+    const uint64_t now = current_context_id();
+    if (e == cudaSuccess && now != 0) done.insert({kernel, now});
     return e;
 }
 
@@ -126,19 +159,6 @@ SS1_API int ss1_create(int64_t K, int64_t N, int c, int BK, int BN, uint64_t see
         return SS1_ERR_OUT_OF_MEMORY;
     }
     *L->status_host = 0;
-    if (ss1::dec_supported(*L, 1) && L->NB <= L->num_sms) {   // K-split partials of the decode kernel
-        if (cudaMalloc(&L->d_dec_ws, ss1::dec_workspace_floats(*L) * sizeof(float)) != cudaSuccess ||
-            cudaMalloc(&L->d_dec_cnt, (size_t)L->NB * 4 * sizeof(uint32_t)) != cudaSuccess) {
-            cudaGetLastError();
-            release(L);
-            return SS1_ERR_OUT_OF_MEMORY;
-        }
-        if (cudaMemset(L->d_dec_cnt, 0, (size_t)L->NB * 4 * sizeof(uint32_t)) != cudaSuccess) {
-            cudaGetLastError();
-            release(L);
-            return SS1_ERR_CUDA;
-        }
-    }
     if (cudaHostGetDevicePointer((void**)&L->status_dev, L->status_host, 0) != cudaSuccess) {
         cudaGetLastError();
         release(L);
@@ -204,15 +224,6 @@ SS1_API int ss1_device_status(ss1_handle h, int32_t* detail) {
     if (!live(h)) return SS1_ERR_BAD_HANDLE;
     const int32_t v = __atomic_exchange_n(h->status_host, 0, __ATOMIC_ACQ_REL);
     if (detail) *detail = v;
-    if (v != 0 && h->d_dec_cnt) {   // a launch that gave up may have left split counters behind
-        int prev = -1;
-        cudaGetDevice(&prev);
-        if (prev != h->device) cudaSetDevice(h->device);
-        cudaDeviceSynchronize();
-        cudaMemset(h->d_dec_cnt, 0, (size_t)h->NB * 4 * sizeof(uint32_t));
-        cudaGetLastError();
-        if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
-    }
     return v == 0 ? SS1_OK : SS1_ERR_DEVICE_TIMEOUT;
 }
 

@@ -21,18 +21,24 @@
 //                K-chunks) arrive by TMA (one more lane of warp 0) into a two-unit ring;
 //                otherwise the CTA's X columns are copied in once where they fit in 20 KB, or
 //                the gathers go to L1 / L2. Then the epilogue.
-// Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: every warp writes its
-// 32 neurons' fp32 partial to the workspace and counts itself in; the last warp to arrive for
-// those neurons sums all splits' partials in split order (the same bits every call), writes Y
-// and resets its counter.
-// Every wait is bounded; a wait that runs out sets the CTA's abort flag and the status word.
+// Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: the K-splits of one
+// N-block form one thread-block cluster. Every CTA leaves its fp32 partial [rows x 128 neurons]
+// in its own shared memory; after a cluster barrier, CTA r sums rows r, r + splits, ... over the
+// splits' partials, read through distributed shared memory in split order (the same bits every
+// call), and writes them to Y. Nothing is written outside X, Wc and Y, so calls are re-entrant.
+// Every mbarrier wait is bounded; a wait that runs out sets the CTA's abort flag and the status
+// word, and every thread still reaches both cluster barriers.
 #include "ss1_internal.cuh"
 #include "ptx_sm100.cuh"
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 namespace ss1 {
 
@@ -42,15 +48,14 @@ namespace {
 
 constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
 constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
-constexpr int kWStage = kNeu * kStageC * 2;   // 16 KB of Wc per stage
-constexpr int kNW = 4;                    // Wc stages in the ring
+constexpr int kWRing = 64 * 1024;         // shared memory of the Wc ring: 4 bf16 or 8 FP8 stages
 constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
 constexpr int kNB = 3;                    // sketch stages in the ring
 constexpr int kPrefetchStages = 16;       // Wc stages asked of L2 before the previous kernel ends
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
-constexpr int kThreads = (kFirstBuild + kBuildWarps) * 32;
+constexpr int kFirstConv = kFirstBuild + kBuildWarps, kConvWarps = 4;   // FP8 weights: the converter warps
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // L2 prefetch of one 2D tile of a tensor map: no shared memory, no completion to wait for.
@@ -68,20 +73,40 @@ __device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int c0, i
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-template <int MP>
+// FP8 = true: Wc arrives as E4M3 codes [128 neurons x 64 columns] (8 KB, 64-byte swizzle); four
+// converter warps widen each stage to bf16 (exact) straight into TMEM, where it is the UMMA's A
+// operand, and the epilogue multiplies neuron n's sum by its scale.
+template <int MP, bool FP8>
 struct DecCfg {
+    static constexpr int W_STAGE = kNeu * kStageC * (FP8 ? 1 : 2);   // 8 or 16 KB
+    static constexpr int NW = kWRing / W_STAGE;                       // Wc stages in the ring (8 or 4)
+    static constexpr int THREADS = (kFirstBuild + kBuildWarps + (FP8 ? kConvWarps : 0)) * 32;
+    static constexpr int MIN_CTAS = (FP8 && MP == 64) ? 1 : 2;          // registers: 168 for MP = 64
     static constexpr int B_STAGE = MP * 128;                    // [MP rows x 64] bf16
     static constexpr int OFF_W = 0;
-    static constexpr int OFF_B = kNW * kWStage;
+    static constexpr int OFF_B = kWRing;
     static constexpr int OFF_X = OFF_B + kNB * B_STAGE;
     static constexpr int X_BYTES = MP == kXChunkRows ? 2 * kXUnitBytes : kXBytes;   // the ring, or the range
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
-    static constexpr int NBAR = 2 * kNW + 2 * kNB + 1 + 4;
+    static constexpr int NBAR = 2 * NW + 2 * kNB + 1 + 4;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-    static constexpr uint32_t TMEM_COLS = MP <= 32 ? 32 : 64;
+    // accumulator MP columns; FP8: plus kNB bf16 A stages of 32 columns from A_COL
+    static constexpr int A_COL = MP <= 32 ? 32 : 64;
+    static constexpr uint32_t TMEM_COLS = FP8 ? (MP <= 32 ? 128 : 256) : (MP <= 32 ? 32 : 64);
     static_assert(MP % 16 == 0 && MP >= 16 && MP <= 64, "UMMA N for M = 128");
     static_assert(B_STAGE % 1024 == 0 && OFF_B % 1024 == 0, "swizzle atoms stay aligned");
+    static_assert(!FP8 || (A_COL >= MP && A_COL + kNB * 32 <= (int)TMEM_COLS), "TMEM layout");
+    static_assert(NW <= 31, "one loader lane per ring slot, plus the X lane");
 };
+
+// Two E4M3 codes (low byte = the even column) -> bf16x2, exactly: every E4M3 value has at most
+// four significant bits and an exponent inside bf16's range.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
 
 __device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
     *abort_flag = 1;
@@ -96,21 +121,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-template <int MP, int C>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int MP, int C, bool FP8>
+__global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN_CTAS)
     dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Y, const uint16_t* __restrict__ src,
-               int M, int K, int N, int S, int KC, int splits, int chunked, int ui, int bi, float* __restrict__ ws,
-               uint32_t* __restrict__ cnt, int32_t* status) {
-    using F = DecCfg<MP>;
+               const float* __restrict__ scale, int M, int K, int N, int S, int KC, int splits, int chunked, int ui,
+               int bi, int32_t* status) {
+    using F = DecCfg<MP, FP8>;
+    constexpr int kNW = F::NW, kWStage = F::W_STAGE, kThreads = F::THREADS, kACol = F::A_COL;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* wring = smem + F::OFF_W;
     uint8_t* bring = smem + F::OFF_B;
     uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + F::OFF_BAR);
     uint64_t* w_empty = w_full + kNW;
-    uint64_t* b_full = w_empty + kNW;     // the two build warps of the stage have written it
-    uint64_t* b_empty = b_full + kNB;     // the stage's UMMAs have completed
+    uint64_t* b_full = w_empty + kNW;     // the two build warps (and, FP8, the four converter warps) are done
+    uint64_t* b_empty = b_full + kNB;     // the stage's UMMAs have completed (its B stage and A stage are free)
     uint64_t* acc_full = b_empty + kNB;
     uint64_t* x_full = acc_full + 1;      // [2] chunk mode: an X chunk has landed
     uint64_t* x_empty = x_full + 2;       // [2] chunk mode: every stage of the chunk has been built
@@ -142,8 +168,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         reinterpret_cast<uint4*>(bring)[i] = make_uint4(0u, 0u, 0u, 0u);
     ptx::fence_proxy_async_smem();
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], 1); }
-        for (int i = 0; i < kNB; ++i) { ptx::mbar_init(&b_full[i], kBuildWarps / 2); ptx::mbar_init(&b_empty[i], 1); }
+        // FP8: a Wc slot is free once the converter warps have read it (bf16: once its UMMAs completed)
+        for (int i = 0; i < kNW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], FP8 ? kConvWarps : 1); }
+        for (int i = 0; i < kNB; ++i) {
+            ptx::mbar_init(&b_full[i], kBuildWarps / 2 + (FP8 ? kConvWarps : 0));
+            ptx::mbar_init(&b_empty[i], 1);
+        }
         ptx::mbar_init(acc_full, 1);
         for (int i = 0; i < 2; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
         *abort_flag = 0;
@@ -222,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool ok = true;
         for (int g = 0; g < G && ok; ++g) {
             const int ws_ = g % kNW, bs = g % kNB;
-            if (!warp_wait(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag) ||
+            if ((!FP8 && !warp_wait(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag)) ||
                 !warp_wait(&b_full[bs], (uint32_t)((g / kNB) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 2);
                 ok = false;
@@ -232,10 +262,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (lane == 0) {
                 const uint64_t wd = wdesc0 + (uint64_t)((ws_ * kWStage) >> 4);
                 const uint64_t bd = bdesc0 + (uint64_t)((bs * F::B_STAGE) >> 4);
+                const uint32_t at = tm + (uint32_t)(kACol + bs * 32);   // FP8: the stage's bf16 A in TMEM
 #pragma unroll
-                for (int kk = 0; kk < kStageC / 16; ++kk)
-                    ptx::umma_bf16_ss(tm, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
-                ptx::umma_commit(&w_empty[ws_]);
+                for (int kk = 0; kk < kStageC / 16; ++kk) {
+                    if (FP8)
+                        ptx::umma_bf16_ts(tm, at + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
+                    else
+                        ptx::umma_bf16_ss(tm, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (!FP8) ptx::umma_commit(&w_empty[ws_]);
                 ptx::umma_commit(&b_empty[bs]);
             }
             __syncwarp();
@@ -248,6 +283,46 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         __syncwarp();
+    } else if (FP8 && warp >= kFirstConv) {
+        // ------------------------------------------------------------------ FP8 -> bf16 A stages
+        // Thread = neuron (TMEM lane 32 q + lane, q = warp % 4): its row of the stage, 64 codes in
+        // four 16-byte chunks (64-byte swizzle: chunk c of row r sits at c ^ ((r >> 1) & 3), so
+        // eight rows read per wavefront hit distinct banks), widened to 32 bf16x2 words and
+        // stored into the stage's TMEM columns.
+        const int q = warp & 3, r = q * 32 + lane;
+        const uint32_t lanes = (uint32_t)(q * 32) << 16;
+        bool ok = true;
+        for (int g = 0; g < G && ok; ++g) {
+            const int ws_ = g % kNW, bs = g % kNB;
+            if (!warp_wait(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag) ||
+                (g >= kNB && !warp_wait(&b_empty[bs], (uint32_t)(((g / kNB) - 1) & 1), abort_flag))) {
+                if (lane == 0) report(status, abort_flag, 7);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint8_t* row = wring + ws_ * kWStage + r * 64;
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 u = *reinterpret_cast<const uint4*>(row + ((c ^ ((r >> 1) & 3)) << 4));
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[c * 8 + 2 * e] = e4m3x2_to_bf16x2((uint16_t)(w4[e] & 0xFFFFu));
+                    v[c * 8 + 2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[e] >> 16));
+                }
+            }
+            ptx::tmem_st_32x32b_x16(tm + lanes + (uint32_t)(kACol + bs * 32), *reinterpret_cast<const uint32_t(*)[16]>(v));
+            ptx::tmem_st_32x32b_x16(tm + lanes + (uint32_t)(kACol + bs * 32 + 16), *reinterpret_cast<const uint32_t(*)[16]>(v + 16));
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(&w_empty[ws_]);   // the codes have been read
+                ptx::mbar_arrive(&b_full[bs]);     // the A stage is in TMEM
+            }
+        }
     } else {
         // ------------------------------------------------------------------ sketch, then epilogue
         // Build thread t: column kl = t % 64 of the stages g with g % 2 == t / 64 (two stages are
@@ -353,32 +428,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int i = 0; i < 16; ++i) d[m0 + i] = __uint_as_float(r[i]);
             }
             if (splits == 1) {
+                const float sc = FP8 ? scale[n] : 1.0f;
 #pragma unroll
                 for (int m = 0; m < MP; ++m)
-                    if (m < M) Y[(size_t)m * N + n] = __float2bfloat16_rn(d[m]);
+                    if (m < M) Y[(size_t)m * N + n] = __float2bfloat16_rn(FP8 ? sc * d[m] : d[m]);
             } else {
-                // workspace: [N-block][split][MP rows][128 neurons] fp32
-                float* mine = ws + ((size_t)(nb * splits + split) * MP) * kNeu + quad * 32 + lane;
+                // this split's partial [MP rows][128 neurons] fp32, in the Wc ring: every stage has
+                // been multiplied (acc_full), so the ring is free
+                float* part = reinterpret_cast<float*>(wring) + quad * 32 + lane;
 #pragma unroll
                 for (int m = 0; m < MP; ++m)
-                    if (m < M) mine[(size_t)m * kNeu] = d[m];
-                __threadfence();
-                __syncwarp();
-                uint32_t prev = 0;
-                if (lane == 0) prev = atomicAdd(&cnt[nb * 4 + quad], 1u);
-                prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev == (uint32_t)(splits - 1)) {   // the last split of these neurons: reduce in order
-                    __threadfence();
-                    const float* base = ws + ((size_t)nb * splits * MP) * kNeu + quad * 32 + lane;
-#pragma unroll 1
-                    for (int m = 0; m < M && m < MP; ++m) {
-                        float v = 0.f;
-                        for (int s = 0; s < splits; ++s) v += __ldcg(base + ((size_t)s * MP + m) * kNeu);
-                        Y[(size_t)m * N + n] = __float2bfloat16_rn(v);
-                    }
-                    __syncwarp();
-                    if (lane == 0) cnt[nb * 4 + quad] = 0u;
-                }
+                    if (m < M) part[(size_t)m * kNeu] = d[m];
             }
         } else if (lane == 0 && !*abort_flag) {
             report(status, abort_flag, 4);
@@ -391,17 +451,37 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tm, F::TMEM_COLS);
     }
+    if (splits > 1) {
+        // The cluster is this N-block's splits (rank = split). After the first barrier every
+        // partial is visible to the cluster; the second keeps each CTA's shared memory alive
+        // until its peers have read it.
+        ptx::cluster_sync();
+        if (warp >= kFirstBuild && warp < kFirstBuild + kBuildWarps) {
+            const int t = threadIdx.x - kFirstBuild * 32;   // neuron of the N-block
+            const float* part = reinterpret_cast<const float*>(wring) + t;
+            const float sc = FP8 ? scale[(size_t)nb * kNeu + t] : 1.0f;
+            for (int m = (int)ptx::cluster_ctarank(); m < M && m < MP; m += splits) {
+                float v = 0.f;
+                for (int s = 0; s < splits; ++s) v += ptx::ld_cluster_f32(ptx::map_to_rank(part + (size_t)m * kNeu, (uint32_t)s));
+                Y[(size_t)m * N + (size_t)nb * kNeu + t] = __float2bfloat16_rn(FP8 ? sc * v : v);
+            }
+        }
+        ptx::cluster_sync();
+    }
 }
 
-bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+// Wc as [N rows x Kc columns]: bf16 with [128 x 64] boxes and the 128-byte swizzle, or E4M3
+// codes (one byte each) with [128 x 64] boxes and the 64-byte swizzle.
+bool make_map_w(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, bool fp8) {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
+    cuuint64_t strides[1] = {cols * (fp8 ? 1 : 2)};
     cuuint32_t box[2] = {kStageC, kNeu};
     cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -418,13 +498,72 @@ bool make_map_x(CUtensorMap* map, const void* base, uint64_t K, uint64_t M, uint
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MP, int C>
-cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    using F = DecCfg<MP>;
-    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&dec_kernel<MP, C>), F::SMEM);
+// How many clusters of `cs` CTAs (the K-splits of one N-block) the device keeps resident at once
+// for this kernel, for cs = 1 .. 16 (16 is a non-portable cluster size; 0 where a size does not
+// fit at all). Clusters are placed whole inside one GPC, so this is not simply the CTA slots
+// divided by cs. Looked up once per (kernel, context).
+struct ClusterFit {
+    int active[17] = {};
+};
+
+ClusterFit cluster_fit(const void* fn, int smem, int threads) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, uint64_t>, ClusterFit> done;
+    const uint64_t ctx = current_context_id();
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = done.find({fn, ctx});
+    if (ctx != 0 && it != done.end()) return it->second;
+    ClusterFit f;
+    cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaGetLastError();
+    for (int cs = 1; cs <= 16; ++cs) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, (unsigned)cs);
+        cfg.blockDim = dim3((unsigned)threads);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = 1;
+        a[0].val.clusterDim.y = (unsigned)cs;
+        a[0].val.clusterDim.z = 1;
+        cfg.attrs = a;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess) f.active[cs] = n;
+        cudaGetLastError();
+    }
+    const uint64_t now = current_context_id();
+    if (now != 0) done[{fn, now}] = f;
+    return f;
+}
+
+// K-splits per N-block: the largest count up to `want` (and `units`) whose NB clusters all fit
+// on the device at once; where none does, the one that keeps the most CTAs resident.
+int pick_splits(const ClusterFit& f, int NB, int want, int units) {
+    int hi = want < units ? want : units;
+    hi = hi > 16 ? 16 : hi;
+    if (hi <= 1) return 1;
+    int best = 1, best_ctas = 0;
+    for (int s = hi; s >= 1; --s) {
+        if (f.active[s] >= NB) return s;
+        const int resident = (f.active[s] < NB ? f.active[s] : NB) * s;
+        if (resident > best_ctas) { best_ctas = resident; best = s; }
+    }
+    return best;
+}
+
+template <int MP, int C, bool FP8>
+cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, const float* scale, void* Y, int64_t M,
+                       cudaStream_t st) {
+    using F = DecCfg<MP, FP8>;
+    const void* fn = reinterpret_cast<const void*>(&dec_kernel<MP, C, FP8>);
+    const cudaError_t attr_err = smem_attr_once(fn, F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
+    // CTAs per SM that the launch bounds allow; the K-split aims at that many per SM
+    const int per_sm = F::MIN_CTAS;
+    const ClusterFit fit = cluster_fit(fn, F::SMEM, F::THREADS);
     CUtensorMap mw, mx;
-    if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N)) return cudaErrorInvalidValue;
+    if (!make_map_w(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, FP8)) return cudaErrorInvalidValue;
     // Chunk mode: up to 16 rows and K-chunks of whole stages; each chunk's X rows then come by
     // TMA into a two-chunk ring and the sketch gathers read shared memory.
     const int Kc = (int)(L.K / L.c);
@@ -434,8 +573,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     const int bi = ui < 256 ? ui : 256;                                    // inputs per TMA box
     // The one-time copy of a CTA's X columns is cheaper where it fits; the ring is for the rest.
     const int nstg0 = (Kc + kStageC - 1) / kStageC;
-    int splits0 = L.d_dec_ws != nullptr ? (2 * L.num_sms) / L.NB : 1;
-    splits0 = splits0 < 1 ? 1 : (splits0 > nstg0 ? nstg0 : splits0);
+    const int splits0 = pick_splits(fit, L.NB, (per_sm * L.num_sms) / L.NB, nstg0);
     const int64_t range_max = ((int64_t)(nstg0 + splits0 - 1) / splits0 * kStageC / L.S + 2) * L.BK;   // inputs
     const bool range_fits = L.BK % 8 == 0 && M * range_max * 2 <= F::X_BYTES;
     const int chunked = (MP == kXChunkRows && !range_fits && L.BK % 8 == 0 && (whole_chunks || whole_stages) &&
@@ -445,41 +583,41 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     } else {
         mx = mw;   // unused
     }
-    // K-splits: about two CTAs per SM over all N-blocks, each with at least one stage (chunk
-    // mode: one K-chunk); a split needs the layer's workspace
+    // K-splits: about per_sm CTAs per SM over all N-blocks, each with at least one stage (chunk
+    // mode: one K-chunk), and at most one cluster's worth per N-block
     const int nstg = (int)((L.K / L.c + kStageC - 1) / kStageC);
     const int units = chunked ? (whole_chunks ? L.KC : nstg) : nstg;
-    int splits = 1;
-    if (L.d_dec_ws != nullptr) {
-        splits = (2 * L.num_sms) / L.NB;
-        if (splits > units) splits = units;
-        if (splits < 1) splits = 1;
-    }
-    // programmatic dependent launch: the CTAs may start while the previous kernel finishes
+    const int splits = pick_splits(fit, L.NB, (per_sm * L.num_sms) / L.NB, units);
+    // programmatic dependent launch: the CTAs may start while the previous kernel finishes; the
+    // splits of one N-block form a cluster
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)L.NB, (unsigned)splits);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(F::THREADS);
     cfg.dynamicSmemBytes = F::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = (unsigned)splits;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_kernel<MP, C>, mw, mx, (const __nv_bfloat16*)X,
-                                             (__nv_bfloat16*)Y, (const uint16_t*)L.d_src, (int)M, (int)L.K, (int)L.N,
-                                             L.S, L.KC, splits, chunked, ui, bi, L.d_dec_ws, L.d_dec_cnt,
-                                             L.status_dev);
+    cfg.numAttrs = splits > 1 ? 2 : 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_kernel<MP, C, FP8>, mw, mx, (const __nv_bfloat16*)X,
+                                             (__nv_bfloat16*)Y, (const uint16_t*)L.d_src, scale, (int)M, (int)L.K,
+                                             (int)L.N, L.S, L.KC, splits, chunked, ui, bi, L.status_dev);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int MP>
-cudaError_t launch_c(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+template <int MP, bool FP8>
+cudaError_t launch_c(const ss1_layer& L, const void* X, const void* Wc, const float* scale, void* Y, int64_t M,
+                     cudaStream_t st) {
     switch (L.c) {
-        case 1: return launch_cfg<MP, 1>(L, X, Wc, Y, M, st);
-        case 2: return launch_cfg<MP, 2>(L, X, Wc, Y, M, st);
-        case 4: return launch_cfg<MP, 4>(L, X, Wc, Y, M, st);
-        default: return launch_cfg<MP, 8>(L, X, Wc, Y, M, st);
+        case 1: return launch_cfg<MP, 1, FP8>(L, X, Wc, scale, Y, M, st);
+        case 2: return launch_cfg<MP, 2, FP8>(L, X, Wc, scale, Y, M, st);
+        case 4: return launch_cfg<MP, 4, FP8>(L, X, Wc, scale, Y, M, st);
+        default: return launch_cfg<MP, 8, FP8>(L, X, Wc, scale, Y, M, st);
     }
 }
 
@@ -492,15 +630,21 @@ bool dec_supported(const ss1_layer& L, int64_t M) {
     return true;
 }
 
-size_t dec_workspace_floats(const ss1_layer& L) {
-    // splits > 1 only where NB <= num_sms, and then NB * splits <= 2 * num_sms slots of 64 x 128
-    return (size_t)(2 * L.num_sms) * 64 * kNeu;
+cudaError_t launch_dec(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    if (M <= 16) return launch_c<16, false>(L, X, Wc, nullptr, Y, M, st);
+    if (M <= 32) return launch_c<32, false>(L, X, Wc, nullptr, Y, M, st);
+    return launch_c<64, false>(L, X, Wc, nullptr, Y, M, st);
 }
 
-cudaError_t launch_dec(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    if (M <= 16) return launch_c<16>(L, X, Wc, Y, M, st);
-    if (M <= 32) return launch_c<32>(L, X, Wc, Y, M, st);
-    return launch_c<64>(L, X, Wc, Y, M, st);
+bool dec_fp8_supported(const ss1_layer& L, int64_t M) {
+    return dec_supported(L, M) && (L.K / L.c) % 16 == 0;   // TMA: rows of Kc bytes, a multiple of 16
+}
+
+cudaError_t launch_dec_fp8(const ss1_layer& L, const void* X, const void* Wq, const float* scale, void* Y, int64_t M,
+                           cudaStream_t st) {
+    if (M <= 16) return launch_c<16, true>(L, X, Wq, scale, Y, M, st);
+    if (M <= 32) return launch_c<32, true>(L, X, Wq, scale, Y, M, st);
+    return launch_c<64, true>(L, X, Wq, scale, Y, M, st);
 }
 
 }  // namespace ss1

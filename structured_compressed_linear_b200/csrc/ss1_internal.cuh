@@ -26,10 +26,6 @@ struct ss1_layer {
     uint16_t* d_src;     // [NB][KC][S][c] slot-major sources (see above)
     uint2* d_gather;     // [NB][KC][BK] per source (slot-major): {k, bf16x2 multiplier (+-1, +-1)}
     uint16_t* d_slot;    // [NB][K] per input: slot inside its chunk (bits 0..7) | kSrcNegBit if the sign is -1
-    // Decode-path workspace (NULL: K is not split): fp32 partials of K-split CTAs, and one arrival
-    // counter per (N-block, 32-neuron quarter), zero between calls.
-    float* d_dec_ws;
-    uint32_t* d_dec_cnt;
     int32_t* status_host;  // pinned, host-mapped status word (0 = ok)
     int32_t* status_dev;   // device alias of status_host
 };
@@ -44,8 +40,12 @@ int auto_kernel(const ss1_layer& L, int64_t M, int dtype);
 // The shape checks of ss1_create.
 bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN);
 
-// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device. The attribute
-// belongs to a device context, so it is set once per (kernel, device); later calls return at once.
+// Unique id of the CUDA context current on this thread (cuCtxGetId), 0 if none is current yet.
+// Ids are never reused, so a context created after a device reset gets a new one.
+uint64_t current_context_id();
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` in the current context. The attribute
+// belongs to a context, so it is set once per (kernel, context); later calls return at once.
 cudaError_t smem_attr_once(const void* kernel, int bytes);
 
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);
@@ -59,7 +59,10 @@ cudaError_t launch_simt(const ss1_layer& L, const void* X, const void* Wc, void*
 // Decode-sized M (bf16): streams Wc once. The tensor-core decode kernel takes N-blocks of 128;
 // the CUDA-core one the rest.
 bool dec_supported(const ss1_layer& L, int64_t M);
-size_t dec_workspace_floats(const ss1_layer& L);
+// The same kernel with FP8 (E4M3) Wc and one float scale per neuron (Y = scale[n] * sum).
+bool dec_fp8_supported(const ss1_layer& L, int64_t M);
+cudaError_t launch_dec_fp8(const ss1_layer& L, const void* X, const void* Wq, const float* scale, void* Y, int64_t M,
+                           cudaStream_t st);
 cudaError_t launch_dec(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 bool smallm_supported(const ss1_layer& L, int64_t M);
 cudaError_t launch_smallm(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M,
@@ -75,5 +78,10 @@ cudaError_t launch_tc2(const ss1_layer& L, const void* X, const void* Wc, void* 
 bool tc3_supported(const ss1_layer& L);
 cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
+
+// Dense -> SS1 projection (bf16 or fp32): Wc[n, j] = scale * sum_{k : h(k) = j} g(k) W[n, k]
+// (scale = 1 / c for the projection, 1 for the weight gradient's tied sum).
+bool project_fast_ok(const ss1_layer& L, const void* W, const void* Wc, int dtype);
+cudaError_t launch_project(const ss1_layer& L, const void* W, void* Wc, int dtype, float scale, cudaStream_t st);
 
 }  // namespace ss1

@@ -11,7 +11,6 @@ namespace {
 constexpr size_t kRegionBytes = (size_t)16 << 20;   // the five tables
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSms = 192;                         // devices with more SMs run the decode kernel unsplit
 
 constexpr size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
@@ -23,31 +22,30 @@ constexpr size_t region_bytes_for(size_t entries) {
 }
 static_assert(region_bytes_for(SS1_NOALLOC_MAX_ENTRIES) <= kRegionBytes, "the largest accepted layer fits the region");
 
-// One region and one status word per device context that uses this entry point, and the decode
-// kernel's K-split scratch: fp32 partials (2 * SMs slots of 64 x 128) and arrival counters (four
-// per N-block, at most one N-block per SM when K is split).
+// One region and one status word per device context that uses this entry point.
 __device__ __align__(256) uint8_t g_region[kRegionBytes];
 __device__ __align__(256) int32_t g_status[64];
-__device__ __align__(256) float g_dec_ws[(size_t)2 * kMaxSms * 64 * 128];
-__device__ __align__(256) uint32_t g_dec_cnt[4 * kMaxSms];
 
 struct DeviceSlot {
     bool ready = false;
+    uint64_t context = 0;   // id of the context the addresses below belong to
     uint8_t* region = nullptr;
     int32_t* status = nullptr;
-    float* dec_ws = nullptr;
-    uint32_t* dec_cnt = nullptr;
     int num_sms = 0;
 };
 
 std::mutex g_mu;
 DeviceSlot g_dev[kMaxDevices];
 
-// One-time set-up per device: compute capability, SM count and the region's address.
+// One-time set-up per device context: compute capability, SM count and the regions' addresses.
+// A __device__ symbol has one address per context, so the set-up runs again when the device's
+// current context is not the one it ran in (after cudaDeviceReset, say).
 int device_slot(int dev, DeviceSlot* out) {
     std::lock_guard<std::mutex> lk(g_mu);
     DeviceSlot& d = g_dev[dev];
-    if (!d.ready) {
+    const uint64_t ctx = ss1::current_context_id();
+    if (!d.ready || ctx == 0 || ctx != d.context) {
+        d.ready = false;
         int major = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -57,21 +55,15 @@ int device_slot(int dev, DeviceSlot* out) {
         if (major != 10) return SS1_ERR_UNSUPPORTED_DEVICE;
         void* region = nullptr;
         void* status = nullptr;
-        void* dec_ws = nullptr;
-        void* dec_cnt = nullptr;
         if (cudaGetSymbolAddress(&region, g_region) != cudaSuccess ||
-            cudaGetSymbolAddress(&status, g_status) != cudaSuccess ||
-            cudaGetSymbolAddress(&dec_ws, g_dec_ws) != cudaSuccess ||
-            cudaGetSymbolAddress(&dec_cnt, g_dec_cnt) != cudaSuccess || region == nullptr || status == nullptr ||
-            dec_ws == nullptr || dec_cnt == nullptr) {
+            cudaGetSymbolAddress(&status, g_status) != cudaSuccess || region == nullptr || status == nullptr) {
             cudaGetLastError();
             return SS1_ERR_CUDA;
         }
         d.region = static_cast<uint8_t*>(region);
         d.status = static_cast<int32_t*>(status);
-        d.dec_ws = static_cast<float*>(dec_ws);
-        d.dec_cnt = static_cast<uint32_t*>(dec_cnt);
         d.num_sms = sms;
+        d.context = ss1::current_context_id();   // cudaGetSymbolAddress made the context current
         d.ready = true;
     }
     *out = d;
@@ -118,16 +110,8 @@ extern "C" SS1_API int ss1_forward_noalloc(int64_t K, int64_t N, int c, int BK, 
     L.status_host = nullptr;
     L.status_dev = device_status ? device_status : d.status;
 
-    // the decode kernel splits K as it does for a handle, with the static scratch; its counters
-    // start at zero every call
-    const bool dec_split = ss1::dec_supported(L, M) && L.NB <= L.num_sms && L.num_sms <= kMaxSms;
-    if (dec_split) {
-        L.d_dec_ws = d.dec_ws;
-        L.d_dec_cnt = d.dec_cnt;
-    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(L.status_dev, 0, sizeof(int32_t), st);
-    if (e == cudaSuccess && dec_split) e = cudaMemsetAsync(L.d_dec_cnt, 0, (size_t)L.NB * 4 * sizeof(uint32_t), st);
     if (e == cudaSuccess) e = ss1::launch_hashgen(L, st);
     if (e == cudaSuccess) e = ss1::launch_gather_tables(L, st);
     if (e == cudaSuccess) {

@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libss1.so")
 
 SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel", "ss1_destroy",
            "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc",
-           "ss1_test_device_timeout")
+           "ss1_test_device_timeout", "ss1_project", "ss1_backward_workspace", "ss1_backward_input",
+           "ss1_backward_weight", "ss1_quantize_fp8", "ss1_forward_fp8")
 
 #: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
 NOALLOC_MAX_ENTRIES = 983040
@@ -63,6 +64,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ss1_strerror.argtypes = [i32]
     L.ss1_forward_noalloc.argtypes = [i64, i64, i32, i32, i32, u64, vp, vp, vp, i64, i32, vp, vp]
     L.ss1_test_device_timeout.argtypes = [vp, i64, vp]
+    L.ss1_project.argtypes = [vp, vp, vp, i32, vp]
+    sz = ctypes.c_size_t
+    L.ss1_backward_workspace.argtypes = [vp, i64, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.ss1_backward_input.argtypes = [vp, vp, vp, vp, i64, i32, vp, sz, vp]
+    L.ss1_backward_weight.argtypes = [vp, vp, vp, vp, i64, i32, vp, sz, vp]
+    L.ss1_quantize_fp8.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+    L.ss1_forward_fp8.argtypes = [vp, vp, vp, vp, vp, i64, vp]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":
@@ -139,6 +147,88 @@ class SS1Layer:
 
     __call__ = forward
 
+    def project(self, W: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Wc[N, K/c] closest to the dense weight W[N, K] (ss1_project)."""
+        if W.dim() != 2 or W.shape != (self.N, self.K):
+            raise ValueError(f"W must be [{self.N}, {self.K}]")
+        if not W.is_cuda or not W.is_contiguous() or W.device.index != self.device:
+            raise ValueError(f"W must be a contiguous CUDA tensor on cuda:{self.device}")
+        shape = (self.N, self.K // self.c)
+        if out is None:
+            out = torch.empty(shape, dtype=W.dtype, device=W.device)
+        elif out.shape != shape or out.dtype != W.dtype or not out.is_contiguous() or out.device != W.device:
+            raise ValueError("out must be a contiguous [N, K/c] tensor of W's dtype on W's device")
+        st = stream if stream is not None else torch.cuda.current_stream(W.device)
+        _check(lib().ss1_project(self.handle, W.data_ptr(), out.data_ptr(), _dtype_code(W.dtype), st.cuda_stream),
+               "ss1_project")
+        return out
+
+    def backward_workspace(self, M: int, dtype: torch.dtype = torch.bfloat16) -> Tuple[int, int]:
+        """Workspace bytes of backward_input and backward_weight (ss1_backward_workspace)."""
+        a, b = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().ss1_backward_workspace(self.handle, M, _dtype_code(dtype), ctypes.byref(a), ctypes.byref(b)),
+               "ss1_backward_workspace")
+        return a.value, b.value
+
+    def _check_cuda(self, **tensors):
+        for name, t in tensors.items():
+            if not t.is_cuda or not t.is_contiguous() or t.device.index != self.device:
+                raise ValueError(f"{name} must be a contiguous CUDA tensor on cuda:{self.device}")
+
+    def backward_input(self, dY: torch.Tensor, Wc: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """dX[M, K] = dY[M, N] W_full (ss1_backward_input)."""
+        if dY.dim() != 2 or dY.shape[1] != self.N or Wc.shape != (self.N, self.K // self.c) or dY.dtype != Wc.dtype:
+            raise ValueError(f"dY must be [M, {self.N}] and Wc [{self.N}, {self.K // self.c}] of one dtype")
+        self._check_cuda(dY=dY, Wc=Wc)
+        M = dY.shape[0]
+        out = torch.empty((M, self.K), dtype=dY.dtype, device=dY.device) if out is None else out
+        need = self.backward_workspace(M, dY.dtype)[0]
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dY.device)
+        st = stream if stream is not None else torch.cuda.current_stream(dY.device)
+        _check(lib().ss1_backward_input(self.handle, dY.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
+                                        _dtype_code(dY.dtype), workspace.data_ptr(), workspace.numel(),
+                                        st.cuda_stream), "ss1_backward_input")
+        return out
+
+    def backward_weight(self, X: torch.Tensor, dY: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """dWc[N, K/c] from the forward's input X[M, K] and dY[M, N] (ss1_backward_weight)."""
+        if X.dim() != 2 or X.shape[1] != self.K or dY.shape != (X.shape[0], self.N) or X.dtype != dY.dtype:
+            raise ValueError(f"X must be [M, {self.K}] and dY [M, {self.N}] of one dtype")
+        self._check_cuda(X=X, dY=dY)
+        M = X.shape[0]
+        out = torch.empty((self.N, self.K // self.c), dtype=X.dtype, device=X.device) if out is None else out
+        need = self.backward_workspace(M, X.dtype)[1]
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+        st = stream if stream is not None else torch.cuda.current_stream(X.device)
+        _check(lib().ss1_backward_weight(self.handle, X.data_ptr(), dY.data_ptr(), out.data_ptr(), M,
+                                         _dtype_code(X.dtype), workspace.data_ptr(), workspace.numel(),
+                                         st.cuda_stream), "ss1_backward_weight")
+        return out
+
+    def forward_fp8(self, X: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Y[M, N] (bf16) with FP8 weights: Wq uint8 E4M3 codes [N, K/c], scale float32 [N] (ss1_forward_fp8)."""
+        if X.dim() != 2 or X.shape[1] != self.K or X.dtype != torch.bfloat16:
+            raise ValueError(f"X must be bf16 [M, {self.K}]")
+        if Wq.shape != (self.N, self.K // self.c) or Wq.dtype != torch.uint8:
+            raise ValueError(f"Wq must be uint8 [{self.N}, {self.K // self.c}]")
+        if scale.shape != (self.N,) or scale.dtype != torch.float32:
+            raise ValueError(f"scale must be float32 [{self.N}]")
+        self._check_cuda(X=X, Wq=Wq, scale=scale)
+        M = X.shape[0]
+        out = torch.empty((M, self.N), dtype=torch.bfloat16, device=X.device) if out is None else out
+        st = stream if stream is not None else torch.cuda.current_stream(X.device)
+        _check(lib().ss1_forward_fp8(self.handle, X.data_ptr(), Wq.data_ptr(), scale.data_ptr(), out.data_ptr(), M,
+                                     st.cuda_stream), "ss1_forward_fp8")
+        return out
+
     def select_kernel(self, M: int, dtype: torch.dtype = torch.bfloat16) -> Kernel:
         k = ctypes.c_int()
         _check(lib().ss1_select_kernel(self.handle, M, _dtype_code(dtype), ctypes.byref(k)), "ss1_select_kernel")
@@ -199,3 +289,36 @@ def forward_noalloc(X: torch.Tensor, Wc: torch.Tensor, K: int, N: int, c: int, B
                                      out.data_ptr(), M, _dtype_code(X.dtype), status_ptr, st.cuda_stream),
            "ss1_forward_noalloc")
     return out
+
+
+def quantize_fp8(Wc: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(Wq uint8 [N, Kc], scale float32 [N]) from bf16 or fp32 Wc[N, Kc] (ss1_quantize_fp8)."""
+    if Wc.dim() != 2 or not Wc.is_cuda or not Wc.is_contiguous():
+        raise ValueError("Wc must be a contiguous 2-D CUDA tensor")
+    N, Kc = Wc.shape
+    Wq = torch.empty((N, Kc), dtype=torch.uint8, device=Wc.device)
+    scale = torch.empty((N,), dtype=torch.float32, device=Wc.device)
+    st = stream if stream is not None else torch.cuda.current_stream(Wc.device)
+    _check(lib().ss1_quantize_fp8(Wc.data_ptr(), _dtype_code(Wc.dtype), N, Kc, Wq.data_ptr(), scale.data_ptr(),
+                                  st.cuda_stream), "ss1_quantize_fp8")
+    return Wq, scale
+
+
+class SS1Function(torch.autograd.Function):
+    """Autograd wrapper: Y = SS1(X; Wc) with the CUDA forward and backward entry points.
+
+    Usage: Y = SS1Function.apply(X, Wc, layer) with `layer` an SS1Layer."""
+
+    @staticmethod
+    def forward(ctx, X, Wc, layer):
+        ctx.layer = layer
+        ctx.save_for_backward(X, Wc)
+        return layer.forward(X.contiguous(), Wc.contiguous())
+
+    @staticmethod
+    def backward(ctx, dY):
+        X, Wc = ctx.saved_tensors
+        dY = dY.contiguous()
+        dX = ctx.layer.backward_input(dY, Wc) if ctx.needs_input_grad[0] else None
+        dWc = ctx.layer.backward_weight(X, dY) if ctx.needs_input_grad[1] else None
+        return dX, dWc, None

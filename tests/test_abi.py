@@ -68,6 +68,16 @@ def test_argument_checks_before_device(lib):
     assert lib.ss1_destroy(bogus) == -7
     assert lib.ss1_test_device_timeout(None, 1000000, None) == -7
     assert lib.ss1_test_device_timeout(bogus, 1000000, None) == -7
+    assert lib.ss1_project(None, None, None, 0, None) == -7
+    assert lib.ss1_project(bogus, None, None, 0, None) == -7
+    assert lib.ss1_backward_workspace(bogus, 1, 0, None, None) == -7
+    assert lib.ss1_backward_input(bogus, None, None, None, 1, 0, None, 0, None) == -7
+    assert lib.ss1_backward_weight(bogus, None, None, None, 1, 0, None, 0, None) == -7
+    assert lib.ss1_forward_fp8(bogus, None, None, None, None, 1, None) == -7
+    assert lib.ss1_quantize_fp8(None, 0, 4, 8, None, None, None) == -1       # NULL pointers
+    assert lib.ss1_quantize_fp8(None, 5, 4, 8, None, None, None) == -1       # dtype
+    assert lib.ss1_quantize_fp8(None, 0, 0, 8, None, None, None) == 0        # no rows: nothing to do
+    assert lib.ss1_quantize_fp8(0x1001, 0, 4, 8, 0x2000, 0x3000, None) == -5  # Wc not 2-byte aligned
     # the allocation-free forward checks its arguments and its table limit first
     fwd = lib.ss1_forward_noalloc
     assert fwd(768, 768, 3, 64, 64, 0, None, None, None, 1, 0, None, None) == -1         # c

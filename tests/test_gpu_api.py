@@ -154,7 +154,6 @@ def test_small_m_repeated_calls_bit_identical(M):
     layer.close()
 
 
-@pytest.mark.skip(reason="written, not yet run on a GPU: enable after its first run")
 def test_device_timeout_is_reported_and_cleared():
     """A bounded wait that runs out (on a barrier nothing completes) sets the handle's status
     word; the next forward reports SS1_ERR_DEVICE_TIMEOUT, ss1_device_status gives the site and
@@ -181,4 +180,37 @@ def test_device_timeout_is_reported_and_cleared():
     ref = O.ss1_forward(to_np64(X), to_np64(Wc), h, g, BN)
     got = to_np64(Y.cpu())
     assert float((np.abs(got - ref).max(1) / np.abs(ref).max(1)).max()) <= 2e-2
+    layer.close()
+
+
+@pytest.mark.parametrize("K,N,c", [(4096, 4096, 2), (4096, 1024, 8), (4096, 14336, 2)])
+def test_decode_calls_on_one_handle_run_concurrently(K, N, c):
+    """ss1_forward only reads the handle: decode-sized calls on one handle, issued on two streams
+    with no ordering between them (many launches, so they overlap on the device), each match the
+    oracle and agree with a serial call bit for bit. The decode kernel's K-split partial sums stay
+    inside one thread-block cluster's shared memory."""
+    ss1 = get_ss1()
+    BK, BN = 256, 128
+    layer = _layer(ss1, K, N, c, BK, BN, seed=31)
+    gen = torch.Generator().manual_seed(K + N + c)
+    Xs = [torch.randn(M, K, generator=gen).to(torch.bfloat16) for M in (1, 5, 16)]
+    Wc = (torch.randn(N, K // c, generator=gen) * 0.02).to(torch.bfloat16)
+    Wd = Wc.cuda()
+    Xd = [x.cuda() for x in Xs]
+    serial = [layer.forward(x, Wd) for x in Xd]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [[torch.empty_like(y) for y in serial] for _ in range(8)]
+    for it in range(8):
+        for i, (x, st) in enumerate(zip(Xd, streams)):
+            layer.forward(x, Wd, out=outs[it][i], stream=st)
+    torch.cuda.synchronize()
+    assert layer.device_status() == (0, 0)
+    h, g = O.ss1_tables(K, N, c, BK, BN, 31)
+    for i, x in enumerate(Xs):
+        ref = O.ss1_forward(to_np64(x), to_np64(Wc), h, g, BN)
+        got = to_np64(serial[i].cpu())
+        assert float((np.abs(got - ref).max(1) / np.abs(ref).max(1)).max()) <= 2e-2
+        for it in range(8):
+            assert torch.equal(outs[it][i], serial[i])
     layer.close()
