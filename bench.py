@@ -50,9 +50,16 @@ def parse():
     ap.add_argument("--decode-block", type=int, choices=[2, 8], default=None, metavar="C",
                     help="time one Llama-3-8B block's seven projections back to back at compression C "
                          "(rows: --m, default 1) instead of the workload step")
-    ap.add_argument("--op", choices=["forward", "project", "backward"], default="forward",
+    ap.add_argument("--op", choices=["forward", "project", "backward", "chain"], default="forward",
                     help="project: time ss1_project (dense W[N, K] -> Wc[N, K/c]) on the workload's layer shapes; "
-                         "backward: time ss1_backward_input + ss1_backward_weight on the workload's layers")
+                         "backward: time ss1_backward_input + ss1_backward_weight on the workload's layers; "
+                         "chain: the DLRM top-MLP chain (bias + ReLU between layers) as one ss1_chain_forward")
+    ap.add_argument("--graph", action="store_true",
+                    help="--decode-block: capture the block's launches in a CUDA graph and replay it (GPU time "
+                         "without the host's per-launch cost)")
+    ap.add_argument("--only", default=None, metavar="KxNcC",
+                    help="keep only the workload's layers of this shape and compression, e.g. 4096x14336c2 "
+                         "(a smaller step for profiling one kernel launch)")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 (E4M3) weights with per-neuron scales (ss1_forward_fp8; decode-sized rows only)")
     ap.add_argument("--nvtx", action="store_true",
@@ -280,13 +287,29 @@ def run_decode_block(args, peaks, peak_src, dev):
     for s in range(max(3, args.warmup) * ncopy):
         block(s % ncopy)
     torch.cuda.synchronize()
+    graph = None
+    if args.graph:   # one graph holding a block on every Wc copy, replayed; set-up already done above
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for cp in range(ncopy):
+                block(cp)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for s in range(args.steps):
-        block(s % ncopy)
+    if graph is not None:
+        reps = max(1, args.steps // ncopy)
+        for _ in range(reps):
+            graph.replay()
+        nblocks = reps * ncopy
+    else:
+        for s in range(args.steps):
+            block(s % ncopy)
+        nblocks = args.steps
     e1.record()
     torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) / args.steps * 1e3
+    us = e0.elapsed_time(e1) / nblocks * 1e3
     for layer in layers:
         st, detail = layer.device_status()
         if st != 0:
@@ -300,7 +323,8 @@ def run_decode_block(args, peaks, peak_src, dev):
         "higher_is_better": False, "dtype": "bf16 activations, " + ("e4m3 weights" if args.fp8 else "bf16 weights"),
         "data": "synthetic",
         "config": {"workload": f"llama-3-8b block at M={M}, c={c}, BK=256, BN=128", "kernels": kernels,
-                   "l2": f"Wc rotated over {ncopy} copies ({ncopy * wc_bytes / 1e6:.0f} MB), no flush"},
+                   "l2": f"Wc rotated over {ncopy} copies ({ncopy * wc_bytes / 1e6:.0f} MB), no flush",
+                   "launch": "CUDA graph replay" if graph is not None else "one API call per layer from Python"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes": byts,
                      "peak_source": peak_src},
@@ -453,6 +477,81 @@ def run_backward(args, layers, wid, peaks, peak_src, dev):
     }), flush=True)
 
 
+def run_chain(args, layers, wid, peaks, peak_src, dev):
+    """The DLRM top-MLP chain of the sweep workload (1024 -> 1024 -> 512 -> 256 at M = 65536, c = 2):
+    bias + ReLU after the first two layers, one ss1_chain_forward per step (one persistent launch
+    when the layers allow it), against the same layers as three ss1_forward_ex calls. L2 flushed
+    before every step; CUDA events around the chain."""
+    import torch
+    from structured_compressed_linear_b200 import ss1
+    from structured_compressed_linear_b200.workloads import WORKLOADS, make_inputs
+    chain = [L for L in WORKLOADS[5] if L.workload == "dlrm-top-mlp"]
+    X, _ = make_inputs(chain[0])
+    lays, Wcs, bs = [], [], []
+    gen = torch.Generator().manual_seed(5)
+    for L in chain:
+        lays.append(ss1.SS1Layer(L.K, L.N, L.c, L.BK, L.BN, L.seed))
+        Wcs.append(make_inputs(L)[1].to(dev))
+        bs.append((torch.randn(L.N, generator=gen) * 0.1).to(torch.bfloat16).to(dev))
+    acts = [ss1.Act.RELU, ss1.Act.RELU, ss1.Act.NONE]
+    Xd = X.to(dev)
+    outs = [torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev) for L in chain]
+    fused = ss1.chain_fused(lays)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def as_chain():
+        ss1.chain_forward(lays, Xd, Wcs, bs, acts, outs)
+
+    def by_layer():
+        cur = Xd
+        for ly, W, b, a, o in zip(lays, Wcs, bs, acts, outs):
+            ly.forward_ex(cur, W, b, a, out=o)
+            cur = o
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ts)
+
+    sampler = ClockSampler(dev.index or 0)
+    with sampler:
+        ms_chain = timed(as_chain)
+        ms_layers = timed(by_layer)
+    for ly in lays:
+        st, detail = ly.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {detail:#x}")
+        ly.close()
+    dense = sum(layer_work(L)[0] for L in chain)
+    actual = sum(layer_work(L)[1] for L in chain)
+    t_roof = sum(max(layer_work(L)[1] / (peaks["bf16_tflops"] * 1e12), layer_work(L)[2] / (peaks["hbm_gbs"] * 1e9))
+                 for L in chain)
+    print(json.dumps({
+        "metric": "SS1 DLRM top-MLP chain (1024-1024-512-256, bias + ReLU) dense-equiv TFLOP/s on 1 B200",
+        "value": dense / (ms_chain * 1e-3) / 1e12, "unit": "TFLOP/s (dense-equivalent 2*M*N*K per layer)",
+        "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_chain,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded, the sweep workload's chain)",
+        "config": {"workload": f"dlrm-top-mlp chain at M = {chain[0].M}, c = 2, BK = BN = 128",
+                   "one_launch": fused, "l2": "flushed before every step"},
+        "layer_by_layer_ms": ms_layers,
+        "roofline": {"bound": "per layer, the slower of tensor and HBM", "achieved_tflops": actual / (ms_chain * 1e-3) / 1e12,
+                     "frac": t_roof / (ms_chain * 1e-3), "frac_layer_by_layer": t_roof / (ms_layers * 1e-3),
+                     "peak_source": peak_src},
+        "gpu_launches": args.steps * (1 if fused else len(chain)), "clocks": sampler.summary(),
+    }), flush=True)
+
+
 def run_reference(args, layers, wid, rank, world):
     if rank != 0:
         return
@@ -522,8 +621,9 @@ def workload_config(layers, wid, world):
     }
 
 
-def select_layers(workload, m):
-    """The layers one bench step runs: the workload's layers at row count m, or at its largest."""
+def select_layers(workload, m, only=None):
+    """The layers one bench step runs: the workload's layers at row count m, or at its largest;
+    with `only` ("KxNcC"), just the layers of that shape and compression."""
     from structured_compressed_linear_b200.workloads import WORKLOADS, BENCH_WORKLOAD
     wid = workload or BENCH_WORKLOAD
     layers = WORKLOADS[wid]
@@ -533,6 +633,10 @@ def select_layers(workload, m):
             raise SystemExit(f"workload {wid} has no layers with M = {m}")
     elif len({L.M for L in layers}) != 1:
         layers = [L for L in layers if L.M == max(x.M for x in layers)]
+    if only is not None:
+        layers = [L for L in layers if f"{L.K}x{L.N}c{L.c}" == only]
+        if not layers:
+            raise SystemExit(f"workload {wid} has no layer {only}")
     return wid, layers
 
 
@@ -553,9 +657,9 @@ def main():
         run_decode_block(args, peaks, peak_src, torch.device("cuda", local))
         return
 
-    wid, layers = select_layers(args.workload, args.m)
+    wid, layers = select_layers(args.workload, args.m, args.only)
 
-    if args.op in ("project", "backward"):   # one GPU: the projection or the backward kernels
+    if args.op in ("project", "backward", "chain"):   # one GPU: projection, backward, or the MLP chain
         if rank != 0:
             return
         import torch
@@ -563,7 +667,7 @@ def main():
         build.build()
         torch.cuda.set_device(local)
         peaks, peak_src = load_peaks()
-        run = run_project if args.op == "project" else run_backward
+        run = {"project": run_project, "backward": run_backward, "chain": run_chain}[args.op]
         run(args, layers, wid, peaks, peak_src, torch.device("cuda", local))
         return
 

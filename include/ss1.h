@@ -58,6 +58,16 @@ enum ss1_kernel {
     SS1_KERNEL_SMALLM = 3   /* bf16, decode-sized M: streams Wc once (tensor cores for BN = 128) */
 };
 
+/* Activation of the fused epilogue (ss1_forward_ex, ss1_chain_forward). */
+enum ss1_activation {
+    SS1_ACT_NONE = 0,
+    SS1_ACT_RELU = 1,   /* max(v, 0)                                       */
+    SS1_ACT_GELU = 2    /* v * Phi(v) = 0.5 v (1 + erf(v / sqrt(2))), exact */
+};
+
+/* Layers that one ss1_chain_forward call takes at most. */
+#define SS1_CHAIN_MAX_LAYERS 4
+
 enum ss1_status {
     SS1_OK = 0,
     SS1_ERR_INVALID_ARG = -1,        /* a size, dtype, kernel or shape precondition failed   */
@@ -153,6 +163,45 @@ SS1_API int ss1_device_status(ss1_handle h, int32_t* detail);
 
 /* ss1_strerror -- static, NUL-terminated text for a status code. */
 SS1_API const char* ss1_strerror(int status);
+
+/*
+ * ss1_forward_ex -- Y = act(SS1(X) + bias): the layer with a per-neuron bias and an activation.
+ * "SS1: Accelerating Inference with Fast and Expressive Sketch Structured Transform", section
+ * "Measured effects": SS1 layers replace the layers of the DLRM MLPerf top MLP; an MLP adds a
+ * bias and an activation to each layer, which the pages leave to the model.
+ *   bias : device, [N] of `dtype`, or NULL (no bias).   act : enum ss1_activation.
+ *   kernel : enum ss1_kernel (AUTO picks as ss1_forward does). Other arguments as ss1_forward.
+ * The tensor-core kernel for c >= 2 (every large-M bf16 layer of the workloads) adds the bias
+ * and applies the activation to the fp32 sum in its epilogue, then rounds once; the other
+ * kernels write Y and one elementwise pass follows (a second rounding for bf16).
+ * Errors: as ss1_forward_with; INVALID_ARG for an unknown act; MISALIGNED for a bias not
+ * aligned to its element.
+ */
+SS1_API int ss1_forward_ex(ss1_handle h, const void* X, const void* Wc, const void* bias, int act, void* Y, int64_t M,
+                           int dtype, int kernel, void* stream);
+
+/*
+ * ss1_chain_forward -- a chain of bf16 SS1 layers, each the input of the next (an MLP):
+ *   Y[0] = act[0](SS1_0(X) + bias[0]),  Y[l] = act[l](SS1_l(Y[l - 1]) + bias[l]).
+ * Same source as ss1_forward_ex (the DLRM top MLP of "Measured effects").
+ *   layers : n_layers (1 .. SS1_CHAIN_MAX_LAYERS) handles; K of layer l + 1 == N of layer l.
+ *   X : device bf16 [M, K of layer 0].   Wc[l] : device bf16 [N_l, K_l / c_l].
+ *   bias : NULL, or an array of n_layers device pointers (bf16 [N_l], each may be NULL).
+ *   act : NULL (no activation), or n_layers enum ss1_activation values.
+ *   Y : n_layers device pointers, Y[l] bf16 [M, N_l], all written (the caller owns them; the
+ *       intermediate outputs are kept, as an MLP's backward pass needs them).
+ * When every layer runs on the tensor-core kernel for c >= 2 with one (BK, c) and the same
+ * N-block grouping (ss1_chain_fused says whether), the whole chain is one persistent launch:
+ * each CTA carries whole 128-row tiles through every layer in order, so no layer waits for
+ * another CTA. Otherwise the layers run one ss1_forward_ex after another. Asynchronous.
+ * Errors: BAD_HANDLE, INVALID_ARG (sizes, NULL, act), MISALIGNED (X, Wc, Y 16-byte, bias 2-byte),
+ * CUDA, DEVICE_TIMEOUT.
+ */
+SS1_API int ss1_chain_forward(const ss1_handle* layers, int n_layers, const void* X, const void* const* Wc,
+                              const void* const* bias, const int* act, void* const* Y, int64_t M, void* stream);
+
+/* ss1_chain_fused -- *fused = 1 if ss1_chain_forward runs these layers as one launch, else 0. */
+SS1_API int ss1_chain_fused(const ss1_handle* layers, int n_layers, int* fused);
 
 /*
  * ss1_project -- the SS1 weights closest to a dense weight: Wc = argmin || W_full(Wc) - W ||_F.
@@ -310,6 +359,23 @@ SS1_API int ss1_forward_noalloc(int64_t K, int64_t N, int c, int BK, int BN, uin
  * Asynchronous. Errors: BAD_HANDLE, INVALID_ARG (limit_ns out of range), CUDA (launch failure).
  */
 SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, void* stream);
+
+/*
+ * ss1_test_forward_timeout -- exercises a forward kernel's own time-out path without a fault, for
+ * tests of failure handling (the SS1 pages have no counterpart). Runs the tensor-core kernel for
+ * c >= 2 (the one ss1_forward picks for large bf16 batches) on X, Wc, Y as ss1_forward would
+ * (a test variant of it, built for layers with BK = 128, c = 2 and an even count of N-blocks),
+ * with every bounded wait cut to limit_ns nanoseconds (1 .. 2e9) and CTA 0's first sketch-matrix
+ * warp withholding its arrival for the third sketch segment, so CTA 0 stalls. The first of its
+ * waits to run out writes the status word ((1 << 8) | 0x80 | site: kernel id 1, the wait's site),
+ * the CTA's other warps give up their waits, every copy and matrix multiply in flight completes,
+ * the tensor memory is freed and the kernel returns; Y is not valid. Afterwards ss1_forward on this handle
+ * returns SS1_ERR_DEVICE_TIMEOUT until ss1_device_status has read and cleared the word.
+ * Asynchronous. Errors: BAD_HANDLE, INVALID_ARG (limit_ns out of range, M < 1, NULL pointer),
+ * MISALIGNED, UNSUPPORTED_SHAPE (not such a layer), CUDA.
+ */
+SS1_API int ss1_test_forward_timeout(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int64_t limit_ns,
+                                     void* stream);
 
 #ifdef __cplusplus
 }

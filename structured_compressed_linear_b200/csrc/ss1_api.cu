@@ -2,9 +2,12 @@
 // The operation and every entry point are specified in include/ss1.h.
 #include "ss1_internal.cuh"
 
+#include <cuda_bf16.h>
+
 #include <cuda.h>
 
 #include <functional>
+#include <map>
 #include <mutex>
 #include <new>
 #include <utility>
@@ -51,11 +54,35 @@ int kernel_for(const ss1_layer& L, int64_t M, int dtype) {
     return SS1_KERNEL_SIMT;
 }
 
+template <typename T>
+__global__ void bias_act_kernel(T* __restrict__ Y, const T* __restrict__ bias, int act, int64_t M, int64_t N) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= M * N) return;
+    float v = (float)Y[i];
+    if (bias) v += (float)bias[i % N];
+    if (act == SS1_ACT_RELU) v = fmaxf(v, 0.0f);
+    else if (act == SS1_ACT_GELU) v = 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));   // v * Phi(v)
+    Y[i] = (T)v;
+}
+
 }  // namespace
 
 namespace ss1 {
 
 bool handle_live(const ss1_layer* h) { return live(h); }
+
+cudaError_t launch_bias_act(void* Y, const void* bias, int act, int64_t M, int64_t N, int dtype, cudaStream_t st) {
+    const int64_t n = M * N;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    if (dtype == SS1_DTYPE_BF16)
+        bias_act_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(
+            (__nv_bfloat16*)Y, (const __nv_bfloat16*)bias, act, M, N);
+    else
+        bias_act_kernel<float><<<(unsigned)blocks, threads, 0, st>>>((float*)Y, (const float*)bias, act, M, N);
+    return cudaGetLastError();
+}
 
 uint64_t current_context_id() {
     using GetCurrent = CUresult (*)(CUcontext*);
@@ -97,6 +124,50 @@ cudaError_t smem_attr_once(const void* kernel, int bytes) {
 }
 
 int auto_kernel(const ss1_layer& L, int64_t M, int dtype) { return kernel_for(L, M, dtype); }
+
+ClusterFit cluster_fit(const void* fn, int smem, int threads) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, uint64_t>, ClusterFit> done;
+    const uint64_t ctx = current_context_id();
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = done.find({fn, ctx});
+    if (ctx != 0 && it != done.end()) return it->second;
+    ClusterFit f;
+    cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaGetLastError();
+    for (int cs = 1; cs <= 16; ++cs) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, (unsigned)cs);
+        cfg.blockDim = dim3((unsigned)threads);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 1;
+        at[0].val.clusterDim.y = (unsigned)cs;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess) f.active[cs] = n;
+        cudaGetLastError();
+    }
+    const uint64_t now = current_context_id();
+    if (now != 0) done[{fn, now}] = f;
+    return f;
+}
+
+int pick_splits(const ClusterFit& f, int groups, int want, int units) {
+    int hi = want < units ? want : units;
+    hi = hi > 16 ? 16 : hi;
+    if (hi <= 1) return 1;
+    int best = 1, best_ctas = 0;
+    for (int s = hi; s >= 1; --s) {
+        if (f.active[s] >= groups) return s;
+        const int resident = (f.active[s] < groups ? f.active[s] : groups) * s;
+        if (resident > best_ctas) { best_ctas = resident; best = s; }
+    }
+    return best;
+}
 
 bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN) {
     if (K < 1 || N < 1 || BK < 1 || BN < 1) return false;
@@ -274,6 +345,86 @@ SS1_API int ss1_forward_with(ss1_handle h, const void* X, const void* Wc, void* 
 
 SS1_API int ss1_forward(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int dtype, void* stream) {
     return ss1_forward_with(h, X, Wc, Y, M, dtype, SS1_KERNEL_AUTO, stream);
+}
+
+SS1_API int ss1_forward_ex(ss1_handle h, const void* X, const void* Wc, const void* bias, int act, void* Y, int64_t M,
+                           int dtype, int kernel, void* stream) {
+    if (!live(h)) return SS1_ERR_BAD_HANDLE;
+    if (act < SS1_ACT_NONE || act > SS1_ACT_GELU) return SS1_ERR_INVALID_ARG;
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & (dtype == SS1_DTYPE_BF16 ? 1u : 3u))) return SS1_ERR_MISALIGNED;
+    if (!bias && act == SS1_ACT_NONE) return ss1_forward_with(h, X, Wc, Y, M, dtype, kernel, stream);
+    if (M < 0 || (dtype != SS1_DTYPE_BF16 && dtype != SS1_DTYPE_FP32)) return SS1_ERR_INVALID_ARG;
+    if (kernel == SS1_KERNEL_AUTO) kernel = kernel_for(*h, M, dtype);
+    // the tensor-core kernel for c >= 2 applies bias and activation in its epilogue, before rounding
+    if (kernel == SS1_KERNEL_TC && dtype == SS1_DTYPE_BF16 && ss1::tc3_supported(*h) && M > 0) {
+        if (M > ((int64_t)1 << 31) / 2) return SS1_ERR_INVALID_ARG;
+        if (*(volatile int32_t*)h->status_host != 0) return SS1_ERR_DEVICE_TIMEOUT;
+        if (!X || !Wc || !Y) return SS1_ERR_INVALID_ARG;
+        if (!aligned16(X) || !aligned16(Wc) || !aligned16(Y)) return SS1_ERR_MISALIGNED;
+        int prev = -1;
+        if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        const cudaError_t e = ss1::launch_tc3(*h, X, Wc, Y, M, bias, act, (cudaStream_t)stream);
+        if (prev != h->device) cudaSetDevice(prev);
+        if (e != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        return SS1_OK;
+    }
+    // other kernels: the forward, then one elementwise pass over Y (a second rounding)
+    const int rc = ss1_forward_with(h, X, Wc, Y, M, dtype, kernel, stream);
+    if (rc != SS1_OK || M == 0) return rc;
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    const cudaError_t e = ss1::launch_bias_act(Y, bias, act, M, h->N, dtype, (cudaStream_t)stream);
+    if (prev != h->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    return SS1_OK;
+}
+
+SS1_API int ss1_chain_fused(const ss1_handle* layers, int n_layers, int* fused) {
+    if (!layers || !fused || n_layers < 1 || n_layers > SS1_CHAIN_MAX_LAYERS) return SS1_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l)
+        if (!live(layers[l])) return SS1_ERR_BAD_HANDLE;
+    *fused = ss1::tc3_chain_ok(reinterpret_cast<const ss1_layer* const*>(layers), n_layers) ? 1 : 0;
+    return SS1_OK;
+}
+
+SS1_API int ss1_chain_forward(const ss1_handle* layers, int n_layers, const void* X, const void* const* Wc,
+                              const void* const* bias, const int* act, void* const* Y, int64_t M, void* stream) {
+    if (!layers || !Wc || !Y || n_layers < 1 || n_layers > SS1_CHAIN_MAX_LAYERS) return SS1_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!live(layers[l])) return SS1_ERR_BAD_HANDLE;
+        if (l > 0 && layers[l]->K != layers[l - 1]->N) return SS1_ERR_INVALID_ARG;
+        if (act && (act[l] < SS1_ACT_NONE || act[l] > SS1_ACT_GELU)) return SS1_ERR_INVALID_ARG;
+        if (*(volatile int32_t*)layers[l]->status_host != 0) return SS1_ERR_DEVICE_TIMEOUT;
+    }
+    if (M < 0 || M > ((int64_t)1 << 31) / 2) return SS1_ERR_INVALID_ARG;
+    if (M == 0) return SS1_OK;
+    if (!X) return SS1_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!Wc[l] || !Y[l]) return SS1_ERR_INVALID_ARG;
+        if (!aligned16(Wc[l]) || !aligned16(Y[l]) || (bias && bias[l] && (reinterpret_cast<uintptr_t>(bias[l]) & 1u)))
+            return SS1_ERR_MISALIGNED;
+    }
+    if (!aligned16(X)) return SS1_ERR_MISALIGNED;
+    const ss1_layer* const* Ls = reinterpret_cast<const ss1_layer* const*>(layers);
+    if (ss1::tc3_chain_ok(Ls, n_layers)) {   // one persistent launch for the whole chain
+        int prev = -1;
+        const int dev = layers[0]->device;
+        if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        const cudaError_t e = ss1::launch_tc3_chain(Ls, n_layers, X, Wc, Y, bias, act, M, (cudaStream_t)stream);
+        if (prev != dev) cudaSetDevice(prev);
+        if (e != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+        return SS1_OK;
+    }
+    // otherwise layer by layer
+    for (int l = 0; l < n_layers; ++l) {
+        const int rc = ss1_forward_ex(layers[l], l == 0 ? X : Y[l - 1], Wc[l], bias ? bias[l] : nullptr,
+                                      act ? act[l] : SS1_ACT_NONE, Y[l], M, SS1_DTYPE_BF16, SS1_KERNEL_AUTO, stream);
+        if (rc != SS1_OK) return rc;
+    }
+    return SS1_OK;
 }
 
 }  // extern "C"

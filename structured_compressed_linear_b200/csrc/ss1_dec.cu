@@ -36,9 +36,7 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
-#include <map>
 #include <mutex>
-#include <utility>
 
 namespace ss1 {
 
@@ -496,60 +494,6 @@ bool make_map_x(CUtensorMap* map, const void* base, uint64_t K, uint64_t M, uint
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// How many clusters of `cs` CTAs (the K-splits of one N-block) the device keeps resident at once
-// for this kernel, for cs = 1 .. 16 (16 is a non-portable cluster size; 0 where a size does not
-// fit at all). Clusters are placed whole inside one GPC, so this is not simply the CTA slots
-// divided by cs. Looked up once per (kernel, context).
-struct ClusterFit {
-    int active[17] = {};
-};
-
-ClusterFit cluster_fit(const void* fn, int smem, int threads) {
-    static std::mutex mu;
-    static std::map<std::pair<const void*, uint64_t>, ClusterFit> done;
-    const uint64_t ctx = current_context_id();
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = done.find({fn, ctx});
-    if (ctx != 0 && it != done.end()) return it->second;
-    ClusterFit f;
-    cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaGetLastError();
-    for (int cs = 1; cs <= 16; ++cs) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(1, (unsigned)cs);
-        cfg.blockDim = dim3((unsigned)threads);
-        cfg.dynamicSmemBytes = (size_t)smem;
-        cudaLaunchAttribute a[1];
-        a[0].id = cudaLaunchAttributeClusterDimension;
-        a[0].val.clusterDim.x = 1;
-        a[0].val.clusterDim.y = (unsigned)cs;
-        a[0].val.clusterDim.z = 1;
-        cfg.attrs = a;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess) f.active[cs] = n;
-        cudaGetLastError();
-    }
-    const uint64_t now = current_context_id();
-    if (now != 0) done[{fn, now}] = f;
-    return f;
-}
-
-// K-splits per N-block: the largest count up to `want` (and `units`) whose NB clusters all fit
-// on the device at once; where none does, the one that keeps the most CTAs resident.
-int pick_splits(const ClusterFit& f, int NB, int want, int units) {
-    int hi = want < units ? want : units;
-    hi = hi > 16 ? 16 : hi;
-    if (hi <= 1) return 1;
-    int best = 1, best_ctas = 0;
-    for (int s = hi; s >= 1; --s) {
-        if (f.active[s] >= NB) return s;
-        const int resident = (f.active[s] < NB ? f.active[s] : NB) * s;
-        if (resident > best_ctas) { best_ctas = resident; best = s; }
-    }
-    return best;
 }
 
 template <int MP, int C, bool FP8>

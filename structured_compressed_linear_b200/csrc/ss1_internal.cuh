@@ -44,6 +44,22 @@ bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN);
 // Ids are never reused, so a context created after a device reset gets a new one.
 uint64_t current_context_id();
 
+// How many clusters of cs CTAs (cluster dimensions (1, cs, 1)) the device keeps resident at once
+// for a kernel, cs = 1 .. 16 (16 is a non-portable size; 0 where a size does not fit at all).
+// Clusters are placed whole inside one GPC, so this is not the CTA slots divided by cs. Looked
+// up once per (kernel, context).
+struct ClusterFit {
+    int active[17] = {};
+};
+ClusterFit cluster_fit(const void* fn, int smem, int threads);
+// K-splits per output group when each group's splits form one cluster: the largest count up to
+// `want` (and `units`, at most 16) whose `groups` clusters all fit on the device at once; where
+// none does, the one that keeps the most CTAs resident.
+int pick_splits(const ClusterFit& f, int groups, int want, int units);
+
+// Y[m, n] = act(Y[m, n] + bias[n]) in place (bias may be null), for kernels without the fused epilogue.
+cudaError_t launch_bias_act(void* Y, const void* bias, int act, int64_t M, int64_t N, int dtype, cudaStream_t st);
+
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` in the current context. The attribute
 // belongs to a context, so it is set once per (kernel, context); later calls return at once.
 cudaError_t smem_attr_once(const void* kernel, int bytes);
@@ -76,7 +92,18 @@ cudaError_t launch_tc2(const ss1_layer& L, const void* X, const void* Wc, void* 
 // Sketch-as-GEMM variant (c >= 2): the sketch of each chunk is a tcgen05.mma with an on-chip
 // 0/+-1 matrix; 128 rows x one or two N-blocks per tile.
 bool tc3_supported(const ss1_layer& L);
-cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
+// bias: bf16 [N] or null; act: 0 none, 1 ReLU, 2 GELU (applied to the fp32 sum before rounding).
+cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, const void* bias, int act,
+                       cudaStream_t st);
+// Test of the time-out path: the same launch with every wait limited to wait_ns, and CTA 0's
+// first build warp withholding its arrival for the third sketch segment, so a wait runs out.
+cudaError_t launch_tc3_withhold(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M,
+                                uint64_t wait_ns, cudaStream_t st);
+// A chain of up to four layers in one persistent launch (layer l + 1 reads layer l's Y): every
+// layer tc3-supported with the first layer's BK, c and N-block grouping, K of l + 1 == N of l.
+bool tc3_chain_ok(const ss1_layer* const* Ls, int n);
+cudaError_t launch_tc3_chain(const ss1_layer* const* Ls, int n, const void* X, const void* const* Wc, void* const* Y,
+                             const void* const* bias, const int* act, int64_t M, cudaStream_t st);
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st);
 
 // Dense -> SS1 projection (bf16 or fp32): Wc[n, j] = scale * sum_{k : h(k) = j} g(k) W[n, k]

@@ -42,3 +42,20 @@ extern "C" SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, v
     if (prev != h->device) cudaSetDevice(prev);
     return e == cudaSuccess ? SS1_OK : SS1_ERR_CUDA;
 }
+
+extern "C" SS1_API int ss1_test_forward_timeout(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M,
+                                                int64_t limit_ns, void* stream) {
+    if (!ss1::handle_live(h)) return SS1_ERR_BAD_HANDLE;
+    if (limit_ns < 1 || limit_ns > 2000000000 || M < 1 || M > ((int64_t)1 << 31) / 2) return SS1_ERR_INVALID_ARG;
+    if (!X || !Wc || !Y) return SS1_ERR_INVALID_ARG;
+    if (((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Wc) | reinterpret_cast<uintptr_t>(Y)) & 15u) != 0)
+        return SS1_ERR_MISALIGNED;
+    if (!ss1::tc3_supported(*h) || h->BK != 128 || h->c != 2 || h->NB % 2 != 0) return SS1_ERR_UNSUPPORTED_SHAPE;
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    const cudaError_t e = ss1::launch_tc3_withhold(*h, X, Wc, Y, M, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream));
+    if (prev != h->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) { cudaGetLastError(); return SS1_ERR_CUDA; }
+    return SS1_OK;
+}

@@ -5,14 +5,19 @@
 // compression factor c) and then multiplied with the compressed weights.
 //
 // This kernel runs every valid shape in bf16 or fp32 and is the fp32 path of the library.
-// A CTA owns TM rows x TN columns that lie inside one N-block nb. Per K-chunk kc and per
-// group of up to 32 slots it
+// A CTA owns TM rows x TN columns that lie inside one N-block nb, and a range of K-chunks. Per
+// K-chunk kc and per group of up to 32 slots it
 //   1. sketches   Xs[m][s] = sum_j sign_j * X[m, kc*BK + k_j]   (fp32, in shared memory)
 //   2. stages     Wt[s][n] = Wc[n, kc*S + s]                     (fp32, transposed)
 //   3. multiplies acc[m][n] += Xs[m][s] * Wt[s][n]                (fp32 FMA, 16x16 threads)
 // and finally rounds once to the output type. Sketch sums and the GEMM are both fp32, so
 // for fp32 data the only roundings are those of fp32 arithmetic.
+// Small batches give few output tiles, so the K-chunks are split over the CTAs of a thread-block
+// cluster: each leaves its fp32 partial tile in shared memory, and after a cluster barrier CTA r
+// sums rows r, r + splits, ... of all the partials in split order (the same bits every call)
+// through distributed shared memory and writes Y.
 #include "ss1_internal.cuh"
+#include "ptx_sm100.cuh"
 
 #include <cuda_bf16.h>
 
@@ -30,15 +35,20 @@ __device__ __forceinline__ void from_f32(__nv_bfloat16& d, float v) { d = __floa
 template <typename T, int TM, int TN>
 __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X, const T* __restrict__ Wc,
                                                         T* __restrict__ Y, const uint16_t* __restrict__ src,
-                                                        int M, int K, int N, int c, int BK, int BN, int S) {
+                                                        int M, int K, int N, int c, int BK, int BN, int S, int ntiles_n) {
     constexpr int RM = TM / 16, RN = TN / 16;
-    __shared__ float Xs[TM][kSlotGroup + 1];
-    __shared__ float Wt[kSlotGroup][TN];
+    constexpr int XS_WORDS = TM * (kSlotGroup + 1), WT_WORDS = kSlotGroup * TN;
+    static_assert(XS_WORDS + WT_WORDS >= TM * TN, "the partial tile fits in the staging buffers");
+    __shared__ float stage_buf[XS_WORDS + WT_WORDS];
+    float (*Xs)[kSlotGroup + 1] = reinterpret_cast<float (*)[kSlotGroup + 1]>(stage_buf);
+    float (*Wt)[TN] = reinterpret_cast<float (*)[TN]>(stage_buf + XS_WORDS);
 
-    const int n0 = blockIdx.x * TN;
+    const int n0 = (int)(blockIdx.x % (unsigned)ntiles_n) * TN;
     const int nb = n0 / BN;
-    const int m0 = blockIdx.y * TM;
+    const int m0 = (int)(blockIdx.x / (unsigned)ntiles_n) * TM;
     const int KC = K / BK;
+    const int splits = (int)gridDim.y, split = (int)blockIdx.y;
+    const int kc_lo = (int)((int64_t)KC * split / splits), kc_hi = (int)((int64_t)KC * (split + 1) / splits);
     const int Kc = K / c;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
 
@@ -48,7 +58,7 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
 #pragma unroll
         for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
 
-    for (int kc = 0; kc < KC; ++kc) {
+    for (int kc = kc_lo; kc < kc_hi; ++kc) {
         const uint16_t* sblk = src + ((size_t)nb * KC + kc) * (size_t)S * c;
         for (int s0 = 0; s0 < S; s0 += kSlotGroup) {
             const int sc = min(kSlotGroup, S - s0);
@@ -85,21 +95,58 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
             __syncthreads();
         }
     }
+    if (splits == 1) {
 #pragma unroll
-    for (int i = 0; i < RM; ++i) {
-        const int m = m0 + ty + 16 * i;
-        if (m >= M) continue;
+        for (int i = 0; i < RM; ++i) {
+            const int m = m0 + ty + 16 * i;
+            if (m >= M) continue;
 #pragma unroll
-        for (int j = 0; j < RN; ++j) from_f32(Y[(size_t)m * N + n0 + tx + 16 * j], acc[i][j]);
+            for (int j = 0; j < RN; ++j) from_f32(Y[(size_t)m * N + n0 + tx + 16 * j], acc[i][j]);
+        }
+        return;
     }
+    // the split's partial tile [TM][TN] in the staging buffers (the K loop ended on a barrier)
+#pragma unroll
+    for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RN; ++j) stage_buf[(ty + 16 * i) * TN + tx + 16 * j] = acc[i][j];
+    ptx::cluster_sync();   // every split's partial is visible to the cluster (rank = split)
+    const int rows = M - m0 < TM ? M - m0 : TM;
+    for (int e = (int)ptx::cluster_ctarank() * TN + (int)threadIdx.x; e < rows * TN; e += splits * TN) {
+        // element e = (row, column) of the tile; CTA r takes rows r, r + splits, ...
+        if ((int)threadIdx.x >= TN) break;
+        float v = 0.f;
+        for (int sp = 0; sp < splits; ++sp) v += ptx::ld_cluster_f32(ptx::map_to_rank(stage_buf + e, (uint32_t)sp));
+        from_f32(Y[(size_t)(m0 + e / TN) * N + n0 + e % TN], v);
+    }
+    ptx::cluster_sync();   // the peers have read this CTA's partial
 }
 
 template <typename T, int TM, int TN>
 cudaError_t launch_t(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    dim3 grid((unsigned)(L.N / TN), (unsigned)((M + TM - 1) / TM));
-    simt_kernel<T, TM, TN><<<grid, kThreads, 0, st>>>((const T*)X, (const T*)Wc, (T*)Y, L.d_src, (int)M, (int)L.K,
-                                                      (int)L.N, L.c, L.BK, L.BN, L.S);
-    return cudaGetLastError();
+    const int64_t ntn = L.N / TN, tiles = ntn * ((M + TM - 1) / TM);
+    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    // K-splits (one cluster per output tile) where the tiles alone leave most SMs idle
+    int splits = 1;
+    const void* fn = reinterpret_cast<const void*>(&simt_kernel<T, TM, TN>);
+    if (tiles < 2 * (int64_t)L.num_sms && L.KC > 1)
+        splits = pick_splits(cluster_fit(fn, 0, kThreads), (int)tiles, (int)((2 * (int64_t)L.num_sms) / tiles), L.KC);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)splits;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = splits > 1 ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, simt_kernel<T, TM, TN>, (const T*)X, (const T*)Wc, (T*)Y,
+                                             (const uint16_t*)L.d_src, (int)M, (int)L.K, (int)L.N, L.c, L.BK, L.BN,
+                                             L.S, (int)ntn);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <typename T>

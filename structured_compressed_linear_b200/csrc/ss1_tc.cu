@@ -287,7 +287,7 @@ bool tc_supported(const ss1_layer& L) {
 }
 
 cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
-    if (tc3_supported(L)) return launch_tc3(L, X, Wc, Y, M, st);
+    if (tc3_supported(L)) return launch_tc3(L, X, Wc, Y, M, nullptr, 0, st);
     if (tc2_supported(L)) return launch_tc2(L, X, Wc, Y, M, st);
     // c >= 2 shapes that tc_supported accepts are all taken above (tc2_supported covers them)
     if (L.c != 1 || (M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;

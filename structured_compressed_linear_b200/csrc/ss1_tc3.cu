@@ -46,6 +46,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 namespace ss1 {
@@ -111,7 +112,7 @@ struct Cfg {
     static constexpr int OFF_TAB = OFF_E + EPI;
     static constexpr int OFF_CLR = OFF_TAB;
     static constexpr int OFF_BAR = OFF_CLR + CLR;
-    static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 2 + 2 + NACC + NACC * Q + 2;
+    static constexpr int NBAR = NX + 4 + 2 + 2 * NW + 2 + 2 + 2 + NACC + NACC * Q + 2 + 2;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     static_assert(BK % kUnitK == 0 && BK <= 256 && U % SU == 0, "chunks of whole 64-input units");
     static_assert(S % 16 == 0 && S >= 16 && S <= 128, "UMMA K-steps of 16 over the slots");
@@ -120,30 +121,134 @@ struct Cfg {
     static_assert(NX >= 2 * SU && SMEM <= 227 * 1024, "shared memory budget: X ring holds two segments");
     static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0, "swizzle atoms stay aligned");
     static_assert(NBW <= kMaxBuildWarps, "build warps");
+    // the X loader's first wait for segment g comes before the boxes of segment g + 4 are all
+    // issued, so that segment (the same barrier, one phase later) cannot have completed yet
+    static_assert(NX < 5 * SU, "X ring depth against the four segment barriers");
 };
 
+constexpr int kMaxLayers = 4;
+enum { kActNone = 0, kActRelu = 1, kActGelu = 2 };
+
+// One layer of a launch: its tensor maps (X [M x K], Wc [N x K/c], Y [M x N]), its slot table,
+// and the epilogue's bias (bf16 [N], or null) and activation.
+struct Tc3Layer {
+    CUtensorMap tx, tw, ty;
+    const uint16_t* slot_tab;
+    const __nv_bfloat16* bias;
+    int K, KC, NG, act;
+};
+
+// A launch runs one layer, its (M-tile, N-block group) tiles dealt round-robin to the CTAs, or
+// (chain) up to kMaxLayers layers, each the input of the next: a CTA then takes pairs of M-tiles
+// and carries both through every layer, alternating between them (layer l of tile A, layer l of
+// tile B, layer l + 1 of A, ...), so no other CTA's output is ever waited for and the wait of one
+// tile for its previous layer's stores is covered by the other tile's work.
+struct Tc3Params {
+    Tc3Layer layer[kMaxLayers];
+    int n_layers;
+    int chain;
+    int num_units;   // tiles (one layer) or pairs of M-tiles (chain)
+    int M;           // rows (a chain's pair may end in a tile wholly past M: its stores are skipped)
+    int32_t* status;
+    uint64_t wait_ns;       // limit of every wait (2 s; a test of the time-out path cuts it)
+    int withhold_segment;   // test of the time-out path: CTA 0's first build warp skips this
+                            // segment's arrival, so the sketch warp's wait runs out (-1: never)
+};
+
+struct TileInfo {
+    int l, m0, nb0, ng, KC, h;   // h: which M-tile of the chain's pair (0 or 1)
+};
+
+// Tiles of one chain unit (a pair of M-tiles through all N-block groups of all layers) and their chunks.
+__device__ __forceinline__ void chain_sizes(const Tc3Params& p, int& tiles, int& chunks) {
+    tiles = 0;
+    chunks = 0;
+    for (int l = 0; l < p.n_layers; ++l) {
+        tiles += 2 * p.layer[l].NG;
+        chunks += 2 * p.layer[l].NG * p.layer[l].KC;
+    }
+}
+
+// The j-th tile this CTA computes.
+template <int Q, bool CHAIN>
+__device__ __forceinline__ TileInfo tile_info(const Tc3Params& p, int j) {
+    TileInfo t;
+    if (!CHAIN) {
+        const int tile = (int)blockIdx.x + j * (int)gridDim.x, NG = p.layer[0].NG;
+        t.l = 0;
+        t.h = 0;
+        t.ng = tile % NG;
+        t.m0 = (tile / NG) * kRows;
+        t.KC = p.layer[0].KC;
+    } else {
+        int T, C;
+        chain_sizes(p, T, C);
+        int r = j % T, l = 0;
+        while (l + 1 < p.n_layers && r >= 2 * p.layer[l].NG) r -= 2 * p.layer[l++].NG;
+        t.l = l;
+        t.h = r / p.layer[l].NG;
+        t.ng = r % p.layer[l].NG;
+        t.m0 = (2 * ((int)blockIdx.x + (j / T) * (int)gridDim.x) + t.h) * kRows;
+        t.KC = p.layer[l].KC;
+    }
+    t.nb0 = t.ng * Q;
+    return t;
+}
+
+// The i-th chunk this CTA processes: its tile and its K-chunk kc.
+template <int Q, bool CHAIN>
+__device__ __forceinline__ TileInfo chunk_info(const Tc3Params& p, int i, int& kc) {
+    if (!CHAIN) {
+        const int KC = p.layer[0].KC;
+        kc = i % KC;
+        return tile_info<Q, CHAIN>(p, i / KC);
+    }
+    int T, C;
+    chain_sizes(p, T, C);
+    int r = i % C, l = 0, j = (i / C) * T;
+    while (l + 1 < p.n_layers && r >= 2 * p.layer[l].NG * p.layer[l].KC) {
+        r -= 2 * p.layer[l].NG * p.layer[l].KC;
+        j += 2 * p.layer[l++].NG;
+    }
+    kc = r % p.layer[l].KC;
+    return tile_info<Q, CHAIN>(p, j + r / p.layer[l].KC);
+}
+
+__device__ __forceinline__ float activate(float v, int act) {
+    if (act == kActRelu) return fmaxf(v, 0.0f);
+    if (act == kActGelu) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));   // v * Phi(v)
+    return v;
+}
+
+// The first wait of the CTA to run out writes its site; the warps it stalls then see the abort
+// flag, give up their own waits and leave the word as it is. (Two waits that run out in the same
+// instant may both write; either site is a true one.)
 __device__ __forceinline__ void report(int32_t* status, volatile int* abort_flag, int site) {
-    *abort_flag = 1;
-    *(volatile int32_t*)status = (kStatusKernelTC << 8) | (0x80 + site);
-    __threadfence_system();
+    if (*abort_flag == 0) {
+        *abort_flag = 1;
+        *(volatile int32_t*)status = (kStatusKernelTC << 8) | (0x80 + site);
+        __threadfence_system();
+    }
 }
 
 // Lane 0 waits, the warp follows: one poller per warp instead of 32.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
+                                          uint64_t limit_ns) {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, kWaitNs);
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, abort_flag, limit_ns);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Wait of an MMA-issuing warp: every lane polls the barrier without suspending (one shared-memory
 // broadcast per poll), so the issue resumes as soon as the phase completes.
-__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
+                                               uint64_t limit_ns) {
     bool ok = ptx::mbar_test(bar, parity);
     if (!ok) {
         const uint64_t t0 = ptx::globaltimer_ns();
         for (uint32_t n = 1;; ++n) {
             if (ptx::mbar_test(bar, parity)) { ok = true; break; }
-            if ((n & 63) == 0 && (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitNs)) break;
+            if ((n & 63) == 0 && (*abort_flag || ptx::globaltimer_ns() - t0 > limit_ns)) break;
         }
     }
     return __all_sync(0xffffffffu, ok);
@@ -178,12 +283,13 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int kl) {
     return (uint32_t)(row * 128) + ((uint32_t)((kl >> 3) ^ (row & 7)) << 4) + (uint32_t)(kl & 7) * 2u;
 }
 
-template <int BK, int C, int Q>
-__global__ void __launch_bounds__(kThreads, 1)
-    tc3_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-               const __grid_constant__ CUtensorMap tmap_y, const uint16_t* __restrict__ slot_tab, int K, int KC, int NG,
-               int num_tiles, int32_t* status) {
+// TEST: the variant for the test of the time-out path (runtime wait limit, one withheld arrival);
+// the hot variants keep both out of their loops.
+template <int BK, int C, int Q, bool CHAIN, bool FX, bool TEST>
+__global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant__ Tc3Params p) {
     using F = Cfg<BK, C, Q>;
+    int32_t* status = p.status;
+    const uint64_t wait_ns = TEST ? p.wait_ns : kWaitNs;
     constexpr int S = F::S, QS = F::QS, HW = F::HW, U = F::U, SU = F::SU, NSEG = F::NSEG;
     constexpr int NX = F::NX, NP = F::NP, NW = F::NW, NACC = F::NACC;
     extern __shared__ uint8_t smem_raw[];
@@ -208,12 +314,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* acc_full = xs_free + 2;     // [NACC]
     uint64_t* acc_empty = acc_full + NACC;   // [NACC][Q] the epilogue has read N-block j's columns
     uint64_t* drain = acc_empty + NACC * Q;  // [2] abort path: completion of every MMA a warp issued
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+    uint64_t* layer_done = drain + 2;        // [2] chain: M-tile h of the pair has its layer stored
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(layer_done + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int G = my_tiles * KC;   // chunks this CTA processes
+    const int my_units = (p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    int my_tiles, G;   // tiles and chunks this CTA processes
+    if (CHAIN) {
+        int T, Cm;
+        chain_sizes(p, T, Cm);
+        my_tiles = my_units * T;
+        G = my_units * Cm;
+    } else {
+        my_tiles = my_units;
+        G = my_units * p.layer[0].KC;
+    }
 
     // the sketch panels start zeroed; only their non-zeros are ever written afterwards
     for (int i = threadIdx.x; i < NP * F::P_UNIT / 16; i += kThreads)
@@ -232,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < NACC; ++i) ptx::mbar_init(&acc_full[i], 1);
         for (int i = 0; i < NACC * Q; ++i) ptx::mbar_init(&acc_empty[i], kEpiWarps);
+        ptx::mbar_init(&layer_done[0], kEpiWarps);
+        ptx::mbar_init(&layer_done[1], kEpiWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -239,9 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
-    if (warp == kWarpLoadX && lane == 0) ptx::prefetch_tmap(&tmap_x);
-    if (warp == kWarpLoadW && lane == 0) ptx::prefetch_tmap(&tmap_w);
-    if (warp == kFirstEpi && lane == 0) ptx::prefetch_tmap(&tmap_y);
+    if (lane == 0 && (warp == kWarpLoadX || warp == kWarpLoadW || warp == kFirstEpi)) {
+        for (int l = 0; l < p.n_layers; ++l)
+            ptx::prefetch_tmap(warp == kWarpLoadX ? &p.layer[l].tx : warp == kWarpLoadW ? &p.layer[l].tw : &p.layer[l].ty);
+    }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -250,19 +369,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpLoadX) {
         // ------------------------------------------------------------------ TMA loads of X
         if (lane == 0) {
+            // A slot is free once the segment that read its previous box has completed. Segments
+            // complete in order, so each is waited for once (seen = the latest observed): waiting
+            // again on an old segment could read the barrier a full phase later and block (after
+            // the long stall at a layer boundary, say, when every earlier segment is done).
             Ring xr(NX);
-            int nx = 0;
+            int nx = 0, seen = -1;
+            int layer_waits[2] = {0, 0};
             bool ok = true;
             for (int t = 0; t < my_tiles && ok; ++t) {
-                const int m0 = (((int)blockIdx.x + t * (int)gridDim.x) / NG) * kRows;
-                for (int kc = 0; kc < KC && ok; ++kc)
+                const TileInfo ti = tile_info<Q, CHAIN>(p, t);
+                if (CHAIN && ti.l > 0 && ti.ng == 0) {
+                    // the M-tile's previous layer (this layer's X) has been stored by the epilogue
+                    if (!ptx::mbar_wait(&layer_done[ti.h], (uint32_t)(layer_waits[ti.h] & 1), abort_flag, wait_ns)) {
+                        report(status, abort_flag, 12);
+                        break;
+                    }
+                    ++layer_waits[ti.h];
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
+                const CUtensorMap* tx = &p.layer[ti.l].tx;
+                for (int kc = 0; kc < ti.KC && ok; ++kc)
                     for (int u = 0; u < U; ++u) {
                         if (nx >= NX) {   // the slot's previous unit belongs to segment gp
                             const int gp = (nx - NX) / SU;
-                            if (!ptx::mbar_wait(&seg_done[gp & 3], (uint32_t)((gp >> 2) & 1), abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 1); break; }
+                            if (gp > seen) {
+                                if (!ptx::mbar_wait(&seg_done[gp & 3], (uint32_t)((gp >> 2) & 1), abort_flag, wait_ns)) { ok = false; report(status, abort_flag, 1); break; }
+                                seen = gp;
+                            }
                         }
                         ptx::mbar_arrive_expect_tx(&x_full[xr.slot], kXUnit);
-                        ptx::tma_load_2d(xring + xr.slot * kXUnit, &tmap_x, &x_full[xr.slot], kc * BK + u * kUnitK, m0);
+                        ptx::tma_load_2d(xring + xr.slot * kXUnit, tx, &x_full[xr.slot], kc * BK + u * kUnitK, ti.m0);
                         xr.next();
                         ++nx;
                     }
@@ -276,16 +413,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             int nw = 0;
             bool ok = true;
             for (int t = 0; t < my_tiles && ok; ++t) {
-                const int nb0 = (((int)blockIdx.x + t * (int)gridDim.x) % NG) * Q;
-                for (int kc = 0; kc < KC && ok; ++kc) {
-                    if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, kWaitNs)) { ok = false; report(status, abort_flag, 2); break; }
+                const TileInfo ti = tile_info<Q, CHAIN>(p, t);
+                const int nb0 = ti.nb0;
+                const CUtensorMap* tw = &p.layer[ti.l].tw;
+                for (int kc = 0; kc < ti.KC && ok; ++kc) {
+                    if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, wait_ns)) { ok = false; report(status, abort_flag, 2); break; }
                     ptx::mbar_arrive_expect_tx(&w_full[wr.slot], F::W_STAGE);
                     uint8_t* wdst = wring + wr.slot * F::W_STAGE;
 #pragma unroll
                     for (int j = 0; j < Q; ++j)
 #pragma unroll
-                        for (int p = 0; p < (S + 63) / 64; ++p)
-                            ptx::tma_load_2d(wdst + j * F::W_NB + p * F::W_PANEL, &tmap_w, &w_full[wr.slot], kc * S + p * 64,
+                        for (int pn = 0; pn < (S + 63) / 64; ++pn)
+                            ptx::tma_load_2d(wdst + j * F::W_NB + pn * F::W_PANEL, tw, &w_full[wr.slot], kc * S + pn * 64,
                                              (nb0 + j) * kNeu);
                     wr.next();
                     ++nw;
@@ -308,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < G && ok; ++i) {
             const uint32_t ds = tm + (uint32_t)(F::DS_COL + (i & 1) * QS);
             for (int sg = 0; sg < NSEG; ++sg, ++seg) {
-                if (!warp_wait_spin(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag) ||
-                    (sg == 0 && i >= 2 && !warp_wait_spin(&ds_free[i & 1], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag))) {
+                if (!warp_wait_spin(&sk_ready[seg & 1], (uint32_t)((seg >> 1) & 1), abort_flag, wait_ns) ||
+                    (sg == 0 && i >= 2 && !warp_wait_spin(&ds_free[i & 1], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag, wait_ns))) {
                     ok = false;
                     if (leader) report(status, abort_flag, 3);
                     break;
@@ -350,9 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool leader = lane == 0;
         Ring wr(NW);
         int t = 0, kc = 0;
+        int KC = my_tiles > 0 ? tile_info<Q, CHAIN>(p, 0).KC : 1;
         for (int i = 0; i < G; ++i) {
             const int b = i & 1, a = NACC == 2 ? (t & 1) : 0;
-            if (!warp_wait_spin(&mm_ready[b], (uint32_t)((i >> 1) & 1), abort_flag)) {
+            if (!warp_wait_spin(&mm_ready[b], (uint32_t)((i >> 1) & 1), abort_flag, wait_ns)) {
                 if (leader) report(status, abort_flag, 4);
                 break;
             }
@@ -367,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < Q; ++j) {
                     // a tile's first chunk: N-block j's accumulator columns have been read out
                     if (kc == 0) {
-                        if (!ptx::mbar_wait(&acc_empty[a * Q + j], acc_par, abort_flag, kWaitNs)) {
+                        if (!ptx::mbar_wait(&acc_empty[a * Q + j], acc_par, abort_flag, wait_ns)) {
                             report(status, abort_flag, 11);
                             stalled = true;
                             break;
@@ -393,7 +533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (__shfl_sync(0xffffffffu, stalled ? 1 : 0, 0)) break;
             wr.next();
-            if (++kc == KC) { kc = 0; ++t; }
+            if (++kc == KC) {
+                kc = 0;
+                if (++t < my_tiles) KC = tile_info<Q, CHAIN>(p, t).KC;
+            }
         }
         if (*abort_flag && leader) {
             volatile int no_abort = 0;
@@ -419,8 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto fetch = [&](int g, uint32_t (&e)[2]) {   // table entries of (segment g, su, j)
             if (g < nseg) {
                 const int pu = g * SU + su, i = pu / U, u = pu % U;
-                const int tile = (int)blockIdx.x + (i / KC) * (int)gridDim.x, kc = i % KC;
-                const uint16_t* src = slot_tab + (size_t)((tile % NG) * Q + j) * K + (size_t)kc * BK + u * kUnitK;
+                int kc;
+                const TileInfo ti = chunk_info<Q, CHAIN>(p, i, kc);
+                const Tc3Layer& ly = p.layer[ti.l];
+                const uint16_t* src = ly.slot_tab + (size_t)(ti.nb0 + j) * ly.K + (size_t)kc * BK + u * kUnitK;
                 e[0] = __ldg(src + lane);
                 e[1] = __ldg(src + lane + 32);
             }
@@ -435,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fetch(g + 2, ent);
             uint8_t* panel = pring + ((g & 1) * SU + su) * F::P_UNIT;
             if (g >= 2) {   // the pair's previous segment (g - 2) has been multiplied
-                if (!warp_wait_spin(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag)) {
+                if (!warp_wait_spin(&seg_done[(g - 2) & 3], (uint32_t)(((g - 2) >> 2) & 1), abort_flag, wait_ns)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 5);
                     return;
@@ -451,13 +596,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (j == 0) {   // unit su of the segment: its X box has landed
                 const int xu = g * SU + su;
-                if (!warp_wait_spin(&x_full[xu % NX], (uint32_t)((xu / NX) & 1), abort_flag)) {
+                if (!warp_wait_spin(&x_full[xu % NX], (uint32_t)((xu / NX) & 1), abort_flag, wait_ns)) {
                     ok = false;
                     if (lane == 0) report(status, abort_flag, 8);
                     return;
                 }
             }
-            if (lane == 0) ptx::mbar_arrive(&sk_ready[g & 1]);
+            if (lane == 0 && !(TEST && g == p.withhold_segment && blockIdx.x == 0 && bw == 0)) ptx::mbar_arrive(&sk_ready[g & 1]);
         };
         for (int g = 0; g < nseg && ok; g += 2) {
             segment(g, held0, ent0);
@@ -473,11 +618,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3, half = (warp - kFirstConv) >> 2;
         const uint32_t lanes = (uint32_t)(quad * 32) << 16;
         Ring wr(NW);
-        int t = 0, kc = 0;
         for (int i = 0; i < G; ++i) {
             const int b = i & 1;
             const int gl = i * NSEG + NSEG - 1;   // the chunk's last sketch segment
-            if (!warp_wait_spin(&seg_done[gl & 3], (uint32_t)((gl >> 2) & 1), abort_flag)) {
+            if (!warp_wait_spin(&seg_done[gl & 3], (uint32_t)((gl >> 2) & 1), abort_flag, wait_ns)) {
                 if (lane == 0) report(status, abort_flag, 6);
                 break;
             }
@@ -497,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int p = 0; p < HW / 2; ++p) r[p] = pack_bf16x2(r[2 * p], r[2 * p + 1]);
             uint32_t dst = src;
             if (F::SEP) {
-                if (i >= 2 && !warp_wait_spin(&xs_free[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag)) {
+                if (i >= 2 && !warp_wait_spin(&xs_free[b], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag, wait_ns)) {
                     if (lane == 0) report(status, abort_flag, 10);
                     break;
                 }
@@ -509,14 +653,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             // the first convert warp also waits for the chunk's Wc
-            if (warp == kFirstConv && !warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag)) {
+            if (warp == kFirstConv && !warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag, wait_ns)) {
                 if (lane == 0) report(status, abort_flag, 9);
                 break;
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&mm_ready[b]);
             wr.next();
-            if (++kc == KC) { kc = 0; ++t; }
         }
     } else if (warp >= kFirstEpi && warp < kFirstEpi + kEpiWarps) {
         // ------------------------------------------------------------------ epilogue
@@ -528,17 +671,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tm + ((uint32_t)(quad * 32) << 16);
         int nst = 0;
         for (int t = 0; t < my_tiles; ++t) {
-            const int tile = (int)blockIdx.x + t * (int)gridDim.x;
+            const TileInfo ti = tile_info<Q, CHAIN>(p, t);
+            const Tc3Layer& ly = p.layer[ti.l];
+            const CUtensorMap* ty = &ly.ty;
+            const __nv_bfloat16* bias = ly.bias;
+            const int act = ly.act;
             const int a = NACC == 2 ? (t & 1) : 0;
-            if (!warp_wait(&acc_full[a], (uint32_t)((t / NACC) & 1), abort_flag)) {
+            if (!warp_wait(&acc_full[a], (uint32_t)((t / NACC) & 1), abort_flag, wait_ns)) {
                 if (lane == 0) report(status, abort_flag, 7);
                 break;
             }
             ptx::tc_fence_after();
-            const int row0 = (tile / NG) * kRows + quad * 32;
-            const int col0 = (tile % NG) * Q * kNeu;
-            auto store_block = [&](int q, const uint32_t (&r)[32]) {
+            const int row0 = ti.m0 + quad * 32;
+            const int col0 = ti.nb0 * kNeu;
+            auto store_block = [&](int q, uint32_t (&r)[32]) {
                 uint8_t* box = stg + (nst & 1) * kEpiBox;
+                if constexpr (FX) {   // bias of column col0 + 32 q + j (lane j loads it), then the activation
+                    const float bl = bias ? __bfloat162float(bias[col0 + q * 32 + lane]) : 0.0f;
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        r[jj] = __float_as_uint(activate(__uint_as_float(r[jj]) + __shfl_sync(0xffffffffu, bl, jj), act));
+                }
                 if (lane == 0) ptx::tma_store_wait_read1();   // the store two blocks ago has read `box`
                 __syncwarp();
 #pragma unroll
@@ -549,14 +702,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    ptx::tma_store_2d(&tmap_y, box, col0 + q * 32, row0);
+                    if (row0 < p.M) ptx::tma_store_2d(ty, box, col0 + q * 32, row0);
                     ptx::tma_store_commit();
                 }
                 ++nst;
             };
+            const uint32_t abase = lane_base + (uint32_t)(a * F::ACC_COLS);
+            if constexpr (FX) {
+                // with bias and activation: each block loaded, waited for, then processed, so that
+                // no register an asynchronous TMEM load still writes is touched meanwhile
+#pragma unroll 1
+                for (int q = 0; q < 4 * Q; ++q) {
+                    uint32_t r[32];
+                    ptx::tmem_ld_32x32b_x32(abase + (uint32_t)(q * 32), r);
+                    ptx::tmem_ld_wait();
+                    ptx::tmem_ld_fence_regs<32>(r);
+                    if ((q + 1) % 4 == 0) {   // N-block q / 4 read: the next tile's MMAs into it may start
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&acc_empty[a * Q + q / 4]);
+                    }
+                    store_block(q, r);
+                }
+            } else {
             // two register buffers: the next block's TMEM load is in flight while this block is
             // staged and stored; N-block j is released right after its last block (4j+3) has landed
-            const uint32_t abase = lane_base + (uint32_t)(a * F::ACC_COLS);
             uint32_t ra[32], rb[32];
             ptx::tmem_ld_32x32b_x32(abase, ra);
             ptx::tmem_ld_wait();
@@ -578,6 +748,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_ld_wait();
                     ptx::tmem_ld_fence_regs<32>(ra);
                 }
+            }
+            }
+            if (CHAIN && ti.l + 1 < p.n_layers && ti.ng == ly.NG - 1) {
+                // this warp's rows of the M-tile's layer are stored; once all four warps say so
+                // the next layer may load them (the stores complete before the arrival)
+                if (lane == 0) {
+                    ptx::tma_store_wait0();
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    __threadfence();
+                    ptx::mbar_arrive(&layer_done[ti.h]);
+                }
+                __syncwarp();
             }
         }
         if (lane == 0) ptx::tma_store_wait0();
@@ -605,23 +787,76 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One layer of a launch, as the host describes it.
+struct Tc3Job {
+    const ss1_layer* L;
+    const void* X;
+    const void* Wc;
+    void* Y;
+    const void* bias;
+    int act;
+};
+
 template <int BK, int C, int Q>
-cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+cudaError_t launch_cfg(const Tc3Job* jobs, int n, bool chain, int64_t M, uint64_t wait_ns, int withhold,
+                       cudaStream_t st) {
     using F = Cfg<BK, C, Q>;
     constexpr int S = F::S;
-    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tc3_kernel<BK, C, Q>), F::SMEM);
+    bool fx = chain;
+    for (int l = 0; l < n; ++l) fx = fx || jobs[l].bias != nullptr || jobs[l].act != kActNone;
+    const bool test = withhold >= 0;
+    // the test variant exists for one configuration only (BK = 128, c = 2, two N-blocks per tile)
+    constexpr bool kTestCfg = BK == 128 && C == 2 && Q == 2;
+    if (test && (!kTestCfg || chain || fx)) return cudaErrorInvalidValue;
+    // three variants: one layer without bias or activation, one layer with them, a chain (with them)
+    const void* fn = chain ? reinterpret_cast<const void*>(&tc3_kernel<BK, C, Q, true, true, false>)
+                     : fx  ? reinterpret_cast<const void*>(&tc3_kernel<BK, C, Q, false, true, false>)
+                           : reinterpret_cast<const void*>(&tc3_kernel<BK, C, Q, false, false, false>);
+    if constexpr (kTestCfg)
+        if (test) fn = reinterpret_cast<const void*>(&tc3_kernel<BK, C, Q, false, false, true>);
+    const cudaError_t attr_err = smem_attr_once(fn, F::SMEM);
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap mx, mw, my;
+    Tc3Params prm;
+    memset(&prm, 0, sizeof(prm));
     const CUtensorMapSwizzle wsw = S >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                            : (S == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-    if (!make_map(&mx, X, (uint64_t)L.K, (uint64_t)M, kUnitK, kRows, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
-    if (!make_map(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kNeu, wsw)) return cudaErrorInvalidValue;
-    if (!make_map(&my, Y, (uint64_t)L.N, (uint64_t)M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
-    const int NG = L.NB / Q;
-    const int64_t tiles = (M + kRows - 1) / kRows * NG;
-    const int grid = (int)(tiles < L.num_sms ? tiles : L.num_sms);
-    tc3_kernel<BK, C, Q><<<grid, kThreads, F::SMEM, st>>>(mx, mw, my, L.d_slot, (int)L.K, L.KC, NG, (int)tiles,
-                                                          L.status_dev);
+    for (int l = 0; l < n; ++l) {
+        const ss1_layer& L = *jobs[l].L;
+        Tc3Layer& ly = prm.layer[l];
+        if (!make_map(&ly.tx, jobs[l].X, (uint64_t)L.K, (uint64_t)M, kUnitK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&ly.tw, jobs[l].Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kNeu, wsw) ||
+            !make_map(&ly.ty, jobs[l].Y, (uint64_t)L.N, (uint64_t)M, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+        ly.slot_tab = L.d_slot;
+        ly.bias = static_cast<const __nv_bfloat16*>(jobs[l].bias);
+        ly.K = (int)L.K;
+        ly.KC = L.KC;
+        ly.NG = L.NB / Q;
+        ly.act = jobs[l].act;
+    }
+    prm.n_layers = n;
+    prm.chain = chain ? 1 : 0;
+    prm.status = jobs[0].L->status_dev;
+    prm.wait_ns = wait_ns;
+    prm.withhold_segment = withhold;
+    const int64_t mtiles = (M + kRows - 1) / kRows;
+    const int64_t units = chain ? (mtiles + 1) / 2 : mtiles * prm.layer[0].NG;   // chain: pairs of M-tiles
+    const int sms = jobs[0].L->num_sms;
+    prm.num_units = (int)units;
+    prm.M = (int)M;
+    const int grid = (int)(units < sms ? units : sms);
+    if (chain)
+        tc3_kernel<BK, C, Q, true, true, false><<<grid, kThreads, F::SMEM, st>>>(prm);
+    else if (fx)
+        tc3_kernel<BK, C, Q, false, true, false><<<grid, kThreads, F::SMEM, st>>>(prm);
+    else if constexpr (kTestCfg) {
+        if (test)
+            tc3_kernel<BK, C, Q, false, false, true><<<grid, kThreads, F::SMEM, st>>>(prm);
+        else
+            tc3_kernel<BK, C, Q, false, false, false><<<grid, kThreads, F::SMEM, st>>>(prm);
+    } else {
+        tc3_kernel<BK, C, Q, false, false, false><<<grid, kThreads, F::SMEM, st>>>(prm);
+    }
     return cudaGetLastError();
 }
 
@@ -643,11 +878,16 @@ bool tc3_supported(const ss1_layer& L) {
     return true;
 }
 
-cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+namespace {
+
+// Dispatch on (BK, c, Q) of the first layer; every layer of a chain has the same three.
+cudaError_t launch_jobs(const Tc3Job* jobs, int n, bool chain, int64_t M, cudaStream_t st, uint64_t wait_ns = kWaitNs,
+                        int withhold = -1) {
+    const ss1_layer& L = *jobs[0].L;
     if ((M + kRows - 1) / kRows * L.NB > (int64_t)1 << 30) return cudaErrorInvalidValue;
     const int q = pick_q(L);
 #define SS1_TC3_CASE(bk, cc, qq) \
-    if (L.BK == bk && L.c == cc && q == qq) return launch_cfg<bk, cc, qq>(L, X, Wc, Y, M, st);
+    if (L.BK == bk && L.c == cc && q == qq) return launch_cfg<bk, cc, qq>(jobs, n, chain, M, wait_ns, withhold, st);
     SS1_TC3_CASE(128, 2, 2)
     SS1_TC3_CASE(128, 2, 1)
     SS1_TC3_CASE(128, 4, 2)
@@ -660,6 +900,39 @@ cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* 
     SS1_TC3_CASE(256, 8, 1)
 #undef SS1_TC3_CASE
     return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_tc3(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, const void* bias, int act,
+                       cudaStream_t st) {
+    const Tc3Job job{&L, X, Wc, Y, bias, act};
+    return launch_jobs(&job, 1, false, M, st);
+}
+
+cudaError_t launch_tc3_withhold(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M,
+                                uint64_t wait_ns, cudaStream_t st) {
+    const Tc3Job job{&L, X, Wc, Y, nullptr, kActNone};
+    return launch_jobs(&job, 1, false, M, st, wait_ns, 2);
+}
+
+bool tc3_chain_ok(const ss1_layer* const* Ls, int n) {
+    if (n < 1 || n > kMaxLayers) return false;
+    for (int l = 0; l < n; ++l) {
+        if (!tc3_supported(*Ls[l])) return false;
+        if (Ls[l]->BK != Ls[0]->BK || Ls[l]->c != Ls[0]->c || pick_q(*Ls[l]) != pick_q(*Ls[0])) return false;
+        if (Ls[l]->device != Ls[0]->device) return false;
+        if (l > 0 && Ls[l]->K != Ls[l - 1]->N) return false;
+    }
+    return true;
+}
+
+cudaError_t launch_tc3_chain(const ss1_layer* const* Ls, int n, const void* X, const void* const* Wc, void* const* Y,
+                             const void* const* bias, const int* act, int64_t M, cudaStream_t st) {
+    Tc3Job jobs[kMaxLayers];
+    for (int l = 0; l < n; ++l) jobs[l] = Tc3Job{Ls[l], l == 0 ? X : Y[l - 1], Wc[l], Y[l], bias ? bias[l] : nullptr,
+                                                 act ? act[l] : kActNone};
+    return launch_jobs(jobs, n, true, M, st);
 }
 
 }  // namespace ss1

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libss1.so")
 SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel", "ss1_destroy",
            "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc",
            "ss1_test_device_timeout", "ss1_project", "ss1_backward_workspace", "ss1_backward_input",
-           "ss1_backward_weight", "ss1_quantize_fp8", "ss1_forward_fp8")
+           "ss1_backward_weight", "ss1_quantize_fp8", "ss1_forward_fp8", "ss1_forward_ex", "ss1_chain_forward",
+           "ss1_chain_fused", "ss1_test_forward_timeout")
 
 #: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
 NOALLOC_MAX_ENTRIES = 983040
@@ -33,6 +34,16 @@ class Kernel(IntEnum):
     TC = 1
     SIMT = 2
     SMALLM = 3
+
+
+class Act(IntEnum):
+    NONE = 0
+    RELU = 1
+    GELU = 2
+
+
+#: Layers one chain_forward call takes at most (SS1_CHAIN_MAX_LAYERS in include/ss1.h).
+CHAIN_MAX_LAYERS = 4
 
 
 class DType(IntEnum):
@@ -71,6 +82,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ss1_backward_weight.argtypes = [vp, vp, vp, vp, i64, i32, vp, sz, vp]
     L.ss1_quantize_fp8.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     L.ss1_forward_fp8.argtypes = [vp, vp, vp, vp, vp, i64, vp]
+    L.ss1_forward_ex.argtypes = [vp, vp, vp, vp, i32, vp, i64, i32, i32, vp]
+    L.ss1_chain_forward.argtypes = [ctypes.POINTER(vp), i32, vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                    ctypes.POINTER(i32), ctypes.POINTER(vp), i64, vp]
+    L.ss1_chain_fused.argtypes = [ctypes.POINTER(vp), i32, ctypes.POINTER(i32)]
+    L.ss1_test_forward_timeout.argtypes = [vp, vp, vp, vp, i64, i64, vp]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":
@@ -212,6 +228,25 @@ class SS1Layer:
                                          st.cuda_stream), "ss1_backward_weight")
         return out
 
+    def forward_ex(self, X: torch.Tensor, Wc: torch.Tensor, bias: Optional[torch.Tensor] = None, act: int = Act.NONE,
+                   out: Optional[torch.Tensor] = None, kernel: int = Kernel.AUTO,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """act(SS1(X) + bias) (ss1_forward_ex); bias [N] of X's dtype or None."""
+        if X.dim() != 2 or X.shape[1] != self.K or Wc.shape != (self.N, self.K // self.c) or X.dtype != Wc.dtype:
+            raise ValueError(f"X must be [M, {self.K}] and Wc [{self.N}, {self.K // self.c}] of one dtype")
+        self._check_cuda(X=X, Wc=Wc)
+        if bias is not None:
+            if bias.shape != (self.N,) or bias.dtype != X.dtype:
+                raise ValueError(f"bias must be [{self.N}] of X's dtype")
+            self._check_cuda(bias=bias)
+        M = X.shape[0]
+        out = torch.empty((M, self.N), dtype=X.dtype, device=X.device) if out is None else out
+        st = stream if stream is not None else torch.cuda.current_stream(X.device)
+        _check(lib().ss1_forward_ex(self.handle, X.data_ptr(), Wc.data_ptr(), bias.data_ptr() if bias is not None else None,
+                                    int(act), out.data_ptr(), M, _dtype_code(X.dtype), int(kernel), st.cuda_stream),
+               "ss1_forward_ex")
+        return out
+
     def forward_fp8(self, X: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
         """Y[M, N] (bf16) with FP8 weights: Wq uint8 E4M3 codes [N, K/c], scale float32 [N] (ss1_forward_fp8)."""
@@ -302,6 +337,43 @@ def quantize_fp8(Wc: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -
     _check(lib().ss1_quantize_fp8(Wc.data_ptr(), _dtype_code(Wc.dtype), N, Kc, Wq.data_ptr(), scale.data_ptr(),
                                   st.cuda_stream), "ss1_quantize_fp8")
     return Wq, scale
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() if t is not None else None for t in ts])
+
+
+def chain_fused(layers) -> bool:
+    """Whether chain_forward runs these layers as one persistent launch (ss1_chain_fused)."""
+    hs = (ctypes.c_void_p * len(layers))(*[ly.handle.value for ly in layers])
+    f = ctypes.c_int()
+    _check(lib().ss1_chain_fused(hs, len(layers), ctypes.byref(f)), "ss1_chain_fused")
+    return bool(f.value)
+
+
+def chain_forward(layers, X: torch.Tensor, Wcs, biases=None, acts=None, outs=None,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Every layer's output of a chain of bf16 SS1 layers (ss1_chain_forward)."""
+    n = len(layers)
+    if not (1 <= n <= CHAIN_MAX_LAYERS) or len(Wcs) != n:
+        raise ValueError(f"1 .. {CHAIN_MAX_LAYERS} layers, one Wc each")
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != layers[0].K or not X.is_contiguous():
+        raise ValueError(f"X must be contiguous bf16 [M, {layers[0].K}]")
+    M = X.shape[0]
+    if outs is None:
+        outs = [torch.empty((M, ly.N), dtype=torch.bfloat16, device=X.device) for ly in layers]
+    for ly, W, Y in zip(layers, Wcs, outs):
+        if W.shape != (ly.N, ly.K // ly.c) or W.dtype != torch.bfloat16 or not W.is_contiguous():
+            raise ValueError("each Wc must be contiguous bf16 [N, K/c] of its layer")
+        if Y.shape != (M, ly.N) or Y.dtype != torch.bfloat16 or not Y.is_contiguous():
+            raise ValueError("each output must be contiguous bf16 [M, N] of its layer")
+    hs = (ctypes.c_void_p * n)(*[ly.handle.value for ly in layers])
+    bias_arr = _ptr_array(biases) if biases is not None else None
+    act_arr = (ctypes.c_int * n)(*[int(a) for a in acts]) if acts is not None else None
+    st = stream if stream is not None else torch.cuda.current_stream(X.device)
+    _check(lib().ss1_chain_forward(hs, n, X.data_ptr(), _ptr_array(Wcs), bias_arr, act_arr, _ptr_array(outs), M,
+                                   st.cuda_stream), "ss1_chain_forward")
+    return outs
 
 
 class SS1Function(torch.autograd.Function):

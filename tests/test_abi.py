@@ -74,6 +74,13 @@ def test_argument_checks_before_device(lib):
     assert lib.ss1_backward_input(bogus, None, None, None, 1, 0, None, 0, None) == -7
     assert lib.ss1_backward_weight(bogus, None, None, None, 1, 0, None, 0, None) == -7
     assert lib.ss1_forward_fp8(bogus, None, None, None, None, 1, None) == -7
+    assert lib.ss1_forward_ex(bogus, None, None, None, 0, None, 1, 0, 0, None) == -7
+    hs = (ctypes.c_void_p * 1)(bogus.value)
+    f = ctypes.c_int()
+    assert lib.ss1_chain_fused(hs, 1, ctypes.byref(f)) == -7
+    assert lib.ss1_chain_fused(hs, 5, ctypes.byref(f)) == -1                 # more than SS1_CHAIN_MAX_LAYERS
+    assert lib.ss1_chain_forward(None, 1, None, None, None, None, None, 1, None) == -1
+    assert lib.ss1_test_forward_timeout(bogus, None, None, None, 1, 1000, None) == -7
     assert lib.ss1_quantize_fp8(None, 0, 4, 8, None, None, None) == -1       # NULL pointers
     assert lib.ss1_quantize_fp8(None, 5, 4, 8, None, None, None) == -1       # dtype
     assert lib.ss1_quantize_fp8(None, 0, 0, 8, None, None, None) == 0        # no rows: nothing to do
@@ -101,6 +108,10 @@ def test_binding_constants_match_header():
         assert consts[f"SS1_DTYPE_{d.name}"] == int(d)
     m = re.search(r"#define\s+SS1_NOALLOC_MAX_ENTRIES\s+(\d+)", text)
     assert m and int(m.group(1)) == ss1.NOALLOC_MAX_ENTRIES
+    for a in ss1.Act:
+        assert consts[f"SS1_ACT_{a.name}"] == int(a)
+    m = re.search(r"#define\s+SS1_CHAIN_MAX_LAYERS\s+(\d+)", text)
+    assert m and int(m.group(1)) == ss1.CHAIN_MAX_LAYERS
 
 
 def test_plain_c_program_uses_the_abi(lib, tmp_path):

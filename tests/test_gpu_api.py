@@ -214,3 +214,40 @@ def test_decode_calls_on_one_handle_run_concurrently(K, N, c):
         for it in range(8):
             assert torch.equal(outs[it][i], serial[i])
     layer.close()
+
+
+def test_forward_kernel_timeout_drains_and_recovers():
+    """The tensor-core kernel's own time-out path: one build warp withholds an arrival and every
+    wait is cut to 5 ms, so the sketch warp's wait runs out. The kernel must return (its copies
+    and matrix multiplies drained, tensor memory freed), the handle must report the site, and the
+    next forward on the same context must match the oracle. No GPU fault is involved."""
+    ss1 = get_ss1()
+    lib = ss1.lib()
+    K, N, c, BK, BN, seed, M = 1024, 768, 2, 128, 128, 5, 4096
+    layer = _layer(ss1, K, N, c, BK, BN, seed)
+    gen = torch.Generator().manual_seed(21)
+    X = torch.randn(M, K, generator=gen).to(torch.bfloat16)
+    Wc = (torch.randn(N, K // c, generator=gen) * 0.03).to(torch.bfloat16)
+    Xd, Wd = X.cuda(), Wc.cuda()
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    assert lib.ss1_test_forward_timeout(layer.handle, Xd.data_ptr(), Wd.data_ptr(), Y.data_ptr(), M, 0, st) == -1
+    assert lib.ss1_test_forward_timeout(layer.handle, Xd.data_ptr(), Wd.data_ptr(), Y.data_ptr(), M, 5_000_000, st) == 0
+    torch.cuda.synchronize()            # the kernel returned
+    with pytest.raises(ss1.SS1Error) as err:
+        layer.forward(Xd, Wd)
+    assert err.value.status == -6
+    st_, detail = layer.device_status()
+    # kernel id 1 (the tensor-core kernel) and the site of the first wait to run out, with the
+    # time-out marker bit: the epilogue's wait for the first accumulator, which starts at launch
+    assert st_ == -6 and detail >> 8 == 1 and detail & 0x80 and 1 <= (detail & 0x7F) <= 12, hex(detail)
+    assert layer.device_status() == (0, 0)
+    out = layer.forward(Xd, Wd)
+    torch.cuda.synchronize()
+    assert layer.device_status() == (0, 0)
+    h, g = O.ss1_tables(K, N, c, BK, BN, seed)
+    rows = np.array([0, 1, 127, 128, 2048, M - 1])
+    ref = O.ss1_forward_rows(to_np64(X), to_np64(Wc), h, g, BN, rows)
+    got = to_np64(out[torch.as_tensor(rows).cuda()])
+    assert float((np.abs(got - ref).max(1) / np.abs(ref).max(1)).max()) <= 2e-2
+    layer.close()

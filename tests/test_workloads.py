@@ -63,6 +63,10 @@ def test_bench_layer_selection():
     assert {L.M for L in layers} == {1} and len(layers) == 8
     with pytest.raises(SystemExit):
         bench.select_layers(4, 3)
+    _, layers = bench.select_layers(4, None, "4096x14336c2")
+    assert [(L.K, L.N, L.c, L.M) for L in layers] == [(4096, 14336, 2, 4096)]
+    with pytest.raises(SystemExit):
+        bench.select_layers(4, None, "1x1c2")
 
 
 def test_bench_work_matches_hand_values():
