@@ -708,7 +708,7 @@ def main():
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(evs=None):
+    def step(evs=None, launches=None):
         for i, (L, layer, Xd, Wd, Yd, _) in enumerate(objs):
             if args.nvtx:
                 torch.cuda.nvtx.range_push(f"ss1_forward {L.K}x{L.N} M={L.M} c={L.c}")
@@ -720,12 +720,15 @@ def main():
                 layer.forward(Xd, Wd, out=Yd)
             if evs is not None:
                 evs[i][1].record(stream)
+            if launches is not None:
+                launches.append(ss1.last_launch())
             if args.nvtx:
                 torch.cuda.nvtx.range_pop()
 
-    for _ in range(max(args.warmup, 3)):
+    launches = []
+    for w in range(max(args.warmup, 3)):
         flush.zero_()
-        step()
+        step(launches=launches if w == 0 else None)
     torch.cuda.synchronize()
     for (L, layer, *_r) in objs:
         st, detail = layer.device_status()
@@ -861,8 +864,9 @@ def main():
                     "dense_tflops": layer_work(L)[0] / (ms * 1e-3) / 1e12,
                     "actual_tflops": layer_work(L)[1] / (ms * 1e-3) / 1e12,
                     "gbs": layer_work(L, isfp8)[2] / (ms * 1e-3) / 1e9,
-                    "roofline_frac": max(t_compute(L), layer_work(L, isfp8)[2] / hbm_peak) / (ms * 1e-3)}
-                   for L, k, ms in zip(layers, kernels, layer_ms)],
+                    "roofline_frac": max(t_compute(L), layer_work(L, isfp8)[2] / hbm_peak) / (ms * 1e-3),
+                    "launch": {"kernel": ln["kernel"], "grid": list(ln["grid"]), "cluster_y": ln["cluster_y"]}}
+                   for L, k, ms, ln in zip(layers, kernels, layer_ms, launches)],
         "roofline": roof,
         "gpu_launches": K * len(objs),
         "clocks": sampler.summary(),

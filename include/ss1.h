@@ -377,6 +377,30 @@ SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, void* stream
 SS1_API int ss1_test_forward_timeout(ss1_handle h, const void* X, const void* Wc, void* Y, int64_t M, int64_t limit_ns,
                                      void* stream);
 
+/*
+ * ss1_last_launch -- the shape of the main kernel that the last layer entry point (ss1_forward,
+ * _with, _ex, ss1_chain_forward, ss1_forward_fp8, ss1_forward_noalloc) called on this host thread
+ * launched: which kernel, its grid, cluster and block. For checking that a launch uses the
+ * machine as intended (how many CTAs, how K is split); it has no counterpart on the SS1 pages.
+ *   kernel : static name: "tc3" (large-M tensor-core kernel, c >= 2), "tc" (c = 1), "tc2",
+ *            "simt", "dec" (tensor-core decode kernel), "dec_fp8", "smallm"; "" before any launch.
+ *   grid_x, grid_y : CTAs of the grid (grid_y: K-splits where the kernel splits K).
+ *   cluster_y : CTAs per thread-block cluster along y (1: no cluster).
+ *   threads, smem_bytes : per CTA (dynamic shared memory).
+ *   resident_clusters[s], s = 1 .. 16 : what the occupancy query behind the K-split choice
+ *            reported (clusters of s CTAs resident at once); all 0 where none was made.
+ * out : host pointer. Errors: INVALID_ARG (NULL).
+ */
+typedef struct {
+    const char* kernel;
+    int grid_x, grid_y;
+    int cluster_y;
+    int threads;
+    int smem_bytes;
+    int resident_clusters[17];
+} ss1_launch_info;
+SS1_API int ss1_last_launch(ss1_launch_info* out);
+
 #ifdef __cplusplus
 }
 #endif

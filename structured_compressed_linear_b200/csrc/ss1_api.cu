@@ -116,7 +116,11 @@ cudaError_t smem_attr_once(const void* kernel, int bytes) {
     const uint64_t ctx = current_context_id();
     std::lock_guard<std::mutex> lk(mu);
     if (ctx != 0 && done.count({kernel, ctx})) return cudaSuccess;
-    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // the largest shared-memory carveout, so that as many CTAs as the shared memory allows are
+    // resident (and the occupancy queries behind the K-split choices count them)
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     // the attribute call makes the device's context current, so its id is known from here on
     const uint64_t now = current_context_id();
     if (e == cudaSuccess && now != 0) done.insert({kernel, now});
@@ -169,6 +173,22 @@ int pick_splits(const ClusterFit& f, int groups, int want, int units) {
     return best;
 }
 
+namespace {
+thread_local ss1_launch_info g_last_launch = {"", 0, 0, 0, 0, 0, {}};
+}
+
+void note_launch(const char* kernel, unsigned grid_x, unsigned grid_y, int cluster_y, int threads, int smem,
+                 const ClusterFit* fit) {
+    ss1_launch_info& r = g_last_launch;
+    r.kernel = kernel;
+    r.grid_x = (int)grid_x;
+    r.grid_y = (int)grid_y;
+    r.cluster_y = cluster_y;
+    r.threads = threads;
+    r.smem_bytes = smem;
+    for (int s = 0; s <= 16; ++s) r.resident_clusters[s] = fit ? fit->active[s] : 0;
+}
+
 bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN) {
     if (K < 1 || N < 1 || BK < 1 || BN < 1) return false;
     if (!(c == 1 || c == 2 || c == 4 || c == 8)) return false;
@@ -179,6 +199,12 @@ bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN) {
 }  // namespace ss1
 
 extern "C" {
+
+SS1_API int ss1_last_launch(ss1_launch_info* out) {
+    if (!out) return SS1_ERR_INVALID_ARG;
+    *out = ss1::g_last_launch;
+    return SS1_OK;
+}
 
 SS1_API const char* ss1_strerror(int status) {
     switch (status) {

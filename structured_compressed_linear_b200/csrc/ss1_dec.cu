@@ -10,17 +10,20 @@
 // with UMMA N = the row count rounded up to 16, so the tensor pipe is busy a few percent of the
 // time and the kernel is a TMA stream of Wc.
 //
-// CTA = (N-block nb, K-split s): the split's stages of 64 compressed columns.
-//   warp 0     : TMA loads of Wc stages [128 neurons x 64 columns] (128-byte swizzle) into a ring,
-//                one issuing lane per ring slot.
+// CTA = (N-block nb, K-split s): the split's stages of 64 compressed columns; one CTA per SM.
+//   warp 0     : lane 0 copies the CTA's X columns (one bulk copy per row) where they fit in
+//                shared memory, then refills a ring of 11 Wc stages [128 neurons x 64 columns]
+//                (128-byte swizzle, 176 KB) by TMA in stage order.
 //   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage.
 //   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
 //                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
-//                stages, warps 4-5 the odd ones), gathering from shared memory: for up to 16 rows
-//                the X rows of each unit (one K-chunk of whole stages, or one stage of whole
-//                K-chunks) arrive by TMA (one more lane of warp 0) into a two-unit ring;
-//                otherwise the CTA's X columns are copied in once where they fit in 20 KB, or
-//                the gathers go to L1 / L2. Then the epilogue.
+//                stages, warps 4-5 the odd ones), gathering from shared memory: the CTA's X
+//                columns copied in once; or, for up to 16 rows whose columns do not fit, the X
+//                rows of each unit (one K-chunk of whole stages, or one stage of whole K-chunks)
+//                by TMA (one more lane of warp 0) into a two-unit ring; else the gathers go to
+//                L1 / L2. Then the epilogue.
+// Before the dependency wait of a programmatic dependent launch the CTA asks L2 for its X
+// columns and its first Wc stages.
 // Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: the K-splits of one
 // N-block form one thread-block cluster. Every CTA leaves its fp32 partial [rows x 128 neurons]
 // in its own shared memory; after a cluster barrier, CTA r sums rows r, r + splits, ... over the
@@ -46,12 +49,10 @@ namespace {
 
 constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
 constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
-constexpr int kWRing = 64 * 1024;         // shared memory of the Wc ring: 4 bf16 or 8 FP8 stages
+constexpr int kWRing = 176 * 1024;        // shared memory of the Wc ring: 11 bf16 or 22 FP8 stages
 constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
-constexpr int kNB = 3;                    // sketch stages in the ring
-constexpr int kPrefetchStages = 16;       // Wc stages asked of L2 before the previous kernel ends
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kFirstConv = kFirstBuild + kBuildWarps, kConvWarps = 4;   // FP8 weights: the converter warps
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -62,6 +63,11 @@ __device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int c0, i
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
                  "r"(c0), "r"(c1)
                  : "memory");
+}
+
+// L2 prefetch of a contiguous range (16-byte aligned, a multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes) : "memory");
 }
 
 // Programmatic dependent launch. pdl_wait blocks until the grids this one depends on have
@@ -77,24 +83,31 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 template <int MP, bool FP8>
 struct DecCfg {
     static constexpr int W_STAGE = kNeu * kStageC * (FP8 ? 1 : 2);   // 8 or 16 KB
-    static constexpr int NW = kWRing / W_STAGE;                       // Wc stages in the ring (8 or 4)
+    static constexpr int NW = kWRing / W_STAGE;                       // Wc stages in the ring (22 or 11)
     static constexpr int THREADS = (kFirstBuild + kBuildWarps + (FP8 ? kConvWarps : 0)) * 32;
-    static constexpr int MIN_CTAS = (FP8 && MP == 64) ? 1 : 2;          // registers: 168 for MP = 64
+    // one CTA per SM with a deep ring: a stage stays in the ring from its load until its UMMAs
+    // complete, and about 128 KB per SM must be on the way from HBM at any time for it to run at
+    // its rate at the latency it has under that load
+    static constexpr int MIN_CTAS = 1;
     static constexpr int B_STAGE = MP * 128;                    // [MP rows x 64] bf16
+    // sketch stages in the ring (the build warps run ahead of the UMMAs); FP8 three, each also
+    // holding a bf16 A stage in TMEM
+    static constexpr int NBS = (FP8 || MP == 64) ? 3 : 4;
     static constexpr int OFF_W = 0;
     static constexpr int OFF_B = kWRing;
-    static constexpr int OFF_X = OFF_B + kNB * B_STAGE;
+    static constexpr int OFF_X = OFF_B + NBS * B_STAGE;
     static constexpr int X_BYTES = MP == kXChunkRows ? 2 * kXUnitBytes : kXBytes;   // the ring, or the range
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
-    static constexpr int NBAR = 2 * NW + 2 * kNB + 1 + 4;
+    static constexpr int NBAR = 2 * NW + 2 * NBS + 1 + 4;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-    // accumulator MP columns; FP8: plus kNB bf16 A stages of 32 columns from A_COL
+    // accumulator MP columns; FP8: plus NBS bf16 A stages of 32 columns from A_COL
     static constexpr int A_COL = MP <= 32 ? 32 : 64;
     static constexpr uint32_t TMEM_COLS = FP8 ? (MP <= 32 ? 128 : 256) : (MP <= 32 ? 32 : 64);
     static_assert(MP % 16 == 0 && MP >= 16 && MP <= 64, "UMMA N for M = 128");
     static_assert(B_STAGE % 1024 == 0 && OFF_B % 1024 == 0, "swizzle atoms stay aligned");
-    static_assert(!FP8 || (A_COL >= MP && A_COL + kNB * 32 <= (int)TMEM_COLS), "TMEM layout");
-    static_assert(NW <= 31, "one loader lane per ring slot, plus the X lane");
+    static_assert(!FP8 || (A_COL >= MP && A_COL + NBS * 32 <= (int)TMEM_COLS), "TMEM layout");
+    static_assert(NW <= 31, "the chunk-mode X loader is lane NW of the load warp");
+    static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Two E4M3 codes (low byte = the even column) -> bf16x2, exactly: every E4M3 value has at most
@@ -119,6 +132,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Wait of the UMMA-issuing warp: every lane polls without suspending, so the issue resumes as
+// soon as the phase completes (a suspending wait costs the issuing thread several hundred cycles).
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+    bool ok = ptx::mbar_test(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = ptx::globaltimer_ns();
+        for (uint32_t n = 1;; ++n) {
+            if (ptx::mbar_test(bar, parity)) { ok = true; break; }
+            if ((n & 63) == 0 && (*abort_flag || ptx::globaltimer_ns() - t0 > kWaitNs)) break;
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
 template <int MP, int C, bool FP8>
 __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN_CTAS)
     dec_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
@@ -126,7 +153,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                const float* __restrict__ scale, int M, int K, int N, int S, int KC, int splits, int chunked, int ui,
                int bi, int32_t* status) {
     using F = DecCfg<MP, FP8>;
-    constexpr int kNW = F::NW, kWStage = F::W_STAGE, kThreads = F::THREADS, kACol = F::A_COL;
+    constexpr int kNW = F::NW, kWStage = F::W_STAGE, kThreads = F::THREADS, kACol = F::A_COL, kNB = F::NBS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* wring = smem + F::OFF_W;
@@ -160,6 +187,14 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         st1 = (int)((int64_t)nstg * (split + 1) / splits);
     }
     const int G = st1 - st0;   // stages of this CTA (>= 1)
+    // Outside chunk mode the X columns of this CTA's K-chunks (all rows) are copied into shared
+    // memory once where they fit (one bulk copy per row; then every gather is a shared-memory
+    // read); else the gathers go to L1 / L2.
+    const int BKc = S * C;
+    const int kc_lo = (st0 * kStageC) / S;
+    const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
+    const int R = (kc_hi - kc_lo + 1) * BKc;   // inputs of the range
+    const bool staged = !chunked && BKc % 8 == 0 && (int64_t)M * R * 2 <= F::X_BYTES;   // 16-byte aligned rows
 
     // sketch stages start zeroed: rows past M are never written afterwards
     for (int i = threadIdx.x; i < kNB * F::B_STAGE / 16; i += kThreads)
@@ -189,24 +224,36 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
     const uint32_t tm = *tmem_slot;
 
     // The launch may overlap the end of the previous kernel on the stream (programmatic
-    // dependent launch). Until that kernel has completed, this CTA only asks L2 for the first
-    // Wc stages it will stream: a prefetch goes through L2, so it cannot return data older than
-    // what that kernel writes. Every global read and write below comes after the wait.
+    // dependent launch). Until that kernel has completed, this CTA only asks L2 for its X columns
+    // and the first Wc stages it will stream: a prefetch goes through L2, so it cannot return
+    // data older than what that kernel writes. Every global read and write below comes after
+    // the wait.
     if (warp == kWarpLoad && lane == 0) {
-        for (int g = 0; g < G && g < kPrefetchStages; ++g)
+        if (staged)
+            for (int m = 0; m < M; ++m) prefetch_l2_bulk(X + (size_t)m * K + (size_t)kc_lo * BKc, (uint32_t)(R * 2));
+        for (int g = 0; g < G && g < kNW; ++g)
             prefetch_l2_2d(&tmap_w, (st0 + g) * kStageC, nb * kNeu);
     }
     if (threadIdx.x == 0) pdl_launch_dependents();
     pdl_wait();
 
     if (warp == kWarpLoad) {
-        // ------------------------------------------------------------------ TMA loads of Wc
-        // Lane l owns ring slot l (stages l, l + kNW, ...): the copies of one issuing thread are
-        // served one after another, so kNW threads keep kNW stages coming from HBM at once.
-        if (lane < kNW) {
-            const int slot = lane;
+        // ------------------------------------------------------------------ TMA loads
+        // The X columns first (the sketch waits for them), one bulk copy per row, by lane 0.
+        if (staged && lane == 0) {
+            ptx::mbar_arrive_expect_tx(&x_full[0], (uint32_t)(M * R * 2));
+            for (int m = 0; m < M; ++m)
+                ptx::bulk_load(smem + F::OFF_X + (size_t)m * R * 2, X + (size_t)m * K + (size_t)kc_lo * BKc,
+                               (uint32_t)(R * 2), &x_full[0]);
+        }
+        __syncwarp();
+        // Wc: lane 0 refills the ring in stage order (stage g into slot g % kNW once the UMMAs of
+        // stage g - kNW have completed). Issuing from several lanes was measured no faster: the
+        // copies of one SM are served one after another either way.
+        if (lane == 0) {
             int issued = 0;
-            for (int g = slot; g < G; g += kNW) {
+            for (int g = 0; g < G; ++g) {
+                const int slot = g % kNW;
                 if (g >= kNW && !ptx::mbar_wait(&w_empty[slot], (uint32_t)(((g / kNW) - 1) & 1), abort_flag, kWaitNs)) {
                     report(status, abort_flag, 1);
                     break;
@@ -215,9 +262,10 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 ptx::tma_load_2d(wring + slot * kWStage, &tmap_w, &w_full[slot], (st0 + g) * kStageC, nb * kNeu);
                 ++issued;
             }
-            if (*abort_flag && issued > 0) {   // this slot's last copy lands before exit
+            if (*abort_flag) {   // the copies in flight land before exit
                 volatile int no_abort = 0;
-                ptx::mbar_wait(&w_full[slot], (uint32_t)((issued - 1) & 1), &no_abort, kWaitNs);
+                for (int g = issued > kNW ? issued - kNW : 0; g < issued; ++g)
+                    ptx::mbar_wait(&w_full[g % kNW], (uint32_t)((g / kNW) & 1), &no_abort, kWaitNs);
             }
         } else if (lane == kNW && chunked) {
             // X units [16 rows x ui] (rows past M read as zero) into a ring of two, as boxes of
@@ -242,6 +290,10 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                     ptx::mbar_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), &no_abort, kWaitNs);
             }
         }
+        if (staged && lane == 0 && *abort_flag) {   // the X copies land before exit
+            volatile int no_abort = 0;
+            ptx::mbar_wait(&x_full[0], 0, &no_abort, kWaitNs);
+        }
     } else if (warp == kWarpMma) {
         // ------------------------------------------------------------------ UMMAs
         constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, MP);
@@ -250,8 +302,8 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         bool ok = true;
         for (int g = 0; g < G && ok; ++g) {
             const int ws_ = g % kNW, bs = g % kNB;
-            if ((!FP8 && !warp_wait(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag)) ||
-                !warp_wait(&b_full[bs], (uint32_t)((g / kNB) & 1), abort_flag)) {
+            if ((!FP8 && !warp_wait_spin(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag)) ||
+                !warp_wait_spin(&b_full[bs], (uint32_t)((g / kNB) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 2);
                 ok = false;
                 break;
@@ -268,8 +320,8 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                     else
                         ptx::umma_bf16_ss(tm, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (!FP8) ptx::umma_commit(&w_empty[ws_]);
-                ptx::umma_commit(&b_empty[bs]);
+                if (!FP8 && g + kNW < G) ptx::umma_commit(&w_empty[ws_]);   // only a slot used again
+                if (g + kNB < G) ptx::umma_commit(&b_empty[bs]);
             }
             __syncwarp();
         }
@@ -328,7 +380,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         // so that a stage waits only for its X gathers, which are all in flight together.
         const int t = threadIdx.x - kFirstBuild * 32;
         const int kl = t % kStageC, half = t / kStageC;
-        const int BK = S * C;
+        const int BK = BKc;
         const uint16_t* tab = src + (size_t)nb * KC * S * C;   // this N-block's entries, column-major order
         auto fetch = [&](int g, uint16_t (&e)[C]) {
             const int j = (st0 + g) * kStageC + kl;
@@ -337,26 +389,15 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 for (int q = 0; q < C; ++q) e[q] = __ldg(tab + (size_t)j * C + q);
             }
         };
-        // The X columns of this CTA's chunks, all rows, staged once in shared memory when they fit
-        // (then every gather is a shared-memory read); else the gathers go to L1 / L2.
-        const int kc_lo = (st0 * kStageC) / S;
-        const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
-        const int R = (kc_hi - kc_lo + 1) * BK;   // inputs of the range
-        const bool staged = !chunked && BK % 8 == 0 && (int64_t)M * R * 2 <= F::X_BYTES;   // 16-byte aligned rows
         const __nv_bfloat16* xsm = reinterpret_cast<const __nv_bfloat16*>(smem + F::OFF_X);
-        if (staged) {
-            const int r8 = R / 8;
-            for (int i = t; i < M * r8; i += kBuildWarps * 32) {
-                const int m = i / r8, c8 = i - m * r8;
-                *reinterpret_cast<uint4*>(smem + F::OFF_X + ((size_t)m * R + c8 * 8) * 2) =
-                    __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + (size_t)kc_lo * BK + c8 * 8));
-            }
-            ptx::named_barrier_sync(1, kBuildWarps * 32);   // the build warps only
-        }
         uint16_t ent[C];
-        fetch(half, ent);
+        fetch(half, ent);   // in flight together with the X copy
         bool ok = true;
-        for (int g = half; g < G; g += 2) {
+        if (staged && !warp_wait(&x_full[0], 0, abort_flag)) {   // the CTA's X columns have landed
+            if (lane == 0) report(status, abort_flag, 8);
+            ok = false;
+        }
+        for (int g = half; g < G && ok; g += 2) {
             const int bs = g % kNB;
             uint16_t cur[C];
 #pragma unroll
@@ -459,8 +500,15 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             const float* part = reinterpret_cast<const float*>(wring) + t;
             const float sc = FP8 ? scale[(size_t)nb * kNeu + t] : 1.0f;
             for (int m = (int)ptx::cluster_ctarank(); m < M && m < MP; m += splits) {
+                // every split's partial requested before the first is added: one remote latency
+                float pv[16];
+#pragma unroll
+                for (int s = 0; s < 16; ++s)
+                    pv[s] = s < splits ? ptx::ld_cluster_f32(ptx::map_to_rank(part + (size_t)m * kNeu, (uint32_t)s)) : 0.f;
                 float v = 0.f;
-                for (int s = 0; s < splits; ++s) v += ptx::ld_cluster_f32(ptx::map_to_rank(part + (size_t)m * kNeu, (uint32_t)s));
+#pragma unroll
+                for (int s = 0; s < 16; ++s)
+                    if (s < splits) v += pv[s];   // in split order
                 Y[(size_t)m * N + (size_t)nb * kNeu + t] = __float2bfloat16_rn(FP8 ? sc * v : v);
             }
         }
@@ -548,6 +596,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, const 
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = splits > 1 ? 2 : 1;
+    note_launch(FP8 ? "dec_fp8" : "dec", cfg.gridDim.x, cfg.gridDim.y, splits, F::THREADS, F::SMEM, &fit);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_kernel<MP, C, FP8>, mw, mx, (const __nv_bfloat16*)X,
                                              (__nv_bfloat16*)Y, (const uint16_t*)L.d_src, scale, (int)M, (int)L.K,
                                              (int)L.N, L.S, L.KC, splits, chunked, ui, bi, L.status_dev);

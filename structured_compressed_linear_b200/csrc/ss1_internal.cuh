@@ -57,11 +57,17 @@ ClusterFit cluster_fit(const void* fn, int smem, int threads);
 // none does, the one that keeps the most CTAs resident.
 int pick_splits(const ClusterFit& f, int groups, int want, int units);
 
+// Records the shape of a layer kernel's launch for ss1_last_launch (per host thread). `fit` is the
+// occupancy query behind a K-split choice, or null.
+void note_launch(const char* kernel, unsigned grid_x, unsigned grid_y, int cluster_y, int threads, int smem,
+                 const ClusterFit* fit);
+
 // Y[m, n] = act(Y[m, n] + bias[n]) in place (bias may be null), for kernels without the fused epilogue.
 cudaError_t launch_bias_act(void* Y, const void* bias, int act, int64_t M, int64_t N, int dtype, cudaStream_t st);
 
-// Raises `kernel`'s dynamic shared-memory limit to `bytes` in the current context. The attribute
-// belongs to a context, so it is set once per (kernel, context); later calls return at once.
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` and asks for the largest shared-memory
+// carveout, in the current context. The attributes belong to a context, so they are set once per
+// (kernel, context); later calls return at once.
 cudaError_t smem_attr_once(const void* kernel, int bytes);
 
 cudaError_t launch_hashgen(const ss1_layer& L, cudaStream_t st);

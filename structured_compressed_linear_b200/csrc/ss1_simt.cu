@@ -116,7 +116,15 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
         // element e = (row, column) of the tile; CTA r takes rows r, r + splits, ...
         if ((int)threadIdx.x >= TN) break;
         float v = 0.f;
-        for (int sp = 0; sp < splits; ++sp) v += ptx::ld_cluster_f32(ptx::map_to_rank(stage_buf + e, (uint32_t)sp));
+        for (int s0 = 0; s0 < splits; s0 += 8) {   // eight partials requested before the first is added
+            float pv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                pv[q] = s0 + q < splits ? ptx::ld_cluster_f32(ptx::map_to_rank(stage_buf + e, (uint32_t)(s0 + q))) : 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (s0 + q < splits) v += pv[q];   // in split order
+        }
         from_f32(Y[(size_t)(m0 + e / TN) * N + n0 + e % TN], v);
     }
     ptx::cluster_sync();   // the peers have read this CTA's partial
@@ -129,8 +137,11 @@ cudaError_t launch_t(const ss1_layer& L, const void* X, const void* Wc, void* Y,
     // K-splits (one cluster per output tile) where the tiles alone leave most SMs idle
     int splits = 1;
     const void* fn = reinterpret_cast<const void*>(&simt_kernel<T, TM, TN>);
-    if (tiles < 2 * (int64_t)L.num_sms && L.KC > 1)
-        splits = pick_splits(cluster_fit(fn, 0, kThreads), (int)tiles, (int)((2 * (int64_t)L.num_sms) / tiles), L.KC);
+    ClusterFit fit;
+    if (tiles < 2 * (int64_t)L.num_sms && L.KC > 1) {
+        fit = cluster_fit(fn, 0, kThreads);
+        splits = pick_splits(fit, (int)tiles, (int)((2 * (int64_t)L.num_sms) / tiles), L.KC);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits);
     cfg.blockDim = dim3(kThreads);
@@ -143,6 +154,7 @@ cudaError_t launch_t(const ss1_layer& L, const void* X, const void* Wc, void* Y,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = splits > 1 ? 1 : 0;
+    note_launch("simt", cfg.gridDim.x, cfg.gridDim.y, splits, kThreads, 0, &fit);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, simt_kernel<T, TM, TN>, (const T*)X, (const T*)Wc, (T*)Y,
                                              (const uint16_t*)L.d_src, (int)M, (int)L.K, (int)L.N, L.c, L.BK, L.BN,
                                              L.S, (int)ntn);

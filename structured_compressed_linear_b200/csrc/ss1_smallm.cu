@@ -180,6 +180,7 @@ int log2_exact(int v) {
 template <int MT, int G, int C>
 cudaError_t launch_tpl(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
     const dim3 grid((unsigned)(L.N / (4 * G)), (unsigned)((M + MT - 1) / MT));
+    note_launch("smallm", grid.x, grid.y, 1, kThreads, 0, nullptr);
     smallm_kernel<MT, G, C><<<grid, kThreads, 0, st>>>((const __nv_bfloat16*)X, (const __nv_bfloat16*)Wc,
                                                        (__nv_bfloat16*)Y, L.d_src, (int)M, (int)L.K, (int)L.N,
                                                        L.BN, log2_exact(L.S), L.KC);

@@ -259,6 +259,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     if (!make_map_2d(&mw, Wc, (uint64_t)(L.K / L.c), (uint64_t)L.N, S >= 64 ? 64 : S, kBN, wsw))
         return cudaErrorInvalidValue;
     dim3 grid((unsigned)L.NB, (unsigned)((M + kBM - 1) / kBM));
+    note_launch("tc", grid.x, grid.y, 1, kThreads, F::SMEM, nullptr);
     tc_kernel<BK><<<grid, kThreads, F::SMEM, st>>>(mx, mw, (__nv_bfloat16*)Y, (int)M, (int)L.N, L.KC, L.status_dev);
     return cudaGetLastError();
 }

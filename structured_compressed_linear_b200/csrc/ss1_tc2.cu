@@ -502,6 +502,7 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     const int64_t mtiles = (M + kRows - 1) / kRows;
     const int64_t tiles = mtiles * L.NB;
     const int grid = (int)(tiles < L.num_sms ? tiles : L.num_sms);
+    note_launch("tc2", (unsigned)grid, 1, 1, kThreads, F::SMEM, nullptr);
     tc2_kernel<BK, C><<<grid, kThreads, F::SMEM, st>>>(mx, (const __nv_bfloat16*)Wc, (__nv_bfloat16*)Y, L.d_gather, (int)M,
                                                        (int)L.N, (int)(L.K / L.c), L.KC, L.NB, (int)tiles, L.status_dev);
     return cudaGetLastError();

@@ -845,6 +845,7 @@ cudaError_t launch_cfg(const Tc3Job* jobs, int n, bool chain, int64_t M, uint64_
     prm.num_units = (int)units;
     prm.M = (int)M;
     const int grid = (int)(units < sms ? units : sms);
+    note_launch("tc3", (unsigned)grid, 1, 1, kThreads, F::SMEM, nullptr);
     if (chain)
         tc3_kernel<BK, C, Q, true, true, false><<<grid, kThreads, F::SMEM, st>>>(prm);
     else if (fx)

@@ -23,7 +23,7 @@ SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel",
            "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc",
            "ss1_test_device_timeout", "ss1_project", "ss1_backward_workspace", "ss1_backward_input",
            "ss1_backward_weight", "ss1_quantize_fp8", "ss1_forward_fp8", "ss1_forward_ex", "ss1_chain_forward",
-           "ss1_chain_fused", "ss1_test_forward_timeout")
+           "ss1_chain_fused", "ss1_test_forward_timeout", "ss1_last_launch")
 
 #: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
 NOALLOC_MAX_ENTRIES = 983040
@@ -52,6 +52,13 @@ class DType(IntEnum):
 
 
 _lib = None
+
+
+class _LaunchInfo(ctypes.Structure):
+    """ss1_launch_info of include/ss1.h."""
+    _fields_ = [("kernel", ctypes.c_char_p), ("grid_x", ctypes.c_int), ("grid_y", ctypes.c_int),
+                ("cluster_y", ctypes.c_int), ("threads", ctypes.c_int), ("smem_bytes", ctypes.c_int),
+                ("resident_clusters", ctypes.c_int * 17)]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -87,6 +94,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     ctypes.POINTER(i32), ctypes.POINTER(vp), i64, vp]
     L.ss1_chain_fused.argtypes = [ctypes.POINTER(vp), i32, ctypes.POINTER(i32)]
     L.ss1_test_forward_timeout.argtypes = [vp, vp, vp, vp, i64, i64, vp]
+    L.ss1_last_launch.argtypes = [ctypes.POINTER(_LaunchInfo)]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":
@@ -337,6 +345,15 @@ def quantize_fp8(Wc: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -
     _check(lib().ss1_quantize_fp8(Wc.data_ptr(), _dtype_code(Wc.dtype), N, Kc, Wq.data_ptr(), scale.data_ptr(),
                                   st.cuda_stream), "ss1_quantize_fp8")
     return Wq, scale
+
+
+def last_launch() -> dict:
+    """Shape of the main kernel launched by the last layer call on this thread (ss1_last_launch)."""
+    info = _LaunchInfo()
+    _check(lib().ss1_last_launch(ctypes.byref(info)), "ss1_last_launch")
+    return {"kernel": (info.kernel or b"").decode(), "grid": (info.grid_x, info.grid_y), "cluster_y": info.cluster_y,
+            "threads": info.threads, "smem_bytes": info.smem_bytes,
+            "resident_clusters": list(info.resident_clusters)}
 
 
 def _ptr_array(ts):

@@ -130,10 +130,31 @@ def test_plain_c_program_uses_the_abi(lib, tmp_path):
         '  if (strcmp(ss1_strerror(SS1_OK), "ok") != 0) return 1;\n'
         "  if (ss1_create(770, 768, 2, 64, 64, 0, &h) != SS1_ERR_INVALID_ARG || h != 0) return 2;\n"
         "  if (ss1_forward(0, 0, 0, 0, 1, SS1_DTYPE_BF16, 0) != SS1_ERR_BAD_HANDLE) return 3;\n"
-        '  puts("c-abi ok");\n  return 0;\n}\n')
+        "  ss1_launch_info li;\n"
+        "  if (ss1_last_launch(&li) != SS1_OK || li.kernel == 0 || li.kernel[0] != 0) return 4;\n"
+        "  if (ss1_last_launch(0) != SS1_ERR_INVALID_ARG) return 5;\n"
+        '  printf("c-abi ok %u\\n", (unsigned)sizeof(ss1_launch_info));\n  return 0;\n}\n')
     exe = tmp_path / "use_ss1"
     libdir = os.path.join(ROOT, "structured_compressed_linear_b200")
     subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), str(src),
                     "-L", libdir, "-lss1", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
-    assert out.returncode == 0 and out.stdout.strip() == "c-abi ok", (out.returncode, out.stdout, out.stderr)
+    from structured_compressed_linear_b200 import ss1
+    expect = f"c-abi ok {ctypes.sizeof(ss1._LaunchInfo)}"
+    assert out.returncode == 0 and out.stdout.strip() == expect, (out.returncode, out.stdout, out.stderr)
+
+
+def test_last_launch_before_any_launch(lib):
+    """ss1_last_launch is per host thread: a thread that launched nothing reads an empty record."""
+    import threading
+    from structured_compressed_linear_b200 import ss1
+    got = {}
+
+    def probe():
+        got["info"] = ss1.last_launch()
+    t = threading.Thread(target=probe)
+    t.start()
+    t.join()
+    info = got["info"]
+    assert info["kernel"] == "" and info["grid"] == (0, 0) and info["resident_clusters"] == [0] * 17
+    assert lib.ss1_last_launch(None) == -1
