@@ -12,9 +12,11 @@
 //
 // CTA = (N-block nb, K-split s): the split's stages of 64 compressed columns; one CTA per SM.
 //   warp 0     : lane 0 copies the CTA's X columns (one bulk copy per row) where they fit in
-//                shared memory, then refills a ring of 11 Wc stages [128 neurons x 64 columns]
-//                (128-byte swizzle, 176 KB) by TMA in stage order.
-//   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage.
+//                shared memory, then refills a ring of Wc stages [128 neurons x 64 columns]
+//                (128-byte swizzle; bf16 8 x 16 KB, FP8 22 x 8 KB) by TMA in stage order.
+//   warp 1     : TMEM allocation; lane 0 issues 4 UMMAs (K = 16) per stage for the even stages
+//                (bf16; FP8 every stage); warp 6 (bf16) the odd stages into a second
+//                accumulator; the epilogue adds the two in order.
 //   warps 2..5 : the sketch of each stage, Xs[m, j] = sum_t sign_t * X[m, chunk(j) * BK + k_t]
 //                (fp32 sum, one rounding to bf16), into a swizzled B stage (warps 2-3 the even
 //                stages, warps 4-5 the odd ones), gathering from shared memory: the CTA's X
@@ -49,12 +51,15 @@ namespace {
 
 constexpr int kNeu = 128;                 // neurons per N-block = UMMA M
 constexpr int kStageC = 64;               // compressed columns per stage (one 128-byte swizzle row)
-constexpr int kWRing = 176 * 1024;        // shared memory of the Wc ring: 11 bf16 or 22 FP8 stages
+constexpr int kWRingFp8 = 176 * 1024;     // shared memory of the FP8 Wc ring: 22 stages
+constexpr int kNwBf16 = 8;                // bf16 Wc stages in the ring
+constexpr int kNmmaBf16 = 2;              // bf16 UMMA warps
 constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kFirstConv = kFirstBuild + kBuildWarps, kConvWarps = 4;   // FP8 weights: the converter warps
+constexpr int kWarpMma2 = kFirstBuild + kBuildWarps;   // bf16: the further UMMA warps, from here
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // L2 prefetch of one 2D tile of a tensor map: no shared memory, no completion to wait for.
@@ -83,8 +88,11 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 template <int MP, bool FP8>
 struct DecCfg {
     static constexpr int W_STAGE = kNeu * kStageC * (FP8 ? 1 : 2);   // 8 or 16 KB
-    static constexpr int NW = kWRing / W_STAGE;                       // Wc stages in the ring (22 or 11)
-    static constexpr int THREADS = (kFirstBuild + kBuildWarps + (FP8 ? kConvWarps : 0)) * 32;
+    static constexpr int NW = FP8 ? kWRingFp8 / W_STAGE : kNwBf16;   // Wc stages in the ring
+    // bf16: NMMA UMMA warps take the stages round-robin into NMMA accumulators, so that the
+    // barrier waits of one (each lets the tensor pipe's queue drain) overlap the others' UMMAs
+    static constexpr int NMMA = FP8 ? 1 : kNmmaBf16;
+    static constexpr int THREADS = (kFirstBuild + kBuildWarps + (FP8 ? kConvWarps : NMMA - 1)) * 32;
     // one CTA per SM with a deep ring: a stage stays in the ring from its load until its UMMAs
     // complete, and about 128 KB per SM must be on the way from HBM at any time for it to run at
     // its rate at the latency it has under that load
@@ -92,9 +100,9 @@ struct DecCfg {
     static constexpr int B_STAGE = MP * 128;                    // [MP rows x 64] bf16
     // sketch stages in the ring (the build warps run ahead of the UMMAs); FP8 three, each also
     // holding a bf16 A stage in TMEM
-    static constexpr int NBS = (FP8 || MP == 64) ? 3 : 4;
+    static constexpr int NBS = FP8 ? 3 : 4;
     static constexpr int OFF_W = 0;
-    static constexpr int OFF_B = kWRing;
+    static constexpr int OFF_B = NW * W_STAGE;
     static constexpr int OFF_X = OFF_B + NBS * B_STAGE;
     static constexpr int X_BYTES = MP == kXChunkRows ? 2 * kXUnitBytes : kXBytes;   // the ring, or the range
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
@@ -102,12 +110,15 @@ struct DecCfg {
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     // accumulator MP columns; FP8: plus NBS bf16 A stages of 32 columns from A_COL
     static constexpr int A_COL = MP <= 32 ? 32 : 64;
-    static constexpr uint32_t TMEM_COLS = FP8 ? (MP <= 32 ? 128 : 256) : (MP <= 32 ? 32 : 64);
+    static constexpr uint32_t TMEM_COLS = FP8 ? (MP <= 32 ? 128 : 256) : (uint32_t)(NMMA * MP < 32 ? 32 : NMMA * MP);
     static_assert(MP % 16 == 0 && MP >= 16 && MP <= 64, "UMMA N for M = 128");
     static_assert(B_STAGE % 1024 == 0 && OFF_B % 1024 == 0, "swizzle atoms stay aligned");
     static_assert(!FP8 || (A_COL >= MP && A_COL + NBS * 32 <= (int)TMEM_COLS), "TMEM layout");
     static_assert(NW <= 31, "the chunk-mode X loader is lane NW of the load warp");
     static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
+    // a ring slot's successive uses go to one UMMA warp, which waits for them in order (a wait on
+    // a barrier's phase parity must never be able to see the phase two uses back)
+    static_assert(NW % NMMA == 0 && NBS % NMMA == 0, "ring depths are multiples of the UMMA warps");
 };
 
 // Two E4M3 codes (low byte = the even column) -> bf16x2, exactly: every E4M3 value has at most
@@ -207,7 +218,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             ptx::mbar_init(&b_full[i], kBuildWarps / 2 + (FP8 ? kConvWarps : 0));
             ptx::mbar_init(&b_empty[i], 1);
         }
-        ptx::mbar_init(acc_full, 1);
+        ptx::mbar_init(acc_full, F::NMMA);
         for (int i = 0; i < 2; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -294,13 +305,17 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             volatile int no_abort = 0;
             ptx::mbar_wait(&x_full[0], 0, &no_abort, kWaitNs);
         }
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma || (F::NMMA > 1 && warp >= kWarpMma2 && warp < kWarpMma2 + F::NMMA - 1)) {
         // ------------------------------------------------------------------ UMMAs
+        // UMMA warp w (w < NMMA) takes stages g = w, w + NMMA, ... into accumulator w (MP columns
+        // from w * MP).
+        const int w = warp == kWarpMma ? 0 : warp - kWarpMma2 + 1;
+        const uint32_t dacc = tm + (uint32_t)(w * MP);
         constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, MP);
         const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, 1024, ptx::kLayoutSW128);
         const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, ptx::kLayoutSW128);
         bool ok = true;
-        for (int g = 0; g < G && ok; ++g) {
+        for (int g = w; g < G && ok; g += F::NMMA) {
             const int ws_ = g % kNW, bs = g % kNB;
             if ((!FP8 && !warp_wait_spin(&w_full[ws_], (uint32_t)((g / kNW) & 1), abort_flag)) ||
                 !warp_wait_spin(&b_full[bs], (uint32_t)((g / kNB) & 1), abort_flag)) {
@@ -316,9 +331,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
 #pragma unroll
                 for (int kk = 0; kk < kStageC / 16; ++kk) {
                     if (FP8)
-                        ptx::umma_bf16_ts(tm, at + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_bf16_ts(dacc, at + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc, (g > w || kk > 0) ? 1u : 0u);
                     else
-                        ptx::umma_bf16_ss(tm, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_bf16_ss(dacc, wd + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (g > w || kk > 0) ? 1u : 0u);
                 }
                 if (!FP8 && g + kNW < G) ptx::umma_commit(&w_empty[ws_]);   // only a slot used again
                 if (g + kNB < G) ptx::umma_commit(&b_empty[bs]);
@@ -465,6 +480,16 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 ptx::tmem_ld_fence_regs<16>(r);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) d[m0 + i] = __uint_as_float(r[i]);
+#pragma unroll
+                for (int a = 1; a < F::NMMA; ++a) {   // plus the other accumulators, in order
+                    if (a < G) {
+                        ptx::tmem_ld_32x32b_x16(tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * MP + m0), r);
+                        ptx::tmem_ld_wait();
+                        ptx::tmem_ld_fence_regs<16>(r);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) d[m0 + i] += __uint_as_float(r[i]);
+                    }
+                }
             }
             if (splits == 1) {
                 const float sc = FP8 ? scale[n] : 1.0f;
