@@ -22,8 +22,8 @@
 //                stages, warps 4-5 the odd ones), gathering from shared memory: the CTA's X
 //                columns copied in once; or, for up to 16 rows whose columns do not fit, the X
 //                rows of each unit (one K-chunk of whole stages, or one stage of whole K-chunks)
-//                by TMA (one more lane of warp 0) into a two-unit ring; else the gathers go to
-//                L1 / L2. Then the epilogue.
+//                by TMA (one more lane of warp 0) into a ring of up to eight units; else the
+//                gathers go to L1 / L2. Then the epilogue.
 // Before the dependency wait of a programmatic dependent launch the CTA asks L2 for its X
 // columns and its first Wc stages.
 // Epilogue: TMEM -> D[n, m]. One split: Y[m, n] = bf16(D[n, m]). Several: the K-splits of one
@@ -57,6 +57,7 @@ constexpr int kNmmaBf16 = 2;              // bf16 UMMA warps
 constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input range, or the chunk ring
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
+constexpr int kMaxXUnits = 8;             // chunk mode: X units in flight at most
 constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
 constexpr int kFirstConv = kFirstBuild + kBuildWarps, kConvWarps = 4;   // FP8 weights: the converter warps
 constexpr int kWarpMma2 = kFirstBuild + kBuildWarps;   // bf16: the further UMMA warps, from here
@@ -104,9 +105,10 @@ struct DecCfg {
     static constexpr int OFF_W = 0;
     static constexpr int OFF_B = NW * W_STAGE;
     static constexpr int OFF_X = OFF_B + NBS * B_STAGE;
-    static constexpr int X_BYTES = MP == kXChunkRows ? 2 * kXUnitBytes : kXBytes;   // the ring, or the range
+    // X: for up to 16 rows the ring of units (or the CTA's range), else the range
+    static constexpr int X_BYTES = MP == kXChunkRows ? (FP8 ? 2 * kXUnitBytes : 80 * 1024) : kXBytes;
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
-    static constexpr int NBAR = 2 * NW + 2 * NBS + 1 + 4;
+    static constexpr int NBAR = 2 * NW + 2 * NBS + 1 + 2 * kMaxXUnits;
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
     // accumulator MP columns; FP8: plus NBS bf16 A stages of 32 columns from A_COL
     static constexpr int A_COL = MP <= 32 ? 32 : 64;
@@ -174,9 +176,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
     uint64_t* b_full = w_empty + kNW;     // the two build warps (and, FP8, the four converter warps) are done
     uint64_t* b_empty = b_full + kNB;     // the stage's UMMAs have completed (its B stage and A stage are free)
     uint64_t* acc_full = b_empty + kNB;
-    uint64_t* x_full = acc_full + 1;      // [2] chunk mode: an X chunk has landed
-    uint64_t* x_empty = x_full + 2;       // [2] chunk mode: every stage of the chunk has been built
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_empty + 2);
+    uint64_t* x_full = acc_full + 1;      // [kMaxXUnits] chunk mode: an X unit has landed
+    uint64_t* x_empty = x_full + kMaxXUnits;   // [kMaxXUnits] chunk mode: every stage of the unit has been built
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_empty + kMaxXUnits);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -206,6 +208,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
     const int kc_hi = (min(st1 * kStageC, Kc) - 1) / S;
     const int R = (kc_hi - kc_lo + 1) * BKc;   // inputs of the range
     const bool staged = !chunked && BKc % 8 == 0 && (int64_t)M * R * 2 <= F::X_BYTES;   // 16-byte aligned rows
+    // chunk mode: X units [16 rows x ui] in flight, as many as the X region holds (at most kMaxXUnits)
+    const int xub = kXChunkRows * ui * 2;
+    const int nxu = chunked ? min(kMaxXUnits, F::X_BYTES / xub) : 1;
 
     // sketch stages start zeroed: rows past M are never written afterwards
     for (int i = threadIdx.x; i < kNB * F::B_STAGE / 16; i += kThreads)
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             ptx::mbar_init(&b_empty[i], 1);
         }
         ptx::mbar_init(acc_full, F::NMMA);
-        for (int i = 0; i < 2; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
+        for (int i = 0; i < kMaxXUnits; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -279,26 +284,26 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                     ptx::mbar_wait(&w_full[g % kNW], (uint32_t)((g / kNW) & 1), &no_abort, kWaitNs);
             }
         } else if (lane == kNW && chunked) {
-            // X units [16 rows x ui] (rows past M read as zero) into a ring of two, as boxes of
+            // X units [16 rows x ui] (rows past M read as zero) into a ring of nxu, as boxes of
             // [16 x bi] stored one after another
             const int nun = G / spc, un0 = st0 / spc;
             int issued = 0;
             for (int u = 0; u < nun; ++u) {
-                const int xs = u & 1;
-                if (u >= 2 && !ptx::mbar_wait(&x_empty[xs], (uint32_t)(((u >> 1) - 1) & 1), abort_flag, kWaitNs)) {
+                const int xs = u % nxu;
+                if (u >= nxu && !ptx::mbar_wait(&x_empty[xs], (uint32_t)(((u / nxu) - 1) & 1), abort_flag, kWaitNs)) {
                     report(status, abort_flag, 5);
                     break;
                 }
-                ptx::mbar_arrive_expect_tx(&x_full[xs], (uint32_t)(kXChunkRows * ui * 2));
+                ptx::mbar_arrive_expect_tx(&x_full[xs], (uint32_t)xub);
                 for (int b = 0; b < ui / bi; ++b)
-                    ptx::tma_load_2d(smem + F::OFF_X + xs * kXUnitBytes + b * (kXChunkRows * bi * 2), &tmap_x,
+                    ptx::tma_load_2d(smem + F::OFF_X + xs * xub + b * (kXChunkRows * bi * 2), &tmap_x,
                                      &x_full[xs], (un0 + u) * ui + b * bi, 0);
                 ++issued;
             }
             if (*abort_flag) {
                 volatile int no_abort = 0;
-                for (int u = issued > 2 ? issued - 2 : 0; u < issued; ++u)
-                    ptx::mbar_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), &no_abort, kWaitNs);
+                for (int u = issued > nxu ? issued - nxu : 0; u < issued; ++u)
+                    ptx::mbar_wait(&x_full[u % nxu], (uint32_t)((u / nxu) & 1), &no_abort, kWaitNs);
             }
         }
         if (staged && lane == 0 && *abort_flag) {   // the X copies land before exit
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             uint8_t* stage = bring + bs * F::B_STAGE;
             const int j = (st0 + g) * kStageC + kl;   // compressed column
             const int u = chunked ? g / spc : 0;      // chunk mode: the stage's unit in this CTA
-            if (chunked && !warp_wait(&x_full[u & 1], (uint32_t)((u >> 1) & 1), abort_flag)) {
+            if (chunked && !warp_wait(&x_full[u % nxu], (uint32_t)((u / nxu) & 1), abort_flag)) {
                 if (lane == 0) report(status, abort_flag, 6);
                 ok = false;
                 break;
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 const int kc = j / S;   // the column's K-chunk
                 // chunk mode: the chunk's inputs start at ii0 within its unit, inside one box
                 const int ii0 = chunked ? kc * BK - (st0 / spc + u) * ui : 0;
-                const __nv_bfloat16* xk = chunked  ? xsm + (size_t)(u & 1) * (kXUnitBytes / 2) +
+                const __nv_bfloat16* xk = chunked  ? xsm + (size_t)(u % nxu) * (xub / 2) +
                                                          (size_t)(ii0 / bi) * (kXChunkRows * bi) + (ii0 % bi)
                                           : staged ? xsm + (size_t)(kc - kc_lo) * BK
                                                    : X + (size_t)kc * BK;
@@ -463,7 +468,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(&b_full[bs]);
-                if (chunked) ptx::mbar_arrive(&x_empty[u & 1]);   // this stage's reads of the unit are done
+                if (chunked) ptx::mbar_arrive(&x_empty[u % nxu]);   // this stage's reads of the unit are done
             }
         }
         // epilogue: warp (quad) holds neurons nb * 128 + quad * 32 + lane
