@@ -88,11 +88,18 @@ struct Cfg {
     static constexpr int W_NB = kNeu * S * 2;            // one N-block's Wc chunk
     static constexpr int W_STAGE = Q * W_NB;
     static constexpr int NP = 2 * SU;                    // sketch panels: two segments
-    static constexpr int NW = 2;
     static constexpr int NBW = SU * Q;                   // build warps in use: one per (unit, N-block)
     static constexpr int EPI = kEpiWarps * 2 * kEpiBox;
     static constexpr int CLR = 0;
-    static constexpr int FIXED = NP * P_UNIT + NW * W_STAGE + EPI + CLR;
+    // The Wc ring holds two chunks, or, where that frees room for one more X box, three half
+    // chunks (a chunk's Wc panels in two halves, WH = 2): NWS slots of WU bytes, WH per chunk.
+    static constexpr int WPAN = Q * ((S + 63) / 64);     // Wc panels per chunk
+    static constexpr int NX_WHOLE = (kSmemBudget - NP * P_UNIT - 2 * W_STAGE - EPI - CLR) / kXUnit;
+    static constexpr int NX_HALF = (kSmemBudget - NP * P_UNIT - 3 * (W_STAGE / 2) - EPI - CLR) / kXUnit;
+    static constexpr int WH = (WPAN % 2 == 0 && NX_WHOLE < 2 * U + 1 && NX_HALF > NX_WHOLE) ? 2 : 1;
+    static constexpr int WU = W_STAGE / WH;
+    static constexpr int NW = WH == 2 ? 3 : 2;           // Wc ring slots
+    static constexpr int FIXED = NP * P_UNIT + NW * WU + EPI + CLR;
     static constexpr int NX_FIT = (kSmemBudget - FIXED) / kXUnit;
     static constexpr int NX = NX_FIT < 2 * U + 1 ? NX_FIT : 2 * U + 1;
     // TMEM columns: Q accumulators (x NACC buffers), two fp32 sketch buffers D_s (QS columns each)
@@ -108,7 +115,7 @@ struct Cfg {
     static constexpr int OFF_X = 0;
     static constexpr int OFF_P = OFF_X + NX * kXUnit;
     static constexpr int OFF_W = OFF_P + NP * P_UNIT;
-    static constexpr int OFF_E = OFF_W + NW * W_STAGE;
+    static constexpr int OFF_E = OFF_W + NW * WU;
     static constexpr int OFF_TAB = OFF_E + EPI;
     static constexpr int OFF_CLR = OFF_TAB;
     static constexpr int OFF_BAR = OFF_CLR + CLR;
@@ -119,7 +126,9 @@ struct Cfg {
     static_assert(QS % 32 == 0 && QS <= 256 && HW % 16 == 0, "sketch UMMA N and conversion halves");
     static_assert(DS_COL + 2 * QS + (SEP ? QS : 0) <= 512, "TMEM budget");
     static_assert(NX >= 2 * SU && SMEM <= 227 * 1024, "shared memory budget: X ring holds two segments");
-    static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0, "swizzle atoms stay aligned");
+    static_assert(W_PANEL % 1024 == 0 && P_UNIT % 1024 == 0 && OFF_E % 1024 == 0 && WU % 1024 == 0,
+                  "swizzle atoms stay aligned");
+    static_assert(WH == 1 || W_NB == ((S + 63) / 64) * W_PANEL, "a chunk's panels lie back to back");
     static_assert(NBW <= kMaxBuildWarps, "build warps");
     // the X loader's first wait for segment g comes before the boxes of segment g + 4 are all
     // issued, so that segment (the same barrier, one phase later) cannot have completed yet
@@ -412,22 +421,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
             Ring wr(NW);
             int nw = 0;
             bool ok = true;
+            constexpr int PN = (S + 63) / 64, PPU = F::WPAN / F::WH;   // panels per N-block, per slot
             for (int t = 0; t < my_tiles && ok; ++t) {
                 const TileInfo ti = tile_info<Q, CHAIN>(p, t);
                 const int nb0 = ti.nb0;
                 const CUtensorMap* tw = &p.layer[ti.l].tw;
                 for (int kc = 0; kc < ti.KC && ok; ++kc) {
-                    if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, wait_ns)) { ok = false; report(status, abort_flag, 2); break; }
-                    ptx::mbar_arrive_expect_tx(&w_full[wr.slot], F::W_STAGE);
-                    uint8_t* wdst = wring + wr.slot * F::W_STAGE;
+                    if constexpr (F::WH == 1) {
+                        if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, wait_ns)) { ok = false; report(status, abort_flag, 2); break; }
+                        ptx::mbar_arrive_expect_tx(&w_full[wr.slot], F::W_STAGE);
+                        uint8_t* wdst = wring + wr.slot * F::W_STAGE;
 #pragma unroll
-                    for (int j = 0; j < Q; ++j)
+                        for (int j = 0; j < Q; ++j)
 #pragma unroll
-                        for (int pn = 0; pn < (S + 63) / 64; ++pn)
-                            ptx::tma_load_2d(wdst + j * F::W_NB + pn * F::W_PANEL, tw, &w_full[wr.slot], kc * S + pn * 64,
-                                             (nb0 + j) * kNeu);
-                    wr.next();
-                    ++nw;
+                            for (int pn = 0; pn < PN; ++pn)
+                                ptx::tma_load_2d(wdst + j * F::W_NB + pn * F::W_PANEL, tw, &w_full[wr.slot], kc * S + pn * 64,
+                                                 (nb0 + j) * kNeu);
+                        wr.next();
+                        ++nw;
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < F::WH; ++h) {   // slot h of the chunk: panels h*PPU .. +PPU
+                            if (!ptx::mbar_wait(&w_empty[wr.slot], wr.phase ^ 1u, abort_flag, wait_ns)) { ok = false; report(status, abort_flag, 2); break; }
+                            ptx::mbar_arrive_expect_tx(&w_full[wr.slot], F::WU);
+                            uint8_t* wdst = wring + wr.slot * F::WU;
+#pragma unroll
+                            for (int q = 0; q < PPU; ++q) {
+                                const int pnl = h * PPU + q, j = pnl / PN, pn = pnl % PN;
+                                ptx::tma_load_2d(wdst + q * F::W_PANEL, tw, &w_full[wr.slot], kc * S + pn * 64, (nb0 + j) * kNeu);
+                            }
+                            wr.next();
+                            ++nw;
+                        }
+                    }
                 }
             }
             if (*abort_flag) drain_ring(w_full, NW, nw, NW);
@@ -500,7 +526,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
             const uint32_t xs = tm + (uint32_t)(F::SEP ? F::XS_COL + b * (QS / 2) : F::DS_COL + b * QS);
             const uint32_t acc_par = (uint32_t)(((t / NACC) & 1) ^ 1);   // n-th use of buffer a waits use n-1
             const uint32_t acc = tm + (uint32_t)(a * F::ACC_COLS);
-            const uint64_t wd = wdesc0 + (uint64_t)((wr.slot * F::W_STAGE) >> 4);
+            // the chunk's Wc slots (WH of them, in ring order from wr) and their descriptors
+            int wslot[2] = {wr.slot, wr.slot};
+            if constexpr (F::WH == 2) {
+                Ring wr1 = wr;
+                wr1.next();
+                wslot[1] = wr1.slot;
+            }
+            const uint64_t wdb[2] = {wdesc0 + (uint64_t)((wslot[0] * F::WU) >> 4),
+                                     F::WH == 2 ? wdesc0 + (uint64_t)((wslot[1] * F::WU) >> 4) : 0ull};
             bool stalled = false;
             if (leader) {
 #pragma unroll
@@ -519,20 +553,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
                         constexpr int per_panel = F::RB / 2;   // slots per Wc panel row
                         const uint32_t off = (uint32_t)(j * F::W_NB + ((kk * 16) / per_panel) * F::W_PANEL +
                                                         ((kk * 16) % per_panel) * 2);
+                        const int h = F::WH == 1 ? 0 : (int)(off / F::WU);   // which of the chunk's slots
+                        const uint64_t wd = wdb[h] + (uint64_t)((off - (uint32_t)(h * F::WU)) >> 4);
                         // slots s0 .. s0+15 in bf16: SEP, column s0 / 2 of Xs[b]; in place, inside
                         // the converting warp's half of D_s[b]
                         const int s0 = j * S + kk * 16;
                         const uint32_t acol = F::SEP ? (uint32_t)(s0 / 2) : (uint32_t)((s0 / HW) * HW + (s0 % HW) / 2);
-                        ptx::umma_bf16_ts(acc + (uint32_t)(j * kNeu), xs + acol, wd + (uint64_t)(off >> 4), idesc_m,
-                                          (kc > 0 || kk > 0) ? 1u : 0u);
+                        ptx::umma_bf16_ts(acc + (uint32_t)(j * kNeu), xs + acol, wd, idesc_m, (kc > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                ptx::umma_commit(&w_empty[wr.slot]);
+#pragma unroll
+                for (int h = 0; h < F::WH; ++h) ptx::umma_commit(&w_empty[wslot[h]]);
                 ptx::umma_commit(F::SEP ? &xs_free[b] : &ds_free[b]);
                 if (kc == KC - 1) ptx::umma_commit(&acc_full[a]);
             }
             if (__shfl_sync(0xffffffffu, stalled ? 1 : 0, 0)) break;
-            wr.next();
+#pragma unroll
+            for (int h = 0; h < F::WH; ++h) wr.next();
             if (++kc == KC) {
                 kc = 0;
                 if (++t < my_tiles) KC = tile_info<Q, CHAIN>(p, t).KC;
@@ -652,14 +689,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
             for (int c = 0; c < HW / 2; c += 8) ptx::tmem_st_32x32b_x8(dst + (uint32_t)c, r + c);
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
-            // the first convert warp also waits for the chunk's Wc
-            if (warp == kFirstConv && !warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag, wait_ns)) {
+            // the first convert warp also waits for the chunk's Wc (its WH slots)
+            bool w_ok = true;
+            if constexpr (F::WH == 1) {
+                w_ok = warp != kFirstConv || warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag, wait_ns);
+                wr.next();
+            } else {
+#pragma unroll
+                for (int h = 0; h < F::WH; ++h) {
+                    if (warp == kFirstConv && w_ok && !warp_wait_spin(&w_full[wr.slot], wr.phase, abort_flag, wait_ns)) w_ok = false;
+                    wr.next();
+                }
+            }
+            if (!w_ok) {
                 if (lane == 0) report(status, abort_flag, 9);
                 break;
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&mm_ready[b]);
-            wr.next();
         }
     } else if (warp >= kFirstEpi && warp < kFirstEpi + kEpiWarps) {
         // ------------------------------------------------------------------ epilogue
