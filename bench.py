@@ -557,33 +557,35 @@ def run_reference(args, layers, wid, rank, world):
     if rank != 0:
         return
     cfg = workload_config(layers, wid, world)
-    prepared = prepare_oracle(layers, max_rows=2048)
+    prepared = prepare_oracle(layers, max_rows=4096)
     threads = oracle_threads()
-    rows = None
-    # each step a bounded sample, so that the whole run stays within a few minutes
-    budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        _, _, rows = oracle_sample_rate(prepared, budget, rows)
-    # every step repeats the sample until it has run for about `budget`; the rate is the dense
-    # work of all those passes over their time (oracle_sample_rate's own figure)
+    n = len(prepared)
+    # Step s times layer s mod n of the workload with all its prepared rows: the same rows the
+    # cpu_baseline leg times, so the rate is the same quantity (the oracle's cost per row falls
+    # as rows are added, its per-layer expansion of W_full being fixed), and each step stays
+    # bounded (one layer pass) whatever K and W are.
+    all_rows = 1 << 30
+    for w in range(args.warmup):
+        _oracle_pass([prepared[w % n]], all_rows)
     work, secs = 0.0, 0.0
-    for _ in range(args.steps):
-        rate, dt, rows = oracle_sample_rate(prepared, budget, rows)
-        work += rate * 1e12 * dt
-        secs += dt
+    for s in range(args.steps):
+        d, t = _oracle_pass([prepared[s % n]], all_rows)
+        work += d
+        secs += t
     value = work / secs / 1e12
     step_ms = secs / args.steps * 1e3
     full_ms = sum(2.0 * L.M * L.N * L.K for L in layers) / (value * 1e12) * 1e3
+    rows = max(p[1].shape[0] for p in prepared)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
         "full_step_ms_extrapolated": full_ms,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"first {rows} rows of each layer, repeated for about {budget:.2f} s per step "
-                                   f"(float64 definition, numpy BLAS); ms_per_step is the timed sample per step, "
-                                   f"full_step_ms_extrapolated the whole workload at the same rate (rows are "
-                                   f"independent)"},
+                         "sample": f"step s: layer s mod {n} of the workload, its first {rows} rows (all rows up "
+                                   f"to 4096; float64 definition, numpy BLAS); ms_per_step is that pass, "
+                                   f"full_step_ms_extrapolated the whole workload at the measured rate (rows "
+                                   f"are independent)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -14,7 +14,8 @@
 // Tile: 128 rows of X (UMMA M) x Q N-blocks (Q = 2 for most shapes); one persistent CTA per SM
 // takes tiles N-block-pair fastest. Per K-chunk:
 //   * X-load warp  : X[m0:+128, chunk] as [128 x 64] TMA boxes (128B swizzle) into a ring.
-//   * W-load warp  : the Q N-blocks' Wc[nb*128:+128, kc*S:+S] as TMA boxes into a 2-stage ring.
+//   * W-load warp  : the Q N-blocks' Wc[nb*128:+128, kc*S:+S] as TMA boxes into a ring of two
+//                    chunks, or of three half chunks where that leaves room for one more X box.
 //   * build warps  : one per (64-input unit, N-block) of a sketch segment (up to four). Each
 //                    writes its unit's non-zeros into the stacked [Q*S x 64] K-major panel of
 //                    the B operand (two entries per lane) and clears the previous use's entries,

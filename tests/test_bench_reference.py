@@ -1,8 +1,8 @@
 """The benchmark's reference arm (the CPU oracle timed on the host cores), on CPU.
 
 Its value must be the oracle's own measured rate: the dense work of every timed pass over
-the time of those passes. A fixed fake rate pins the arithmetic exactly; a short real run
-checks that the arm and the cpu_baseline leg's measurement agree.
+the time of those passes, on the same rows as the cpu_baseline leg. A fake pass pins the
+arithmetic exactly; a short real run checks that the arm and the cpu_baseline leg agree.
 """
 
 import argparse
@@ -23,22 +23,23 @@ def _run_reference(layers, steps=2, warmup=1):
 
 
 def test_reference_value_is_the_sample_rate(monkeypatch):
-    """Each step repeats its sample for ~budget seconds; the arm must report the rate those
-    repeats ran at, not one pass's work over all of their time."""
+    """Each step is one layer's pass; the arm must report the dense work of the timed passes
+    over their time, and time one layer per step in rotation."""
     calls = []
 
-    def fake_rate(prepared, budget, rows=None):
-        calls.append(budget)
-        return 0.125, 2.0, 32          # TFLOP/s over 2 s of repeated passes of 32 rows
+    def fake_pass(prepared, rows):
+        calls.append(prepared[0][0])
+        return 0.25e12, 2.0           # 0.25 TFLOP of dense work in 2 s
 
-    monkeypatch.setattr(bench, "oracle_sample_rate", fake_rate)
-    line = _run_reference([WORKLOADS[1][0]], steps=3, warmup=1)
+    monkeypatch.setattr(bench, "_oracle_pass", fake_pass)
+    layers = WORKLOADS[2]
+    line = _run_reference(layers, steps=3, warmup=1)
     assert line["impl"] == "reference"
     assert abs(line["value"] - 0.125) < 1e-12
     assert abs(line["cpu_baseline"]["value"] - 0.125) < 1e-12
-    assert abs(line["ms_per_step"] - 2000.0) < 1e-9        # the timed sample per step
+    assert abs(line["ms_per_step"] - 2000.0) < 1e-9        # the timed pass per step
     assert line["e2e"]["value"] == line["value"]
-    assert len(calls) == 4
+    assert calls == [layers[0], layers[0], layers[1], layers[2]]   # warm-up, then steps 0, 1, 2
 
 
 def test_reference_arm_agrees_with_cpu_baseline_rate():
