@@ -479,7 +479,7 @@ def run_backward(args, layers, wid, peaks, peak_src, dev):
 
 
 def run_chain(args, layers, wid, peaks, peak_src, dev):
-    """The DLRM top-MLP chain of the sweep workload (1024 -> 1024 -> 512 -> 256 at M = 65536, c = 2):
+    """The DLRM top-MLP chain of the sweep workload (1024 -> 1024 -> 512 -> 256 at M = 65536, or --m, c = 2):
     bias + ReLU after the first two layers, one ss1_chain_forward per step (one persistent launch
     when the layers allow it), against the same layers as three ss1_forward_ex calls. L2 flushed
     before every step; CUDA events around the chain."""
@@ -487,6 +487,8 @@ def run_chain(args, layers, wid, peaks, peak_src, dev):
     from structured_compressed_linear_b200 import ss1
     from structured_compressed_linear_b200.workloads import WORKLOADS, make_inputs
     chain = [L for L in WORKLOADS[5] if L.workload == "dlrm-top-mlp"]
+    if args.m:
+        chain = [L.with_M(args.m) for L in chain]
     X, _ = make_inputs(chain[0])
     lays, Wcs, bs = [], [], []
     gen = torch.Generator().manual_seed(5)
@@ -660,7 +662,10 @@ def main():
         run_decode_block(args, peaks, peak_src, torch.device("cuda", local))
         return
 
-    wid, layers = select_layers(args.workload, args.m, args.only)
+    if args.op == "chain":   # the MLP chain at its own row count (--m overrides it)
+        wid, layers = 5, []
+    else:
+        wid, layers = select_layers(args.workload, args.m, args.only)
 
     if args.op in ("project", "backward", "chain"):   # one GPU: projection, backward, or the MLP chain
         if rank != 0:
