@@ -15,14 +15,14 @@
 // N-block of the neuron, scaled by 1 / c. The work is a gather: each output reads c inputs of
 // its row. The kernel is bound by HBM (W read once, Wc written once).
 //
-// Fast kernel: a CTA takes a tile of R rows of one N-block x one K-chunk at a time.
-//   * load : W[rows, chunk] with 16-byte loads into shared memory, transposed so that one
-//            32-bit word holds the same input of two rows (bf16) or of one row (fp32); the
-//            word pitch is 1 mod 32, so the gathers below are free of bank conflicts.
-//   * gather: lane = row pair (bf16) or row (fp32); warp w takes slots w, w + 8, ...; every
-//            lane reads the slot's c sources (the same inputs for all rows of the N-block)
-//            and sums them in fp32, times 1 / c, rounded once to the output type.
-//   * store: the tile's outputs go through a slot-major staging buffer to 16-byte stores.
+// The work is one (N-block, K-chunk) of W at a time: the chunk's table of sources is the same for
+// all BN rows of the N-block, so a CTA reads it once and keeps it in registers, and each warp
+// streams rows of W through its own small shared-memory buffer, gathering from it.
+//   * fp32: the row kernel, one row per buffer fill.
+//   * bf16: the pair kernel, two rows interleaved per buffer fill (one 32-bit word holds the
+//     same input of both rows), so each shared-memory load serves two outputs.
+// Each output sums its c terms pairwise in fp32, times the factor, rounded once to the output
+// type; the order of the sum is the same in both kernels.
 // Shapes whose rows or chunks are not 16-byte multiples take a plain kernel: one thread per
 // output, reading its c inputs from global memory.
 #include "ss1_internal.cuh"
@@ -35,167 +35,186 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
-// Word pitch of the transposed tile: >= BK and 1 mod 32.
-__host__ __device__ constexpr int tile_pitch(int BK) { return ((BK + 31) / 32) * 32 + 1; }
+// Row kernel: a CTA takes one (N-block, K-chunk, row range) and its 8 warps take the range's
+// rows in turn. The chunk's table (BK entries, slot-major) is read once per CTA: lane l keeps the
+// sources of its slots l, l + 32, ... (S * C = BK <= 256, so at most 8 entries). Per row, a warp
+// reads the row's chunk (BK elements) with 16-byte loads, kRowsAhead of its rows ahead of the one
+// it gathers (4 KB in flight per warp), stores it into its own shared-memory row buffer, and
+// each lane sums its slots' C signed terms (pairwise), scales and writes them: 32
+// consecutive outputs per store instruction. The N-block's rows are split over several CTAs when
+// the (N-block, K-chunk) pairs alone would leave SMs idle.
 
-template <bool BF16>
-struct Elem;
-template <>
-struct Elem<true> {
-    using T = __nv_bfloat16;
-    static constexpr int kPerVec = 8;      // elements per 16-byte vector
-    static constexpr int kRowsPerWord = 2;
-};
-template <>
-struct Elem<false> {
-    using T = float;
-    static constexpr int kPerVec = 4;
-    static constexpr int kRowsPerWord = 1;
-};
-
-__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
-    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&b);
-}
-
-// Shared memory of one CTA (in 32-bit words): the transposed tile [R / rows-per-word][pitch],
-// the staging buffer [S][R / rows-per-word + 1] and the chunk's slot-major table (BK entries).
-template <bool BF16>
-__host__ __device__ constexpr size_t smem_words(int R, int BK, int S) {
-    const int units = R / Elem<BF16>::kRowsPerWord;
-    return (size_t)units * tile_pitch(BK) + (size_t)S * (units + 1) + (size_t)(BK + 1) / 2;
-}
-
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
-    project_kernel(const typename Elem<BF16>::T* __restrict__ W, typename Elem<BF16>::T* __restrict__ Wc,
-                   const uint16_t* __restrict__ src_tab, int K, int BK, int BN, int c, int R, int KC,
-                   int64_t units_total, float scale) {
-    using E = Elem<BF16>;
-    using T = typename E::T;
-    constexpr int RPW = E::kRowsPerWord;
-    extern __shared__ uint32_t sm[];
-    const int S = BK / c;
-    const int Kc = K / c;
-    const int units = R / RPW;                 // row units (pairs for bf16, rows for fp32) per tile
-    const int pitch = tile_pitch(BK);
-    uint32_t* tile = sm;
-    uint32_t* stage = tile + (size_t)units * pitch;
-    const int spitch = units + 1;
-    uint16_t* tab = reinterpret_cast<uint16_t*>(stage + (size_t)S * spitch);
+template <typename T, int C>
+__global__ void __launch_bounds__(kThreads, 3)
+    project_rows_kernel(const T* __restrict__ W, T* __restrict__ Wc, const uint16_t* __restrict__ src_tab, int K,
+                        int BK, int BN, int KC, int rows_per_cta, float scale) {
+    constexpr int E = (int)sizeof(T);
+    constexpr int kMaxVec = 256 * E / 512;                  // 16-byte vectors per lane of a 256-input row
+    constexpr int kRowsAhead = 8 / kMaxVec;
+    constexpr int kSlots = 8 / C;                           // slots per lane at most (S <= 256 / C)
+    __shared__ __align__(16) uint8_t rowbuf[kWarps][256 * E];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int vecs = BK / E::kPerVec;          // 16-byte vectors per row of the chunk
-
-    // The next unit's W tile and table entries are loaded into registers while this unit is
-    // gathered and stored (at most 8 16-byte vectors per thread: 32 row pairs x 32 vectors of
-    // bf16, or 32 rows x 64 vectors of fp32, over 256 threads).
-    constexpr int kIters = BF16 ? 4 : 8;
-    uint4 ld[8];
-    uint16_t tab_next = 0;
-    auto fetch = [&](int64_t u) {
-        if (u >= units_total) return;
-        const int kc = (int)(u % KC);
-        const int64_t n0 = (u / KC) * R;
-        const int nb = (int)(n0 / BN);
-        if ((int)threadIdx.x < BK) tab_next = src_tab[((size_t)nb * KC + kc) * BK + threadIdx.x];
+    const int kc = blockIdx.x, nb = blockIdx.y;
+    const int S = BK / C, Kc = K / C;
+    const int nvec = BK * E / 16;                           // 16-byte vectors in a row's chunk
+    uint16_t ent[kSlots * C];                               // slot lane + 32 k, term j: ent[k * C + j]
+    const uint16_t* tab = src_tab + ((size_t)nb * KC + kc) * BK;
 #pragma unroll
-        for (int it = 0; it < kIters; ++it) {
-            const int i = threadIdx.x + it * kThreads;
-            if (i < units * vecs) {
-                const int p = i % units, q = i / units;     // lanes take consecutive row units
-                if (BF16) {
-                    const T* r0 = W + (size_t)(n0 + 2 * p) * K + (size_t)kc * BK + q * 8;
-                    ld[2 * it] = __ldg(reinterpret_cast<const uint4*>(r0));
-                    ld[2 * it + 1] = __ldg(reinterpret_cast<const uint4*>(r0 + K));
-                } else {
-                    ld[it] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)(n0 + p) * K + (size_t)kc * BK + q * 4));
-                }
+    for (int k = 0; k < kSlots; ++k)
+#pragma unroll
+        for (int j = 0; j < C; ++j) {
+            const int sl = lane + 32 * k;
+            ent[k * C + j] = sl < S ? __ldg(tab + sl * C + j) : (uint16_t)0;
+        }
+    const int r_lo = blockIdx.z * rows_per_cta, r_hi = min(BN, r_lo + rows_per_cta);
+    const T* wrow0 = W + ((size_t)nb * BN + r_lo) * K + (size_t)kc * BK;
+    T* crow0 = Wc + ((size_t)nb * BN + r_lo) * Kc + (size_t)kc * S;
+    const int rows = r_hi - r_lo;
+    uint4 buf[kRowsAhead][kMaxVec];
+    auto load = [&](int r, uint4 (&v)[kMaxVec]) {
+        if (r < rows) {
+#pragma unroll
+            for (int q = 0; q < kMaxVec; ++q) {
+                const int vi = lane + 32 * q;
+                if (vi < nvec) v[q] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + vi);
             }
         }
     };
-    fetch(blockIdx.x);
-    for (int64_t u = blockIdx.x; u < units_total; u += gridDim.x) {
-        const int64_t rt = u / KC;
-        const int kc = (int)(u % KC);
-        const int64_t n0 = rt * R;
-        // ---- the fetched tile into shared memory, transposed; its table entries
-        if ((int)threadIdx.x < BK) tab[threadIdx.x] = tab_next;
 #pragma unroll
-        for (int it = 0; it < kIters; ++it) {
-            const int i = threadIdx.x + it * kThreads;
-            if (i < units * vecs) {
-                const int p = i % units, q = i / units;
-                if (BF16) {
-                    const uint4 a = ld[2 * it], b = ld[2 * it + 1];
-                    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-                    uint32_t* dst = tile + (size_t)p * pitch + q * 8;
+    for (int a = 0; a < kRowsAhead; ++a) load(warp + a * kWarps, buf[a]);
+    uint8_t* rb = rowbuf[warp];
+    const T* x = reinterpret_cast<const T*>(rb);
+    for (int r0 = warp; r0 < rows; r0 += kRowsAhead * kWarps) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        dst[2 * e] = __byte_perm(aw[e], bw[e], 0x5410);       // inputs 2e of rows 2p, 2p+1
-                        dst[2 * e + 1] = __byte_perm(aw[e], bw[e], 0x7632);   // inputs 2e+1
-                    }
-                } else {
-                    uint32_t* dst = tile + (size_t)p * pitch + q * 4;
-                    dst[0] = ld[it].x; dst[1] = ld[it].y; dst[2] = ld[it].z; dst[3] = ld[it].w;
-                }
+        for (int a = 0; a < kRowsAhead; ++a) {
+            const int r = r0 + a * kWarps;
+            if (r >= rows) break;
+#pragma unroll
+            for (int q = 0; q < kMaxVec; ++q) {
+                const int vi = lane + 32 * q;
+                if (vi < nvec) reinterpret_cast<uint4*>(rb)[vi] = buf[a][q];
             }
-        }
-        __syncthreads();
-        fetch(u + gridDim.x);   // in flight during the gather and the stores below
-        // ---- gather: Wc[rows of unit, slot s] = (1/c) sum_j sign_j * W[rows, src_j]
-        if (lane < units) {
-            const uint32_t* row = tile + (size_t)lane * pitch;
-            for (int s = warp; s < S; s += kWarps) {
-                // the c signed terms, summed pairwise (a tree): c equal terms then add up exactly
-                float lo[8], hi[8];
+            load(r + kRowsAhead * kWarps, buf[a]);   // in flight during this row's gather
+            __syncwarp();
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    lo[j] = 0.0f;
-                    hi[j] = 0.0f;
-                    if (j < c) {
-                        const uint16_t e = tab[s * c + j];
-                        const uint32_t w = row[e & kSrcIdxMask];
-                        const bool neg = (e & kSrcNegBit) != 0;
-                        const float a = BF16 ? __uint_as_float(w << 16) : __uint_as_float(w);
-                        lo[j] = neg ? -a : a;
-                        if (BF16) {
-                            const float b = __uint_as_float(w & 0xFFFF0000u);
-                            hi[j] = neg ? -b : b;
+            for (int k = 0; k < kSlots; ++k) {
+                const int sl = lane + 32 * k;
+                if (sl < S) {
+                    float t[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        t[j] = 0.0f;
+                        if (j < C) {
+                            const uint16_t e = ent[k * C + j];
+                            const float v = (float)x[e & kSrcIdxMask];
+                            t[j] = (e & kSrcNegBit) ? -v : v;
                         }
                     }
+#pragma unroll
+                    for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                        for (int j = 0; j < w2; ++j) t[j] += t[j + w2];
+                    crow0[(size_t)r * Kc + sl] = (T)(t[0] * scale);
                 }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+// bf16 pair kernel: the row kernel with two rows (r, r + 8) gathered at once. Their chunks are
+// interleaved in the warp's buffer, one 32-bit word holding input k of both rows, so one
+// shared-memory load serves both rows' terms: half the gathers of the row kernel, which is bound
+// by them. The interleaved store writes, from lanes 0-3 and 4-7 of each quarter warp, the two
+// halves of a lane's 32 bytes in opposite order, so the 8 lanes of a phase cover all 32 banks.
+template <int C>
+__global__ void __launch_bounds__(kThreads, 3)
+    project_pairs_kernel(const __nv_bfloat16* __restrict__ W, __nv_bfloat16* __restrict__ Wc,
+                         const uint16_t* __restrict__ src_tab, int K, int BK, int BN, int KC, int rows_per_cta,
+                         float scale) {
+    constexpr int kPairsAhead = 4;                          // 8 rows of 512 bytes in flight per warp
+    constexpr int kSlots = 8 / C;
+    __shared__ __align__(16) uint32_t pairbuf[kWarps][256];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int kc = blockIdx.x, nb = blockIdx.y;
+    const int S = BK / C, Kc = K / C;
+    const int nvec = BK / 8;                                // 16-byte vectors in a row's chunk
+    uint16_t ent[kSlots * C];
+    const uint16_t* tab = src_tab + ((size_t)nb * KC + kc) * BK;
 #pragma unroll
-                for (int w2 = 4; w2 >= 1; w2 >>= 1)
+    for (int k = 0; k < kSlots; ++k)
 #pragma unroll
-                    for (int j = 0; j < w2; ++j) {
-                        lo[j] += lo[j + w2];
-                        hi[j] += hi[j + w2];
+        for (int j = 0; j < C; ++j) {
+            const int sl = lane + 32 * k;
+            ent[k * C + j] = sl < S ? __ldg(tab + sl * C + j) : (uint16_t)0;
+        }
+    const int r_lo = blockIdx.z * rows_per_cta, r_hi = min(BN, r_lo + rows_per_cta);
+    const __nv_bfloat16* wrow0 = W + ((size_t)nb * BN + r_lo) * K + (size_t)kc * BK;
+    __nv_bfloat16* crow0 = Wc + ((size_t)nb * BN + r_lo) * Kc + (size_t)kc * S;
+    const int rows = r_hi - r_lo;
+    // pair p of this warp: rows warp + 16 p and warp + 16 p + 8
+    uint4 buf[kPairsAhead][2];
+    auto load = [&](int p, uint4 (&v)[2]) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = warp + 16 * p + 8 * i;
+            v[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows && lane < nvec) v[i] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + lane);
+        }
+    };
+#pragma unroll
+    for (int a = 0; a < kPairsAhead; ++a) load(a, buf[a]);
+    uint32_t* pb = pairbuf[warp];
+    const int sw = (lane >> 2) & 1;
+    for (int p0 = 0; warp + 16 * p0 < rows; p0 += kPairsAhead) {
+#pragma unroll
+        for (int a = 0; a < kPairsAhead; ++a) {
+            const int p = p0 + a;
+            const int ra = warp + 16 * p, rb = ra + 8;
+            if (ra >= rows) break;
+            if (lane < nvec) {
+                const uint4 u = buf[a][0], v = buf[a][1];
+                const uint4 lo = make_uint4(__byte_perm(u.x, v.x, 0x5410), __byte_perm(u.x, v.x, 0x7632),
+                                            __byte_perm(u.y, v.y, 0x5410), __byte_perm(u.y, v.y, 0x7632));
+                const uint4 hi = make_uint4(__byte_perm(u.z, v.z, 0x5410), __byte_perm(u.z, v.z, 0x7632),
+                                            __byte_perm(u.w, v.w, 0x5410), __byte_perm(u.w, v.w, 0x7632));
+                uint4* dst = reinterpret_cast<uint4*>(pb) + 2 * lane;
+                dst[sw] = sw ? hi : lo;
+                dst[1 - sw] = sw ? lo : hi;
+            }
+            load(p + kPairsAhead, buf[a]);   // in flight during this pair's gather
+            __syncwarp();
+            const bool second = rb < rows;
+#pragma unroll
+            for (int k = 0; k < kSlots; ++k) {
+                const int sl = lane + 32 * k;
+                if (sl < S) {
+                    float ta[8], tb[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        ta[j] = 0.0f;
+                        tb[j] = 0.0f;
+                        if (j < C) {
+                            const uint16_t e = ent[k * C + j];
+                            const uint32_t w = pb[e & kSrcIdxMask];
+                            const float va = __uint_as_float(w << 16), vb = __uint_as_float(w & 0xFFFF0000u);
+                            ta[j] = (e & kSrcNegBit) ? -va : va;
+                            tb[j] = (e & kSrcNegBit) ? -vb : vb;
+                        }
                     }
-                stage[(size_t)s * spitch + lane] =
-                    BF16 ? pack2_bf16(lo[0] * scale, hi[0] * scale) : __float_as_uint(lo[0] * scale);
-            }
-        }
-        __syncthreads();
-        // ---- store: Wc[n0 + r, kc * S + s .. + kPerVec) as 16-byte vectors; lane = row
-        const int svecs = S / E::kPerVec;
-        for (int i = threadIdx.x; i < R * svecs; i += kThreads) {
-            const int r = i % R, sv = i / R;
-            uint32_t out[4];
-            if (BF16) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t w0 = stage[(size_t)(sv * 8 + 2 * e) * spitch + r / 2];
-                    const uint32_t w1 = stage[(size_t)(sv * 8 + 2 * e + 1) * spitch + r / 2];
-                    out[e] = (r & 1) ? __byte_perm(w0, w1, 0x7632) : __byte_perm(w0, w1, 0x5410);
+                    for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                        for (int j = 0; j < w2; ++j) {
+                            ta[j] += ta[j + w2];
+                            tb[j] += tb[j + w2];
+                        }
+                    crow0[(size_t)ra * Kc + sl] = __float2bfloat16_rn(ta[0] * scale);
+                    if (second) crow0[(size_t)rb * Kc + sl] = __float2bfloat16_rn(tb[0] * scale);
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) out[e] = stage[(size_t)(sv * 4 + e) * spitch + r];
             }
-            *reinterpret_cast<uint4*>(Wc + (size_t)(n0 + r) * Kc + (size_t)kc * S + sv * E::kPerVec) =
-                make_uint4(out[0], out[1], out[2], out[3]);
+            __syncwarp();
         }
-        __syncthreads();
     }
 }
 
@@ -227,27 +246,14 @@ __global__ void project_plain_kernel(const T* __restrict__ W, T* __restrict__ Wc
     Wc[i] = (T)(t[0] * scale);
 }
 
-int pick_rows(int BN, bool bf16) {
-    const int cands_bf16[3] = {64, 32, 16}, cands_f32[2] = {32, 16};
-    if (bf16) {
-        for (int r : cands_bf16)
-            if (BN % r == 0) return r;
-    } else {
-        for (int r : cands_f32)
-            if (BN % r == 0) return r;
-    }
-    return 0;
-}
-
 }  // namespace
 
 bool project_fast_ok(const ss1_layer& L, const void* W, const void* Wc, int dtype) {
+    (void)Wc;
     const int e = dtype == SS1_DTYPE_BF16 ? 2 : 4;
-    const int per_vec = 16 / e;
-    if (pick_rows(L.BN, dtype == SS1_DTYPE_BF16) == 0) return false;
-    if (L.BK % per_vec != 0 || L.S % per_vec != 0) return false;
-    if ((L.K * e) % 16 != 0 || ((L.K / L.c) * e) % 16 != 0) return false;
-    return ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(Wc)) & 15u) == 0;
+    // the row kernel's 16-byte loads: rows and chunks start on 16-byte boundaries
+    if ((L.BK * e) % 16 != 0 || (L.K * e) % 16 != 0) return false;
+    return (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
 }
 
 cudaError_t launch_project(const ss1_layer& L, const void* W, void* Wc, int dtype, float scale, cudaStream_t st) {
@@ -265,25 +271,31 @@ cudaError_t launch_project(const ss1_layer& L, const void* W, void* Wc, int dtyp
                                                                                (int)L.K, L.BK, L.BN, L.c, scale);
         return cudaGetLastError();
     }
-    const int R = pick_rows(L.BN, bf16);
-    const size_t smem = (bf16 ? smem_words<true>(R, L.BK, L.S) : smem_words<false>(R, L.BK, L.S)) * 4;
-    const void* fn = bf16 ? reinterpret_cast<const void*>(&project_kernel<true>)
-                          : reinterpret_cast<const void*>(&project_kernel<false>);
-    // the largest tile (32 row units of a 256-input chunk, 256 slots at c = 1)
-    constexpr int kMaxSmem = (int)(smem_words<true>(64, 256, 256) * 4);
-    static_assert(smem_words<false>(32, 256, 256) * 4 <= (size_t)kMaxSmem, "fp32 tile fits the same limit");
-    if (smem > (size_t)kMaxSmem) return cudaErrorInvalidValue;
-    const cudaError_t ae = smem_attr_once(fn, kMaxSmem);
-    if (ae != cudaSuccess) return ae;
-    const int64_t units = (L.N / R) * L.KC;
-    const int64_t cap = (int64_t)L.num_sms * 8;
-    const int grid = (int)(units < cap ? units : cap);
-    if (bf16)
-        project_kernel<true><<<grid, kThreads, smem, st>>>((const __nv_bfloat16*)W, (__nv_bfloat16*)Wc, L.d_src,
-                                                            (int)L.K, L.BK, L.BN, L.c, R, L.KC, units, scale);
-    else
-        project_kernel<false><<<grid, kThreads, smem, st>>>((const float*)W, (float*)Wc, L.d_src, (int)L.K, L.BK,
-                                                             L.BN, L.c, R, L.KC, units, scale);
+    if (L.KC > 0x7FFFFFFF || L.NB > 65535) return cudaErrorInvalidValue;
+    // split the N-block's rows only while the (N-block, K-chunk) pairs leave SMs idle
+    const int64_t pairs = L.KC * L.NB, want = L.num_sms > 0 ? L.num_sms : 148;
+    int splits = 1;
+    while (splits * 2 <= 64 && pairs * splits < want && L.BN / (splits * 2) >= kWarps) splits *= 2;
+    const int rows_per_cta = (L.BN + splits - 1) / splits;
+    const dim3 grid((unsigned)L.KC, (unsigned)L.NB, (unsigned)splits);
+#define SS1_PROJECT_ROWS(CC)                                                                                   \
+    do {                                                                                                       \
+        if (bf16)                                                                                              \
+            project_pairs_kernel<CC><<<grid, kThreads, 0, st>>>((const __nv_bfloat16*)W, (__nv_bfloat16*)Wc,   \
+                                                                L.d_src, (int)L.K, L.BK, L.BN, L.KC,           \
+                                                                rows_per_cta, scale);                          \
+        else                                                                                                   \
+            project_rows_kernel<float, CC><<<grid, kThreads, 0, st>>>((const float*)W, (float*)Wc, L.d_src,    \
+                                                                      (int)L.K, L.BK, L.BN, L.KC, rows_per_cta, \
+                                                                      scale);                                  \
+    } while (0)
+    switch (L.c) {
+        case 1: SS1_PROJECT_ROWS(1); break;
+        case 2: SS1_PROJECT_ROWS(2); break;
+        case 4: SS1_PROJECT_ROWS(4); break;
+        default: SS1_PROJECT_ROWS(8); break;
+    }
+#undef SS1_PROJECT_ROWS
     return cudaGetLastError();
 }
 
