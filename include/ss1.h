@@ -401,6 +401,31 @@ typedef struct {
 } ss1_launch_info;
 SS1_API int ss1_last_launch(ss1_launch_info* out);
 
+/*
+ * ss1_bounds_check -- the record of the checked (debug) build, libss1_checked.so: the same
+ * sources compiled so that every global-memory access a kernel addresses by its own index
+ * arithmetic first tests its element index against the extent of the buffer (tables, X, Wc, Y,
+ * scales, bias, the backward and projection operands). A failed test skips the access and
+ * records the first failure; TMA tile copies are bounded by their tensor maps in hardware. The
+ * normal build makes no tests and has the same entry point.
+ *   checked : receives 1 in the checked build, 0 in the normal one.
+ *   record  : receives the first failed test on the current device since the last call, 0 if
+ *             none: (site << 48) | (element index mod 2^48), site a small positive number
+ *             naming the access; the record is then cleared. Always 0 in the normal build.
+ * The checked build synchronises the current device first (no other effect on the caller's
+ * work). Host pointers. Errors: INVALID_ARG (NULL), CUDA (checked build only).
+ */
+SS1_API int ss1_bounds_check(int* checked, uint64_t* record);
+
+/*
+ * ss1_test_bounds_check -- the checked build's index test run once on the given values, for
+ * tests of the record itself: one thread on the legacy default stream of the current device
+ * tests `index` against `extent` elements (site 63) and accesses no memory. When the index is
+ * out of range, the next ss1_bounds_check reports (63 << 48) | index. Asynchronous.
+ * Errors: UNSUPPORTED_SHAPE in the normal build (nothing is launched), CUDA.
+ */
+SS1_API int ss1_test_bounds_check(int64_t index, int64_t extent);
+
 #ifdef __cplusplus
 }
 #endif

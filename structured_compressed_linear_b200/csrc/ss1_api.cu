@@ -198,7 +198,30 @@ bool layer_args_ok(int64_t K, int64_t N, int c, int BK, int BN) {
 
 }  // namespace ss1
 
+#if SS1_CHECKED
+namespace ss1 {
+__device__ unsigned long long g_bad_access = 0;
+}
+#endif
+
 extern "C" {
+
+SS1_API int ss1_bounds_check(int* checked, uint64_t* record) {
+    if (!checked || !record) return SS1_ERR_INVALID_ARG;
+    *checked = SS1_CHECKED;
+    *record = 0;
+#if SS1_CHECKED
+    unsigned long long v = 0;
+    const unsigned long long zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&v, ss1::g_bad_access, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(ss1::g_bad_access, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return SS1_ERR_CUDA;
+    }
+    *record = v;
+#endif
+    return SS1_OK;
+}
 
 SS1_API int ss1_last_launch(ss1_launch_info* out) {
     if (!out) return SS1_ERR_INVALID_ARG;

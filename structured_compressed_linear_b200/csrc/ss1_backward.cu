@@ -52,16 +52,19 @@ __global__ void __launch_bounds__(256) expand_t_kernel(const T* __restrict__ Wc,
     const int nb = n0 / BN;
     for (int i = threadIdx.x; i < R * S; i += blockDim.x) {
         const int r = i / S, s = i % S;
-        tile[r * (S + 1) + s] = to_f(Wc[(size_t)(n0 + r) * Kc + (size_t)kc * S + s]);
+        const size_t wi = (size_t)(n0 + r) * Kc + (size_t)kc * S + s;
+        tile[r * (S + 1) + s] = SS1_IN(wi, (int64_t)N * Kc, kSiteBwdWc) ? to_f(Wc[wi]) : 0.0f;
     }
     __syncthreads();
     const int32_t* hrow = h + (size_t)nb * K + (size_t)kc * BK;
     const int8_t* grow = g + (size_t)nb * K + (size_t)kc * BK;
     for (int i = threadIdx.x; i < BK * R; i += blockDim.x) {
         const int k = i / R, r = i % R;
-        const int slot = hrow[k] - kc * S;
-        const float v = tile[r * (S + 1) + slot];
-        E[(size_t)(kc * BK + k) * N + n0 + r] = from_f<T>(grow[k] < 0 ? -v : v);
+        const bool tab_ok = SS1_IN(hrow + k - h, (int64_t)(N / BN) * K, kSiteBwdTab);
+        const int slot = tab_ok ? hrow[k] - kc * S : 0;
+        const float v = SS1_IN(slot, S, kSiteBwdSlot) ? tile[r * (S + 1) + slot] : 0.0f;
+        const size_t ei = (size_t)(kc * BK + k) * N + n0 + r;
+        if (SS1_IN(ei, (int64_t)K * N, kSiteBwdE)) E[ei] = from_f<T>(tab_ok && grow[k] < 0 ? -v : v);
     }
 }
 

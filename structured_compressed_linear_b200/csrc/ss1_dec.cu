@@ -246,7 +246,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
     // the wait.
     if (warp == kWarpLoad && lane == 0) {
         if (staged)
-            for (int m = 0; m < M; ++m) prefetch_l2_bulk(X + (size_t)m * K + (size_t)kc_lo * BKc, (uint32_t)(R * 2));
+            for (int m = 0; m < M; ++m)
+                if (SS1_SPAN_IN((size_t)m * K + (size_t)kc_lo * BKc, R, (int64_t)M * K, kSiteDecX))
+                    prefetch_l2_bulk(X + (size_t)m * K + (size_t)kc_lo * BKc, (uint32_t)(R * 2));
         for (int g = 0; g < G && g < kNW; ++g)
             prefetch_l2_2d(&tmap_w, (st0 + g) * kStageC, nb * kNeu);
     }
@@ -259,8 +261,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         if (staged && lane == 0) {
             ptx::mbar_arrive_expect_tx(&x_full[0], (uint32_t)(M * R * 2));
             for (int m = 0; m < M; ++m)
-                ptx::bulk_load(smem + F::OFF_X + (size_t)m * R * 2, X + (size_t)m * K + (size_t)kc_lo * BKc,
-                               (uint32_t)(R * 2), &x_full[0]);
+                if (SS1_SPAN_IN((size_t)m * K + (size_t)kc_lo * BKc, R, (int64_t)M * K, kSiteDecX))
+                    ptx::bulk_load(smem + F::OFF_X + (size_t)m * R * 2, X + (size_t)m * K + (size_t)kc_lo * BKc,
+                                   (uint32_t)(R * 2), &x_full[0]);
         }
         __syncwarp();
         // Wc: lane 0 refills the ring in stage order (stage g into slot g % kNW once the UMMAs of
@@ -406,7 +409,10 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             const int j = (st0 + g) * kStageC + kl;
             if (g < G && j < Kc) {
 #pragma unroll
-                for (int q = 0; q < C; ++q) e[q] = __ldg(tab + (size_t)j * C + q);
+                for (int q = 0; q < C; ++q)
+                    e[q] = SS1_IN(tab + (size_t)j * C + q - src, (int64_t)(N / kNeu) * K, kSiteDecTab)
+                               ? __ldg(tab + (size_t)j * C + q)
+                               : (uint16_t)0;
             }
         };
         const __nv_bfloat16* xsm = reinterpret_cast<const __nv_bfloat16*>(smem + F::OFF_X);
@@ -451,7 +457,10 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                         float v = 0.f;
 #pragma unroll
                         for (int q = 0; q < C; ++q) {
-                            const float x = __bfloat162float(xk[(size_t)m * row + (cur[q] & kSrcIdxMask)]);
+                            const size_t xi = (size_t)m * row + (cur[q] & kSrcIdxMask);
+                            const float x = (chunked || staged || SS1_IN(xk + xi - X, (int64_t)M * K, kSiteDecX))
+                                                ? __bfloat162float(xk[xi])
+                                                : 0.f;
                             v += (cur[q] & kSrcNegBit) ? -x : x;
                         }
                         *reinterpret_cast<__nv_bfloat16*>(stage + m * 128 + (((kl >> 3) ^ (m & 7)) << 4) + (kl & 7) * 2) =
@@ -497,10 +506,11 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 }
             }
             if (splits == 1) {
-                const float sc = FP8 ? scale[n] : 1.0f;
+                const float sc = FP8 && SS1_IN(n, N, kSiteDecScale) ? scale[n] : 1.0f;
 #pragma unroll
                 for (int m = 0; m < MP; ++m)
-                    if (m < M) Y[(size_t)m * N + n] = __float2bfloat16_rn(FP8 ? sc * d[m] : d[m]);
+                    if (m < M && SS1_IN((size_t)m * N + n, (int64_t)M * N, kSiteDecY))
+                        Y[(size_t)m * N + n] = __float2bfloat16_rn(FP8 ? sc * d[m] : d[m]);
             } else {
                 // this split's partial [MP rows][128 neurons] fp32, in the Wc ring: every stage has
                 // been multiplied (acc_full), so the ring is free
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         if (warp >= kFirstBuild && warp < kFirstBuild + kBuildWarps) {
             const int t = threadIdx.x - kFirstBuild * 32;   // neuron of the N-block
             const float* part = reinterpret_cast<const float*>(wring) + t;
-            const float sc = FP8 ? scale[(size_t)nb * kNeu + t] : 1.0f;
+            const float sc = FP8 && SS1_IN((size_t)nb * kNeu + t, N, kSiteDecScale) ? scale[(size_t)nb * kNeu + t] : 1.0f;
             for (int m = (int)ptx::cluster_ctarank(); m < M && m < MP; m += splits) {
                 // every split's partial requested before the first is added: one remote latency
                 float pv[16];
@@ -539,7 +549,8 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
 #pragma unroll
                 for (int s = 0; s < 16; ++s)
                     if (s < splits) v += pv[s];   // in split order
-                Y[(size_t)m * N + (size_t)nb * kNeu + t] = __float2bfloat16_rn(FP8 ? sc * v : v);
+                if (SS1_IN((size_t)m * N + (size_t)nb * kNeu + t, (int64_t)M * N, kSiteDecY))
+                    Y[(size_t)m * N + (size_t)nb * kNeu + t] = __float2bfloat16_rn(FP8 ? sc * v : v);
             }
         }
         ptx::cluster_sync();

@@ -38,8 +38,10 @@ __global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int 
     int8_t* grow = g + (size_t)nb * K + (size_t)kc * BK;
     uint16_t* sb = src + (size_t)b * S * c;
 
+    [[maybe_unused]] const int64_t ntab = (int64_t)(nblocks / KC) * K;   // entries of each table
     if (c == 1) {
         for (int k = 0; k < BK; ++k) {
+            if (!SS1_IN(hrow + k - h, ntab, kSiteHashH) || !SS1_IN(sb + k - src, ntab, kSiteHashSrc)) continue;
             hrow[k] = kc * S + k;
             grow[k] = 1;
             sb[k] = (uint16_t)k;
@@ -64,14 +66,17 @@ __global__ void __launch_bounds__(128) hashgen_kernel(uint64_t seed, int K, int 
         state += kGolden;                                   // draw t = BK-1+k
         const uint64_t r = splitmix_finalise(state);
         const bool neg = (r >> 63) != 0;
-        hrow[k] = kc * S + (int)perm[k] % S;
-        grow[k] = neg ? (int8_t)-1 : (int8_t)1;
+        if (SS1_IN(hrow + k - h, ntab, kSiteHashH)) {
+            hrow[k] = kc * S + (int)perm[k] % S;
+            grow[k] = neg ? (int8_t)-1 : (int8_t)1;
+        }
         where[perm[k]] = (uint8_t)k;
     }
     for (int s = 0; s < S; ++s) {
         for (int j = 0; j < c; ++j) {
             const int k = where[s + j * S];
-            sb[s * c + j] = (uint16_t)(k | (grow[k] < 0 ? kSrcNegBit : 0));
+            if (SS1_IN(k, BK, kSiteHashPerm) && SS1_IN(sb + s * c + j - src, ntab, kSiteHashSrc))
+                sb[s * c + j] = (uint16_t)(k | (grow[k] < 0 ? kSrcNegBit : 0));
         }
     }
 }
@@ -94,7 +99,7 @@ __global__ void slot_table_kernel(const int32_t* __restrict__ h, const int8_t* _
     if (i >= n) return;
     const int k = (int)(i % K);
     const int slot = h[i] - (k / BK) * S;
-    out[i] = (uint16_t)(slot | (g[i] < 0 ? kSrcNegBit : 0));
+    if (SS1_IN(slot, S, kSiteHashSlot)) out[i] = (uint16_t)(slot | (g[i] < 0 ? kSrcNegBit : 0));
 }
 
 }  // namespace

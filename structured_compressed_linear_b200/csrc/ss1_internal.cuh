@@ -14,6 +14,47 @@
 static constexpr uint16_t kSrcNegBit = 0x8000u;
 static constexpr uint16_t kSrcIdxMask = 0x00FFu;
 
+// Checked build. Compiled with SS1_CHECKED=1 (the debug library libss1_checked.so, which stands
+// in for a memory checker), every global-memory access that a kernel addresses by its own index
+// arithmetic first tests the element index against the extent of the buffer, in elements of
+// that buffer. A failed test records (site << 48) | index in one device word (the first failure
+// only; ss1_bounds_check reads and clears it) and the access is skipped: a load yields 0, a store
+// or copy is not made, and a wait on a skipped copy ends at its time limit. Tile copies by TMA
+// are bounded by their tensor maps in hardware and are not tested. In the normal build a test is
+// the constant true and compiles away.
+#ifndef SS1_CHECKED
+#define SS1_CHECKED 0
+#endif
+
+namespace ss1 {
+enum CheckSite : int {
+    kSiteSimtTab = 1, kSiteSimtX, kSiteSimtWc, kSiteSimtY,
+    kSiteSmallmTab, kSiteSmallmX, kSiteSmallmWc, kSiteSmallmY,
+    kSiteDecTab, kSiteDecX, kSiteDecY, kSiteDecScale,
+    kSiteProjTab, kSiteProjW, kSiteProjWc,
+    kSiteTc3Tab, kSiteTc3Bias, kSiteTc2Tab, kSiteTc2Wc, kSiteTc2Y,
+    kSiteBwdWc, kSiteBwdTab, kSiteBwdSlot, kSiteBwdE,
+    kSiteHashH, kSiteHashPerm, kSiteHashSrc, kSiteHashSlot,
+    kSiteSelftest = 63,
+};
+#if SS1_CHECKED
+extern __device__ unsigned long long g_bad_access;
+__device__ __forceinline__ bool check_span(int64_t i, int64_t len, int64_t n, int site) {
+    if (i >= 0 && len >= 0 && i + len <= n) return true;
+    atomicCAS(&g_bad_access, 0ull, ((unsigned long long)site << 48) | ((unsigned long long)i & 0xFFFFFFFFFFFFull));
+    return false;
+}
+#endif
+}  // namespace ss1
+
+#if SS1_CHECKED
+#define SS1_IN(i, n, site) (::ss1::check_span((int64_t)(i), 1, (int64_t)(n), (site)))
+#define SS1_SPAN_IN(i, len, n, site) (::ss1::check_span((int64_t)(i), (int64_t)(len), (int64_t)(n), (site)))
+#else
+#define SS1_IN(i, n, site) true
+#define SS1_SPAN_IN(i, len, n, site) true
+#endif
+
 struct ss1_layer {
     uint64_t magic;
     int device;

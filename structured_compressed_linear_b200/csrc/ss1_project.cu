@@ -64,7 +64,9 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
         for (int j = 0; j < C; ++j) {
             const int sl = lane + 32 * k;
-            ent[k * C + j] = sl < S ? __ldg(tab + sl * C + j) : (uint16_t)0;
+            ent[k * C + j] = sl < S && SS1_IN(tab + sl * C + j - src_tab, (int64_t)gridDim.y * KC * BK, kSiteProjTab)
+                                 ? __ldg(tab + sl * C + j)
+                                 : (uint16_t)0;
         }
     const int r_lo = blockIdx.z * rows_per_cta, r_hi = min(BN, r_lo + rows_per_cta);
     const T* wrow0 = W + ((size_t)nb * BN + r_lo) * K + (size_t)kc * BK;
@@ -76,7 +78,9 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
             for (int q = 0; q < kMaxVec; ++q) {
                 const int vi = lane + 32 * q;
-                if (vi < nvec) v[q] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + vi);
+                if (vi < nvec && SS1_SPAN_IN(wrow0 + (size_t)r * K + vi * (16 / E) - W, 16 / E,
+                                             (int64_t)gridDim.y * BN * K, kSiteProjW))
+                    v[q] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + vi);
             }
         }
     };
@@ -114,7 +118,8 @@ __global__ void __launch_bounds__(kThreads, 3)
                     for (int w2 = 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
                         for (int j = 0; j < w2; ++j) t[j] += t[j + w2];
-                    crow0[(size_t)r * Kc + sl] = (T)(t[0] * scale);
+                    if (SS1_IN(crow0 + (size_t)r * Kc + sl - Wc, (int64_t)gridDim.y * BN * Kc, kSiteProjWc))
+                        crow0[(size_t)r * Kc + sl] = (T)(t[0] * scale);
                 }
             }
             __syncwarp();
@@ -146,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
         for (int j = 0; j < C; ++j) {
             const int sl = lane + 32 * k;
-            ent[k * C + j] = sl < S ? __ldg(tab + sl * C + j) : (uint16_t)0;
+            ent[k * C + j] = sl < S && SS1_IN(tab + sl * C + j - src_tab, (int64_t)gridDim.y * KC * BK, kSiteProjTab)
+                                 ? __ldg(tab + sl * C + j)
+                                 : (uint16_t)0;
         }
     const int r_lo = blockIdx.z * rows_per_cta, r_hi = min(BN, r_lo + rows_per_cta);
     const __nv_bfloat16* wrow0 = W + ((size_t)nb * BN + r_lo) * K + (size_t)kc * BK;
@@ -159,7 +166,9 @@ __global__ void __launch_bounds__(kThreads, 3)
         for (int i = 0; i < 2; ++i) {
             const int r = warp + 16 * p + 8 * i;
             v[i] = make_uint4(0u, 0u, 0u, 0u);
-            if (r < rows && lane < nvec) v[i] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + lane);
+            if (r < rows && lane < nvec &&
+                SS1_SPAN_IN(wrow0 + (size_t)r * K + lane * 8 - W, 8, (int64_t)gridDim.y * BN * K, kSiteProjW))
+                v[i] = __ldg(reinterpret_cast<const uint4*>(wrow0 + (size_t)r * K) + lane);
         }
     };
 #pragma unroll
@@ -209,8 +218,10 @@ __global__ void __launch_bounds__(kThreads, 3)
                             ta[j] += ta[j + w2];
                             tb[j] += tb[j + w2];
                         }
-                    crow0[(size_t)ra * Kc + sl] = __float2bfloat16_rn(ta[0] * scale);
-                    if (second) crow0[(size_t)rb * Kc + sl] = __float2bfloat16_rn(tb[0] * scale);
+                    if (SS1_IN(crow0 + (size_t)ra * Kc + sl - Wc, (int64_t)gridDim.y * BN * Kc, kSiteProjWc))
+                        crow0[(size_t)ra * Kc + sl] = __float2bfloat16_rn(ta[0] * scale);
+                    if (second && SS1_IN(crow0 + (size_t)rb * Kc + sl - Wc, (int64_t)gridDim.y * BN * Kc, kSiteProjWc))
+                        crow0[(size_t)rb * Kc + sl] = __float2bfloat16_rn(tb[0] * scale);
                 }
             }
             __syncwarp();
@@ -235,8 +246,10 @@ __global__ void project_plain_kernel(const T* __restrict__ W, T* __restrict__ Wc
     for (int j = 0; j < 8; ++j) {
         t[j] = 0.0f;
         if (j < c) {
-            const float v = (float)W[n * K + (int64_t)kc * BK + (e[j] & kSrcIdxMask)];
-            t[j] = (e[j] & kSrcNegBit) ? -v : v;
+            const uint16_t ej = SS1_IN(e + j - src_tab, (N / BN) * K, kSiteProjTab) ? e[j] : (uint16_t)0;
+            const int64_t wi = n * K + (int64_t)kc * BK + (ej & kSrcIdxMask);
+            const float v = SS1_IN(wi, N * K, kSiteProjW) ? (float)W[wi] : 0.f;
+            t[j] = (ej & kSrcNegBit) ? -v : v;
         }
     }
 #pragma unroll

@@ -1,5 +1,6 @@
 // ss1_test_device_timeout: the bounded-wait error path, exercised without a fault. The SS1
-// pages have no counterpart; the entry point is specified in include/ss1.h.
+// pages have no counterpart; the entry point is specified in include/ss1.h. Also
+// ss1_test_bounds_check, the checked build's index test on given values.
 //
 // One thread waits on an mbarrier that nothing arrives on, through the same bounded wait the
 // forward kernels use, and writes the handle's status word the way a stalled forward kernel
@@ -29,7 +30,26 @@ __global__ void unsatisfied_wait_kernel(int32_t* status, uint64_t limit_ns) {
     }
 }
 
+#if SS1_CHECKED
+// One thread runs the checked build's index test on (index, extent) and touches no memory
+// besides the record the test writes when it fails.
+__global__ void index_test_kernel(int64_t index, int64_t extent) {
+    if (threadIdx.x == 0) (void)SS1_IN(index, extent, ss1::kSiteSelftest);
+}
+#endif
+
 }  // namespace
+
+extern "C" SS1_API int ss1_test_bounds_check(int64_t index, int64_t extent) {
+#if SS1_CHECKED
+    index_test_kernel<<<1, 32>>>(index, extent);
+    return cudaGetLastError() == cudaSuccess ? SS1_OK : SS1_ERR_CUDA;
+#else
+    (void)index;
+    (void)extent;
+    return SS1_ERR_UNSUPPORTED_SHAPE;
+#endif
+}
 
 extern "C" SS1_API int ss1_test_device_timeout(ss1_handle h, int64_t limit_ns, void* stream) {
     if (!ss1::handle_live(h)) return SS1_ERR_BAD_HANDLE;

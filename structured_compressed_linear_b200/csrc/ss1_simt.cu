@@ -69,8 +69,11 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
                     const T* xr = X + (size_t)(m0 + m) * K + (size_t)kc * BK;
                     const uint16_t* e = sblk + (size_t)(s0 + s) * c;
                     for (int j = 0; j < c; ++j) {
-                        const uint16_t t = e[j];
-                        const float x = to_f32(xr[t & kSrcIdxMask]);
+                        const uint16_t t =
+                            SS1_IN(e + j - src, (int64_t)(N / BN) * K, kSiteSimtTab) ? e[j] : (uint16_t)0;
+                        const float x = SS1_IN(xr + (t & kSrcIdxMask) - X, (int64_t)M * K, kSiteSimtX)
+                                            ? to_f32(xr[t & kSrcIdxMask])
+                                            : 0.f;
                         v += (t & kSrcNegBit) ? -x : x;
                     }
                 }
@@ -78,7 +81,8 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
             }
             for (int i = threadIdx.x; i < TN * kSlotGroup; i += kThreads) {
                 const int n = i / kSlotGroup, s = i % kSlotGroup;
-                Wt[s][n] = (s < sc) ? to_f32(Wc[(size_t)(n0 + n) * Kc + (size_t)kc * S + s0 + s]) : 0.f;
+                const size_t wi = (size_t)(n0 + n) * Kc + (size_t)kc * S + s0 + s;
+                Wt[s][n] = (s < sc && SS1_IN(wi, (int64_t)N * Kc, kSiteSimtWc)) ? to_f32(Wc[wi]) : 0.f;
             }
             __syncthreads();
             for (int s = 0; s < sc; ++s) {
@@ -101,7 +105,10 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
             const int m = m0 + ty + 16 * i;
             if (m >= M) continue;
 #pragma unroll
-            for (int j = 0; j < RN; ++j) from_f32(Y[(size_t)m * N + n0 + tx + 16 * j], acc[i][j]);
+            for (int j = 0; j < RN; ++j) {
+                const size_t yi = (size_t)m * N + n0 + tx + 16 * j;
+                if (SS1_IN(yi, (int64_t)M * N, kSiteSimtY)) from_f32(Y[yi], acc[i][j]);
+            }
         }
         return;
     }
@@ -125,7 +132,8 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(const T* __restrict__ X,
             for (int q = 0; q < 8; ++q)
                 if (s0 + q < splits) v += pv[q];   // in split order
         }
-        from_f32(Y[(size_t)(m0 + e / TN) * N + n0 + e % TN], v);
+        const size_t yi = (size_t)(m0 + e / TN) * N + n0 + e % TN;
+        if (SS1_IN(yi, (int64_t)M * N, kSiteSimtY)) from_f32(Y[yi], v);
     }
     ptx::cluster_sync();   // the peers have read this CTA's partial
 }

@@ -91,13 +91,15 @@ __global__ void __launch_bounds__(kThreads) smallm_kernel(const __nv_bfloat16* _
         uint4 wn[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            wn[i] = q < seg8 ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)i * Kc + j0 + q * 8))
-                             : make_uint4(0, 0, 0, 0);
+            wn[i] = q < seg8 && SS1_SPAN_IN(Wg + (size_t)i * Kc + j0 + q * 8 - Wc, 8, (int64_t)N * Kc, kSiteSmallmWc)
+                        ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)i * Kc + j0 + q * 8))
+                        : make_uint4(0, 0, 0, 0);
         // 2. sketch of this N-block for the segment
         for (int jj = threadIdx.x; jj < seg8 * 8; jj += kThreads) {
             const int j = j0 + jj;                                   // compressed column
-            uint16_t e[C];
-            load_entries<C>(tab + (size_t)j * C, e);
+            uint16_t e[C] = {};
+            if (SS1_SPAN_IN(tab + (size_t)j * C - src, C, (int64_t)(N / BN) * K, kSiteSmallmTab))
+                load_entries<C>(tab + (size_t)j * C, e);
             const __nv_bfloat16* xk = Xg + (size_t)(j >> lgS) * BK;  // its K-chunk
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
@@ -105,7 +107,8 @@ __global__ void __launch_bounds__(kThreads) smallm_kernel(const __nv_bfloat16* _
                 float v = 0.f;
 #pragma unroll
                 for (int t = 0; t < C; ++t) {
-                    const float x = __bfloat162float(xk[(size_t)m * K + (e[t] & kSrcIdxMask)]);
+                    const size_t xi = (size_t)m * K + (e[t] & kSrcIdxMask);
+                    const float x = SS1_IN(xk + xi - X, (int64_t)M * K, kSiteSmallmX) ? __bfloat162float(xk[xi]) : 0.f;
                     v += (e[t] & kSrcNegBit) ? -x : x;
                 }
                 xs[m][jj] = v;
@@ -121,7 +124,9 @@ __global__ void __launch_bounds__(kThreads) smallm_kernel(const __nv_bfloat16* _
             if (qn < seg8) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    wn[i] = __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)i * Kc + j0 + qn * 8));
+                    wn[i] = SS1_SPAN_IN(Wg + (size_t)i * Kc + j0 + qn * 8 - Wc, 8, (int64_t)N * Kc, kSiteSmallmWc)
+                                ? __ldg(reinterpret_cast<const uint4*>(Wg + (size_t)i * Kc + j0 + qn * 8))
+                                : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
@@ -167,7 +172,8 @@ __global__ void __launch_bounds__(kThreads) smallm_kernel(const __nv_bfloat16* _
         float v = 0.f;
 #pragma unroll
         for (int p = 0; p < WPG; ++p) v += red[p * G + nl / 4][nl % 4][m];
-        Y[(size_t)(m0 + m) * N + n0 + nl] = __float2bfloat16_rn(v);
+        const size_t yi = (size_t)(m0 + m) * N + n0 + nl;
+        if (SS1_IN(yi, (int64_t)M * N, kSiteSmallmY)) Y[yi] = __float2bfloat16_rn(v);
     }
 }
 

@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 4
                     for (int i = lane; i < kPieces; i += 32) {
                         const int r = i / kPerRow, c = i % kPerRow;
-                        ptx::cp_async_16(dst + kmajor_off<F::RB>(r, c * 8), src + (size_t)r * Kc + c * 8);
+                        if (SS1_SPAN_IN(src + (size_t)r * Kc + c * 8 - Wc, 8, (int64_t)N * Kc, kSiteTc2Wc))
+                            ptx::cp_async_16(dst + kmajor_off<F::RB>(r, c * 8), src + (size_t)r * Kc + c * 8);
                     }
                     asm volatile("cp.async.commit_group;" ::: "memory");
                     if (pending >= 0) {   // the previous panel's copies have landed
@@ -353,7 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int e0 = (sp * SP + (bt0 + kGroups * u) * SB) * C;   // first source of batch u
 #pragma unroll
                         for (int q = 0; q < kBatch / 2; ++q) {   // two {column, multiplier} entries per load
-                            const uint4 e2 = __ldg(reinterpret_cast<const uint4*>(tab + e0 + 2 * q));
+                            const uint4 e2 =
+                                SS1_SPAN_IN(tab + e0 + 2 * q - gather_tab, 2, (int64_t)NB * KC * BK, kSiteTc2Tab)
+                                    ? __ldg(reinterpret_cast<const uint4*>(tab + e0 + 2 * q))
+                                    : make_uint4(0u, 0u, 0u, 0u);
                             w[u][2 * q] = ptx::tmem_ld_32x32b_x1(xaddr + e2.x);
                             m[u][2 * q] = e2.y;
                             w[u][2 * q + 1] = ptx::tmem_ld_32x32b_x1(xaddr + e2.z);
@@ -464,7 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int piece = i * 32 + lane, y = piece >> 2, c = piece & 3;
                     const uint4 v = *reinterpret_cast<const uint4*>(stg + y * 64 + ((c ^ ((y >> 1) & 3)) << 4));
                     const int m = m0 + rb + y;
-                    if (m < M) *reinterpret_cast<uint4*>(Y + (size_t)m * N + (size_t)nb * kNeu + quad * 32 + c * 8) = v;
+                    if (m < M && SS1_SPAN_IN((size_t)m * N + (size_t)nb * kNeu + quad * 32 + c * 8, 8, (int64_t)M * N,
+                                             kSiteTc2Y))
+                        *reinterpret_cast<uint4*>(Y + (size_t)m * N + (size_t)nb * kNeu + quad * 32 + c * 8) = v;
                 }
                 __syncwarp();
             }

@@ -604,8 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
                 const TileInfo ti = chunk_info<Q, CHAIN>(p, i, kc);
                 const Tc3Layer& ly = p.layer[ti.l];
                 const uint16_t* src = ly.slot_tab + (size_t)(ti.nb0 + j) * ly.K + (size_t)kc * BK + u * kUnitK;
-                e[0] = __ldg(src + lane);
-                e[1] = __ldg(src + lane + 32);
+                [[maybe_unused]] const int64_t tab_n = (int64_t)ly.NG * Q * ly.K;
+                e[0] = SS1_IN(src + lane - ly.slot_tab, tab_n, kSiteTc3Tab) ? __ldg(src + lane) : 0u;
+                e[1] = SS1_IN(src + lane + 32 - ly.slot_tab, tab_n, kSiteTc3Tab) ? __ldg(src + lane + 32) : 0u;
             }
         };
         bool ok = true;
@@ -735,7 +736,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc3_kernel(const __grid_constant_
             auto store_block = [&](int q, uint32_t (&r)[32]) {
                 uint8_t* box = stg + (nst & 1) * kEpiBox;
                 if constexpr (FX) {   // bias of column col0 + 32 q + j (lane j loads it), then the activation
-                    const float bl = bias ? __bfloat162float(bias[col0 + q * 32 + lane]) : 0.0f;
+                    const float bl = bias && SS1_IN(col0 + q * 32 + lane, (int64_t)ly.NG * Q * kNeu, kSiteTc3Bias)
+                                         ? __bfloat162float(bias[col0 + q * 32 + lane])
+                                         : 0.0f;
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj)
                         r[jj] = __float_as_uint(activate(__uint_as_float(r[jj]) + __shfl_sync(0xffffffffu, bl, jj), act));

@@ -18,12 +18,15 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libss1.so")
+#: The bounds-checked debug build of the same sources (ss1_bounds_check in include/ss1.h).
+CHECKED_LIB_PATH = os.path.join(_HERE, "libss1_checked.so")
 
 SYMBOLS = ("ss1_create", "ss1_forward", "ss1_forward_with", "ss1_select_kernel", "ss1_destroy",
            "ss1_get_tables", "ss1_get_info", "ss1_device_status", "ss1_strerror", "ss1_forward_noalloc",
            "ss1_test_device_timeout", "ss1_project", "ss1_backward_workspace", "ss1_backward_input",
            "ss1_backward_weight", "ss1_quantize_fp8", "ss1_forward_fp8", "ss1_forward_ex", "ss1_chain_forward",
-           "ss1_chain_fused", "ss1_test_forward_timeout", "ss1_last_launch")
+           "ss1_chain_fused", "ss1_test_forward_timeout", "ss1_last_launch", "ss1_bounds_check",
+           "ss1_test_bounds_check")
 
 #: (N / BN) * K limit of ss1_forward_noalloc (SS1_NOALLOC_MAX_ENTRIES in include/ss1.h).
 NOALLOC_MAX_ENTRIES = 983040
@@ -95,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.ss1_chain_fused.argtypes = [ctypes.POINTER(vp), i32, ctypes.POINTER(i32)]
     L.ss1_test_forward_timeout.argtypes = [vp, vp, vp, vp, i64, i64, vp]
     L.ss1_last_launch.argtypes = [ctypes.POINTER(_LaunchInfo)]
+    L.ss1_bounds_check.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(u64)]
+    L.ss1_test_bounds_check.argtypes = [i64, i64]
     L.ss1_strerror.restype = ctypes.c_char_p
     for name in SYMBOLS:
         if name != "ss1_strerror":
@@ -104,8 +109,28 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     return L
 
 
+_active = None
+
+
 def lib() -> ctypes.CDLL:
-    return load_library()
+    """The library every call of this module goes through (libss1.so unless use_library chose another)."""
+    return _active if _active is not None else load_library()
+
+
+def use_library(path: str) -> ctypes.CDLL:
+    """Route this module's calls through the library at `path` (CHECKED_LIB_PATH: the checked
+    build); use_library(LIB_PATH) switches back. A handle belongs to the library that made it:
+    destroy layers before switching."""
+    global _active
+    _active = None if path == LIB_PATH else load_library(path)
+    return lib()
+
+
+def bounds_check() -> tuple[bool, int]:
+    """(checked build?, first failed index test since the last call or 0) of the active library."""
+    checked, record = ctypes.c_int(0), ctypes.c_uint64(0)
+    _check(lib().ss1_bounds_check(ctypes.byref(checked), ctypes.byref(record)), "ss1_bounds_check")
+    return bool(checked.value), int(record.value)
 
 
 class SS1Error(RuntimeError):
@@ -137,7 +162,8 @@ class SS1Layer:
     def __init__(self, K: int, N: int, c: int, BK: int, BN: int, seed: int):
         self.K, self.N, self.c, self.BK, self.BN, self.seed = K, N, c, BK, BN, seed
         h = ctypes.c_void_p()
-        _check(lib().ss1_create(K, N, c, BK, BN, seed & 0xFFFFFFFFFFFFFFFF, ctypes.byref(h)), "ss1_create")
+        self._lib = lib()   # the library that owns the handle, for every later call
+        _check(self._lib.ss1_create(K, N, c, BK, BN, seed & 0xFFFFFFFFFFFFFFFF, ctypes.byref(h)), "ss1_create")
         self._h = h
         self.device = torch.cuda.current_device()
 
@@ -165,7 +191,7 @@ class SS1Layer:
         elif out.shape != (M, self.N) or out.dtype != X.dtype or not out.is_contiguous() or out.device != X.device:
             raise ValueError("out must be a contiguous [M, N] tensor of X's dtype on X's device")
         st = stream if stream is not None else torch.cuda.current_stream(X.device)
-        _check(lib().ss1_forward_with(self.handle, X.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
+        _check(self._lib.ss1_forward_with(self.handle, X.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
                                       _dtype_code(X.dtype), int(kernel), st.cuda_stream), "ss1_forward")
         return out
 
@@ -184,14 +210,14 @@ class SS1Layer:
         elif out.shape != shape or out.dtype != W.dtype or not out.is_contiguous() or out.device != W.device:
             raise ValueError("out must be a contiguous [N, K/c] tensor of W's dtype on W's device")
         st = stream if stream is not None else torch.cuda.current_stream(W.device)
-        _check(lib().ss1_project(self.handle, W.data_ptr(), out.data_ptr(), _dtype_code(W.dtype), st.cuda_stream),
+        _check(self._lib.ss1_project(self.handle, W.data_ptr(), out.data_ptr(), _dtype_code(W.dtype), st.cuda_stream),
                "ss1_project")
         return out
 
     def backward_workspace(self, M: int, dtype: torch.dtype = torch.bfloat16) -> Tuple[int, int]:
         """Workspace bytes of backward_input and backward_weight (ss1_backward_workspace)."""
         a, b = ctypes.c_size_t(), ctypes.c_size_t()
-        _check(lib().ss1_backward_workspace(self.handle, M, _dtype_code(dtype), ctypes.byref(a), ctypes.byref(b)),
+        _check(self._lib.ss1_backward_workspace(self.handle, M, _dtype_code(dtype), ctypes.byref(a), ctypes.byref(b)),
                "ss1_backward_workspace")
         return a.value, b.value
 
@@ -213,7 +239,7 @@ class SS1Layer:
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dY.device)
         st = stream if stream is not None else torch.cuda.current_stream(dY.device)
-        _check(lib().ss1_backward_input(self.handle, dY.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
+        _check(self._lib.ss1_backward_input(self.handle, dY.data_ptr(), Wc.data_ptr(), out.data_ptr(), M,
                                         _dtype_code(dY.dtype), workspace.data_ptr(), workspace.numel(),
                                         st.cuda_stream), "ss1_backward_input")
         return out
@@ -231,7 +257,7 @@ class SS1Layer:
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
         st = stream if stream is not None else torch.cuda.current_stream(X.device)
-        _check(lib().ss1_backward_weight(self.handle, X.data_ptr(), dY.data_ptr(), out.data_ptr(), M,
+        _check(self._lib.ss1_backward_weight(self.handle, X.data_ptr(), dY.data_ptr(), out.data_ptr(), M,
                                          _dtype_code(X.dtype), workspace.data_ptr(), workspace.numel(),
                                          st.cuda_stream), "ss1_backward_weight")
         return out
@@ -250,7 +276,7 @@ class SS1Layer:
         M = X.shape[0]
         out = torch.empty((M, self.N), dtype=X.dtype, device=X.device) if out is None else out
         st = stream if stream is not None else torch.cuda.current_stream(X.device)
-        _check(lib().ss1_forward_ex(self.handle, X.data_ptr(), Wc.data_ptr(), bias.data_ptr() if bias is not None else None,
+        _check(self._lib.ss1_forward_ex(self.handle, X.data_ptr(), Wc.data_ptr(), bias.data_ptr() if bias is not None else None,
                                     int(act), out.data_ptr(), M, _dtype_code(X.dtype), int(kernel), st.cuda_stream),
                "ss1_forward_ex")
         return out
@@ -268,30 +294,30 @@ class SS1Layer:
         M = X.shape[0]
         out = torch.empty((M, self.N), dtype=torch.bfloat16, device=X.device) if out is None else out
         st = stream if stream is not None else torch.cuda.current_stream(X.device)
-        _check(lib().ss1_forward_fp8(self.handle, X.data_ptr(), Wq.data_ptr(), scale.data_ptr(), out.data_ptr(), M,
+        _check(self._lib.ss1_forward_fp8(self.handle, X.data_ptr(), Wq.data_ptr(), scale.data_ptr(), out.data_ptr(), M,
                                      st.cuda_stream), "ss1_forward_fp8")
         return out
 
     def select_kernel(self, M: int, dtype: torch.dtype = torch.bfloat16) -> Kernel:
         k = ctypes.c_int()
-        _check(lib().ss1_select_kernel(self.handle, M, _dtype_code(dtype), ctypes.byref(k)), "ss1_select_kernel")
+        _check(self._lib.ss1_select_kernel(self.handle, M, _dtype_code(dtype), ctypes.byref(k)), "ss1_select_kernel")
         return Kernel(k.value)
 
     def tables(self) -> Tuple[np.ndarray, np.ndarray]:
         NB = self.N // self.BN
         h = np.empty((NB, self.K), dtype=np.int32)
         g = np.empty((NB, self.K), dtype=np.int8)
-        _check(lib().ss1_get_tables(self.handle, h.ctypes.data, g.ctypes.data), "ss1_get_tables")
+        _check(self._lib.ss1_get_tables(self.handle, h.ctypes.data, g.ctypes.data), "ss1_get_tables")
         return h, g
 
     def device_status(self) -> Tuple[int, int]:
         d = ctypes.c_int32()
-        st = lib().ss1_device_status(self.handle, ctypes.byref(d))
+        st = self._lib.ss1_device_status(self.handle, ctypes.byref(d))
         return st, d.value
 
     def close(self):
         if getattr(self, "_h", None) is not None:
-            lib().ss1_destroy(self._h)
+            self._lib.ss1_destroy(self._h)
             self._h = None
 
     def __del__(self):
@@ -364,7 +390,7 @@ def chain_fused(layers) -> bool:
     """Whether chain_forward runs these layers as one persistent launch (ss1_chain_fused)."""
     hs = (ctypes.c_void_p * len(layers))(*[ly.handle.value for ly in layers])
     f = ctypes.c_int()
-    _check(lib().ss1_chain_fused(hs, len(layers), ctypes.byref(f)), "ss1_chain_fused")
+    _check(layers[0]._lib.ss1_chain_fused(hs, len(layers), ctypes.byref(f)), "ss1_chain_fused")
     return bool(f.value)
 
 
@@ -388,7 +414,7 @@ def chain_forward(layers, X: torch.Tensor, Wcs, biases=None, acts=None, outs=Non
     bias_arr = _ptr_array(biases) if biases is not None else None
     act_arr = (ctypes.c_int * n)(*[int(a) for a in acts]) if acts is not None else None
     st = stream if stream is not None else torch.cuda.current_stream(X.device)
-    _check(lib().ss1_chain_forward(hs, n, X.data_ptr(), _ptr_array(Wcs), bias_arr, act_arr, _ptr_array(outs), M,
+    _check(layers[0]._lib.ss1_chain_forward(hs, n, X.data_ptr(), _ptr_array(Wcs), bias_arr, act_arr, _ptr_array(outs), M,
                                    st.cuda_stream), "ss1_chain_forward")
     return outs
 

@@ -158,3 +158,25 @@ def test_last_launch_before_any_launch(lib):
     info = got["info"]
     assert info["kernel"] == "" and info["grid"] == (0, 0) and info["resident_clusters"] == [0] * 17
     assert lib.ss1_last_launch(None) == -1
+
+
+def test_normal_build_makes_no_index_tests(lib):
+    """The normal library reports itself unchecked, with an empty record, and launches no self-test."""
+    checked, record = ctypes.c_int(7), ctypes.c_uint64(7)
+    assert lib.ss1_bounds_check(ctypes.byref(checked), ctypes.byref(record)) == 0
+    assert (checked.value, record.value) == (0, 0)
+    assert lib.ss1_bounds_check(None, ctypes.byref(record)) == -1
+    assert lib.ss1_test_bounds_check(5, 4) == -8   # SS1_ERR_UNSUPPORTED_SHAPE: nothing launched
+
+
+def test_checked_build_exports_the_same_entry_points():
+    """libss1_checked.so, the bounds-checked debug build of the same sources, has the full ABI."""
+    from structured_compressed_linear_b200 import build
+    from structured_compressed_linear_b200 import ss1
+    path = build.build(checked=True)
+    assert path == ss1.CHECKED_LIB_PATH
+    clib = ss1.load_library(path)
+    for name in _declared():
+        assert hasattr(clib, name), name
+    record = ctypes.c_uint64(0)
+    assert clib.ss1_bounds_check(None, ctypes.byref(record)) == -1
