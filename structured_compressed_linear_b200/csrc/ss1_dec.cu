@@ -58,9 +58,9 @@ constexpr int kXBytes = 20 * 1024;       // X in shared memory: the CTA's input 
 constexpr int kXChunkRows = 16;          // chunk mode: rows of an X box (M <= 16)
 constexpr int kXUnitBytes = kXChunkRows * 512 * 2;    // one unit: [16 rows x up to 512 inputs]
 constexpr int kMaxXUnits = 8;             // chunk mode: X units in flight at most
-constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kBuildWarps = 4;
-constexpr int kFirstConv = kFirstBuild + kBuildWarps, kConvWarps = 4;   // FP8 weights: the converter warps
-constexpr int kWarpMma2 = kFirstBuild + kBuildWarps;   // bf16: the further UMMA warps, from here
+// Build warps from kFirstBuild: bf16, two row parts of kEpiWarps warps; FP8, one part (the
+// converter warps come after them). The first part also runs the epilogue.
+constexpr int kWarpLoad = 0, kWarpMma = 1, kFirstBuild = 2, kEpiWarps = 4, kConvWarps = 4;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // L2 prefetch of one 2D tile of a tensor map: no shared memory, no completion to wait for.
@@ -93,7 +93,11 @@ struct DecCfg {
     // bf16: NMMA UMMA warps take the stages round-robin into NMMA accumulators, so that the
     // barrier waits of one (each lets the tensor pipe's queue drain) overlap the others' UMMAs
     static constexpr int NMMA = FP8 ? 1 : kNmmaBf16;
-    static constexpr int THREADS = (kFirstBuild + kBuildWarps + (FP8 ? kConvWarps : NMMA - 1)) * 32;
+    static constexpr int ROW_PARTS = FP8 ? 1 : 2;
+    static constexpr int BUILD_WARPS = kEpiWarps * ROW_PARTS;
+    static constexpr int FIRST_CONV = kFirstBuild + BUILD_WARPS;   // FP8: the converter warps, from here
+    static constexpr int WARP_MMA2 = kFirstBuild + BUILD_WARPS;    // bf16: the further UMMA warps, from here
+    static constexpr int THREADS = (kFirstBuild + BUILD_WARPS + (FP8 ? kConvWarps : NMMA - 1)) * 32;
     // one CTA per SM with a deep ring: a stage stays in the ring from its load until its UMMAs
     // complete, and about 128 KB per SM must be on the way from HBM at any time for it to run at
     // its rate at the latency it has under that load
@@ -212,6 +216,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
     const int xub = kXChunkRows * ui * 2;
     const int nxu = chunked ? min(kMaxXUnits, F::X_BYTES / xub) : 1;
 
+    // row parts of the build (bf16): the second (rows MP / 2 ..) only where M reaches it
+    const int nrp = F::ROW_PARTS == 2 && M > MP / 2 ? 2 : 1;
+
     // sketch stages start zeroed: rows past M are never written afterwards
     for (int i = threadIdx.x; i < kNB * F::B_STAGE / 16; i += kThreads)
         reinterpret_cast<uint4*>(bring)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -220,11 +227,14 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         // FP8: a Wc slot is free once the converter warps have read it (bf16: once its UMMAs completed)
         for (int i = 0; i < kNW; ++i) { ptx::mbar_init(&w_full[i], 1); ptx::mbar_init(&w_empty[i], FP8 ? kConvWarps : 1); }
         for (int i = 0; i < kNB; ++i) {
-            ptx::mbar_init(&b_full[i], kBuildWarps / 2 + (FP8 ? kConvWarps : 0));
+            ptx::mbar_init(&b_full[i], kEpiWarps / 2 * nrp + (FP8 ? kConvWarps : 0));
             ptx::mbar_init(&b_empty[i], 1);
         }
         ptx::mbar_init(acc_full, F::NMMA);
-        for (int i = 0; i < kMaxXUnits; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kBuildWarps / 2 * (chunked ? spc : 1)); }
+        for (int i = 0; i < kMaxXUnits; ++i) {
+            ptx::mbar_init(&x_full[i], 1);
+            ptx::mbar_init(&x_empty[i], kEpiWarps / 2 * nrp * (chunked ? spc : 1));
+        }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -313,11 +323,11 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             volatile int no_abort = 0;
             ptx::mbar_wait(&x_full[0], 0, &no_abort, kWaitNs);
         }
-    } else if (warp == kWarpMma || (F::NMMA > 1 && warp >= kWarpMma2 && warp < kWarpMma2 + F::NMMA - 1)) {
+    } else if (warp == kWarpMma || (F::NMMA > 1 && warp >= F::WARP_MMA2 && warp < F::WARP_MMA2 + F::NMMA - 1)) {
         // ------------------------------------------------------------------ UMMAs
         // UMMA warp w (w < NMMA) takes stages g = w, w + NMMA, ... into accumulator w (MP columns
         // from w * MP).
-        const int w = warp == kWarpMma ? 0 : warp - kWarpMma2 + 1;
+        const int w = warp == kWarpMma ? 0 : warp - F::WARP_MMA2 + 1;
         const uint32_t dacc = tm + (uint32_t)(w * MP);
         constexpr uint32_t idesc = ptx::idesc_bf16_f32(kNeu, MP);
         const uint64_t wdesc0 = ptx::smem_desc(ptx::smem_u32(wring), 16, 1024, ptx::kLayoutSW128);
@@ -356,7 +366,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             }
         }
         __syncwarp();
-    } else if (FP8 && warp >= kFirstConv) {
+    } else if (FP8 && warp >= F::FIRST_CONV) {
         // ------------------------------------------------------------------ FP8 -> bf16 A stages
         // Thread = neuron (TMEM lane 32 q + lane, q = warp % 4): its row of the stage, 64 codes in
         // four 16-byte chunks (64-byte swizzle: chunk c of row r sits at c ^ ((r >> 1) & 3), so
@@ -398,11 +408,15 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         }
     } else {
         // ------------------------------------------------------------------ sketch, then epilogue
-        // Build thread t: column kl = t % 64 of the stages g with g % 2 == t / 64 (two stages are
-        // built at once), all rows. A thread's table entries are loaded one of its stages ahead,
-        // so that a stage waits only for its X gathers, which are all in flight together.
+        // Build thread t: column kl = t % 64 of the stages g with g % 2 == (t / 64) % 2 (two stages
+        // are built at once), the rows of row part rp = t / 128 (bf16: rows 0 .. MP / 2 - 1 and
+        // MP / 2 .., FP8: all). A thread's table entries are loaded one of its stages ahead, so
+        // that a stage waits only for its X gathers, which are all in flight together. A second
+        // row part builds only where M reaches it; the first also runs the epilogue.
+        constexpr int kRowsPart = MP / F::ROW_PARTS;
         const int t = threadIdx.x - kFirstBuild * 32;
-        const int kl = t % kStageC, half = t / kStageC;
+        const int kl = t % kStageC, half = (t / kStageC) & 1, rp = t / (2 * kStageC);
+        const bool builds = rp < nrp;
         const int BK = BKc;
         const uint16_t* tab = src + (size_t)nb * KC * S * C;   // this N-block's entries, column-major order
         auto fetch = [&](int g, uint16_t (&e)[C]) {
@@ -423,7 +437,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
             if (lane == 0) report(status, abort_flag, 8);
             ok = false;
         }
-        for (int g = half; g < G && ok; g += 2) {
+        for (int g = half; g < G && ok && builds; g += 2) {
             const int bs = g % kNB;
             uint16_t cur[C];
 #pragma unroll
@@ -451,8 +465,9 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                                           : staged ? xsm + (size_t)(kc - kc_lo) * BK
                                                    : X + (size_t)kc * BK;
                 const size_t row = chunked ? (size_t)bi : staged ? (size_t)R : (size_t)K;
-#pragma unroll
-                for (int m = 0; m < MP; ++m) {
+#pragma unroll(kRowsPart > 16 ? 16 : kRowsPart)
+                for (int mi = 0; mi < kRowsPart; ++mi) {
+                    const int m = rp * kRowsPart + mi;
                     if (m < M) {
                         float v = 0.f;
 #pragma unroll
@@ -469,9 +484,11 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
                 }
             } else {
 #pragma unroll
-                for (int m = 0; m < MP; ++m)
+                for (int mi = 0; mi < kRowsPart; ++mi) {
+                    const int m = rp * kRowsPart + mi;
                     if (m < M)
                         *reinterpret_cast<uint16_t*>(stage + m * 128 + (((kl >> 3) ^ (m & 7)) << 4) + (kl & 7) * 2) = 0;
+                }
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
@@ -482,42 +499,43 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         }
         // epilogue: warp (quad) holds neurons nb * 128 + quad * 32 + lane
         const int quad = warp & 3;
-        if (ok && warp_wait(acc_full, 0, abort_flag) && !*abort_flag) {
+        if (rp > 0) {
+            // the second row part holds no accumulator lanes of its own
+        } else if (ok && warp_wait(acc_full, 0, abort_flag) && !*abort_flag) {
             ptx::tc_fence_after();
             const int n = nb * kNeu + quad * 32 + lane;
-            float d[MP];
+            const float sc = FP8 && splits == 1 && SS1_IN(n, N, kSiteDecScale) ? scale[n] : 1.0f;
+            // this split's partial [MP rows][128 neurons] fp32 goes into the Wc ring: every stage
+            // has been multiplied (acc_full), so the ring is free
+            float* part = reinterpret_cast<float*>(wring) + quad * 32 + lane;
 #pragma unroll
-            for (int m0 = 0; m0 < MP; m0 += 16) {
+            for (int m0 = 0; m0 < MP; m0 += 16) {   // 16 rows at a time: the accumulators summed in order
+                float d[16];
                 uint32_t r[16];
                 ptx::tmem_ld_32x32b_x16(tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)m0, r);
                 ptx::tmem_ld_wait();
                 ptx::tmem_ld_fence_regs<16>(r);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) d[m0 + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) d[i] = __uint_as_float(r[i]);
 #pragma unroll
-                for (int a = 1; a < F::NMMA; ++a) {   // plus the other accumulators, in order
+                for (int a = 1; a < F::NMMA; ++a) {
                     if (a < G) {
                         ptx::tmem_ld_32x32b_x16(tm + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * MP + m0), r);
                         ptx::tmem_ld_wait();
                         ptx::tmem_ld_fence_regs<16>(r);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) d[m0 + i] += __uint_as_float(r[i]);
+                        for (int i = 0; i < 16; ++i) d[i] += __uint_as_float(r[i]);
                     }
                 }
-            }
-            if (splits == 1) {
-                const float sc = FP8 && SS1_IN(n, N, kSiteDecScale) ? scale[n] : 1.0f;
 #pragma unroll
-                for (int m = 0; m < MP; ++m)
-                    if (m < M && SS1_IN((size_t)m * N + n, (int64_t)M * N, kSiteDecY))
-                        Y[(size_t)m * N + n] = __float2bfloat16_rn(FP8 ? sc * d[m] : d[m]);
-            } else {
-                // this split's partial [MP rows][128 neurons] fp32, in the Wc ring: every stage has
-                // been multiplied (acc_full), so the ring is free
-                float* part = reinterpret_cast<float*>(wring) + quad * 32 + lane;
-#pragma unroll
-                for (int m = 0; m < MP; ++m)
-                    if (m < M) part[(size_t)m * kNeu] = d[m];
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + i;
+                    if (m >= M) break;
+                    if (splits > 1)
+                        part[(size_t)m * kNeu] = d[i];
+                    else if (SS1_IN((size_t)m * N + n, (int64_t)M * N, kSiteDecY))
+                        Y[(size_t)m * N + n] = __float2bfloat16_rn(FP8 ? sc * d[i] : d[i]);
+                }
             }
         } else if (lane == 0 && !*abort_flag) {
             report(status, abort_flag, 4);
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(DecCfg<MP, FP8>::THREADS, DecCfg<MP, FP8>::MIN
         // partial is visible to the cluster; the second keeps each CTA's shared memory alive
         // until its peers have read it.
         ptx::cluster_sync();
-        if (warp >= kFirstBuild && warp < kFirstBuild + kBuildWarps) {
+        if (warp >= kFirstBuild && warp < kFirstBuild + kEpiWarps) {
             const int t = threadIdx.x - kFirstBuild * 32;   // neuron of the N-block
             const float* part = reinterpret_cast<const float*>(wring) + t;
             const float sc = FP8 && SS1_IN((size_t)nb * kNeu + t, N, kSiteDecScale) ? scale[(size_t)nb * kNeu + t] : 1.0f;
