@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 namespace ss1 {
@@ -230,6 +231,182 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------- wide persistent kernel
+// c = 1 with N a multiple of 256: one CTA per SM walks the output tiles of 128 rows x 256 columns
+// (tile t = blockIdx.x + i * gridDim.x, its 256 columns fastest, so the CTAs running at once
+// share X row panels in L2). UMMA N = 256 halves the shared-memory bytes the tensor pipe reads
+// per flop against N = 128 (A is read once for twice the columns), which is what holds the
+// 128 x 128 tile below the tensor rate. The K loop runs in stages of 64 columns (X 16 KB + W
+// 32 KB) through a 4-deep ring, across tile boundaries; two TMEM accumulators of 256 columns let
+// the epilogue warps store one tile while the MMA thread fills the other.
+constexpr int kWN = 256;                         // output columns per tile (UMMA N)
+constexpr int kWK = 64;                          // K columns per stage
+constexpr int kWRing = 4;                        // stages in the ring
+constexpr int kWXBytes = kBM * kWK * 2;          // 16 KB
+constexpr int kWWBytes = kWN * kWK * 2;          // 32 KB
+constexpr int kWStage = kWXBytes + kWWBytes;     // 48 KB, a multiple of the 1 KB swizzle atom
+constexpr int kWNBar = 2 * kWRing + 2 + 2 + 1;
+constexpr int kWSmem = kWRing * kWStage + kWNBar * 8 + 16 + 1024;
+static_assert(kWSmem <= 227 * 1024, "shared memory of one CTA");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tcw_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               __nv_bfloat16* __restrict__ Y, int M, int N, int K, int num_tiles, int tiles_n, int32_t* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWRing * kWStage);
+    uint64_t* full = bars;                   // [kWRing] a stage's X and W tiles have landed
+    uint64_t* empty = full + kWRing;         // [kWRing] the stage's UMMAs have completed
+    uint64_t* acc_full = empty + kWRing;     // [2] an accumulator holds a finished tile
+    uint64_t* acc_empty = acc_full + 2;      // [2] the epilogue has read an accumulator
+    uint64_t* mma_done = acc_empty + 2;      // time-out path: the UMMAs in flight have completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int KS = (K + kWK - 1) / kWK;      // stages per tile (TMA reads zeros past K)
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kWRing; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&acc_full[i], 1);
+            ptx::mbar_init(&acc_empty[i], 4);   // one arrival per epilogue warp
+        }
+        ptx::mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 2 * kWN);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap_w);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+                const int m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * kWN;
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int sl = it % kWRing;
+                    if (it >= kWRing &&
+                        !ptx::mbar_wait(&empty[sl], (uint32_t)(((it / kWRing) - 1) & 1), abort_flag, kWaitLimitNs)) {
+                        report(status, abort_flag, 11);
+                        break;
+                    }
+                    uint8_t* st = smem + sl * kWStage;
+                    ptx::mbar_arrive_expect_tx(&full[sl], kWStage);
+                    ptx::tma_load_2d(st, &tmap_x, &full[sl], ks * kWK, m0);
+                    ptx::tma_load_2d(st + kWXBytes, &tmap_w, &full[sl], ks * kWK, n0);
+                }
+            }
+            if (*abort_flag) {   // every issued copy lands before the CTA may exit
+                volatile int no_abort = 0;
+                for (int j = it > kWRing ? it - kWRing : 0; j < it; ++j)
+                    ptx::mbar_wait(&full[j % kWRing], (uint32_t)((j / kWRing) & 1), &no_abort, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kWN);
+            int it = 0, tl = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tl) {
+                const int a = tl & 1;
+                if (tl >= 2 && !ptx::mbar_wait(&acc_empty[a], (uint32_t)(((tl / 2) - 1) & 1), abort_flag, kWaitLimitNs)) {
+                    report(status, abort_flag, 12);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(a * kWN);
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int sl = it % kWRing;
+                    if (!ptx::mbar_wait(&full[sl], (uint32_t)((it / kWRing) & 1), abort_flag, kWaitLimitNs)) {
+                        report(status, abort_flag, 13);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t xb = ptx::smem_u32(smem + sl * kWStage);
+                    const uint32_t wb = xb + (uint32_t)kWXBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kWK / 16; ++kk) {   // 16 columns = 32 bytes along the swizzled row
+                        const uint64_t ad = ptx::smem_desc(xb + (uint32_t)(kk * 32), 16, 1024, ptx::kLayoutSW128);
+                        const uint64_t bd = ptx::smem_desc(wb + (uint32_t)(kk * 32), 16, 1024, ptx::kLayoutSW128);
+                        ptx::umma_bf16_ss(acc, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    ptx::umma_commit(&empty[sl]);
+                }
+                if (!ok) break;
+                ptx::umma_commit(&acc_full[a]);
+            }
+            if (*abort_flag) {   // the UMMAs in flight complete before TMEM is released
+                ptx::umma_commit(mma_done);
+                volatile int no_abort = 0;
+                ptx::mbar_wait(mma_done, 0, &no_abort, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int quad = warp & 3;              // TMEM lanes 32 quad .. 32 quad + 31
+        const int row = quad * 32 + lane;
+        int tl = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
+            const int a = tl & 1;
+            bool ok = ptx::mbar_wait(&acc_full[a], (uint32_t)((tl / 2) & 1), abort_flag, kWaitLimitNs);
+            if (!ok && lane == 0 && !*abort_flag) report(status, abort_flag, 14);
+            ptx::tc_fence_after();
+            ok = __all_sync(0xffffffffu, ok && !*abort_flag);   // tcgen05.ld is warp-collective
+            if (!ok) break;
+            const int m = (tile / tiles_n) * kBM + row;
+            __nv_bfloat16* yrow = Y + (size_t)m * N + (size_t)(tile % tiles_n) * kWN;
+#pragma unroll 1
+            for (int col0 = 0; col0 < kWN; col0 += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * kWN + col0), r);
+                ptx::tmem_ld_wait();
+                if (m < M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 o;
+                        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[q * 8 + 2 * t]),
+                                                                     __uint_as_float(r[q * 8 + 2 * t + 1]));
+                            ow[t] = *reinterpret_cast<uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&acc_empty[a]);   // this warp's lanes of the accumulator are read
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 2 * kWN);
+    }
+}
+
 // ---------------------------------------------------------------------------- host side
 
 bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -264,6 +441,22 @@ cudaError_t launch_cfg(const ss1_layer& L, const void* X, const void* Wc, void* 
     return cudaGetLastError();
 }
 
+cudaError_t launch_wide(const ss1_layer& L, const void* X, const void* Wc, void* Y, int64_t M, cudaStream_t st) {
+    const cudaError_t attr_err = smem_attr_once(reinterpret_cast<const void*>(&tcw_kernel), kWSmem);
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mx, mw;
+    if (!make_map_2d(&mx, X, (uint64_t)L.K, (uint64_t)M, kWK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&mw, Wc, (uint64_t)L.K, (uint64_t)L.N, kWK, kWN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const int64_t tiles_n = L.N / kWN, tiles = tiles_n * ((M + kBM - 1) / kBM);
+    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, L.num_sms > 0 ? L.num_sms : 148);
+    note_launch("tc", grid, 1, 1, kThreads, kWSmem, nullptr);
+    tcw_kernel<<<grid, kThreads, kWSmem, st>>>(mx, mw, (__nv_bfloat16*)Y, (int)M, (int)L.N, (int)L.K, (int)tiles,
+                                               (int)tiles_n, L.status_dev);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -291,7 +484,9 @@ cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y
     if (tc3_supported(L)) return launch_tc3(L, X, Wc, Y, M, nullptr, 0, st);
     if (tc2_supported(L)) return launch_tc2(L, X, Wc, Y, M, st);
     // c >= 2 shapes that tc_supported accepts are all taken above (tc2_supported covers them)
-    if (L.c != 1 || (M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
+    if (L.c != 1) return cudaErrorInvalidValue;
+    if (L.N % kWN == 0) return launch_wide(L, X, Wc, Y, M, st);
+    if ((M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
     if (L.BK == 64) return launch_cfg<64>(L, X, Wc, Y, M, st);
     if (L.BK == 128) return launch_cfg<128>(L, X, Wc, Y, M, st);
     if (L.BK == 256) return launch_cfg<256>(L, X, Wc, Y, M, st);

@@ -44,6 +44,10 @@ def _small_cases():
         cases.append(Layer("bf16-small", 6, 4608, 256, c, 256, 32, "bf16", "normal_outliers", "normal_002", 6))
     # wide N: the widest neuron group per CTA
     cases.append(Layer("bf16-small", 8, 1024, 19456, 4, 128, 128, "bf16", "normal", "normal_002", 7))
+    # c = 1 with N a multiple of 256: the persistent 128 x 256 tile kernel (BK plays no part)
+    for M in (1, 130, 333):
+        cases.append(Layer("bf16-small", M, 1024, 512, 1, 128, 128, "bf16", "normal", "normal_002", 3))
+    cases.append(Layer("bf16-small", 200, 768, 768, 1, 256, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2))
     return cases
 
 
@@ -102,6 +106,8 @@ MULTIWAVE = [
     Layer("multiwave", 4096, 1280, 1280, 4, 128, 128, "bf16", "normal_outliers", "uniform_invsqrtk", 2),
     Layer("multiwave", 4096, 4096, 1024, 2, 256, 128, "bf16", "normal", "normal_002", 3),
     Layer("multiwave", 5000, 3072, 1024, 8, 256, 128, "bf16", "normal", "normal_002", 3),
+    # c = 1, 200 tiles of 128 x 256 on 148 SMs: CTAs take two tiles (both accumulators in turn)
+    Layer("multiwave", 2500, 512, 2560, 1, 64, 128, "bf16", "normal", "uniform_invsqrtk", 4),
 ]
 
 

@@ -32,6 +32,8 @@ SHAPES = [
     (960, 256, 2, 48, 16),
     (36, 48, 4, 12, 16),       # K * 2 bytes = 72: plain kernel
     (1280, 640, 4, 128, 128),
+    (768, 96, 2, 96, 48),      # 16 (N-block, K-chunk) units: rows split in two, pairs cut by the range end
+    (512, 160, 2, 64, 80),     # rows split in four ranges of 20: some warps end on a lone row
 ]
 
 
