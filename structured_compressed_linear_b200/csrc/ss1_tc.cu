@@ -7,8 +7,9 @@
 // A operand. (c >= 2 runs in ss1_tc3.cu, or in ss1_tc2.cu for the shapes tc3 does not take;
 // launch_tc below chooses.)
 //
-// One CTA computes a 128-row x 128-column output tile = rows [m0, m0+128) of N-block nb
-// (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs):
+// Two kernels. Where N is a multiple of 256, tcw_kernel (below): persistent CTAs, 128 x 256 output
+// tiles, two TMEM accumulators. Otherwise tc_kernel: one CTA computes a 128-row x 128-column
+// output tile = rows [m0, m0+128) of N-block nb (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs):
 //   * TMA warp      : X[m0:+128, kc*BK:+BK] -> smem (128B-swizzled, 64-column panels) and
 //                     Wc[nb*128:+128, kc*BK:+BK] -> smem (K-major, 128B swizzle).
 //   * MMA thread    : BK/16 x tcgen05.mma.kind::f16 (M=128, N=128, K=16) into one TMEM
