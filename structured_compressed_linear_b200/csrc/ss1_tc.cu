@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                      __uint_as_float(r[q * 8 + 2 * t + 1]));
                             ow[t] = *reinterpret_cast<uint32_t*>(&b);
                         }
-                        *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
+                        if (SS1_SPAN_IN(yrow + col0 + q * 8 - Y, 8, (int64_t)M * N, kSiteTcY))
+                            *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
                     }
                 }
             }
@@ -390,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                      __uint_as_float(r[q * 8 + 2 * t + 1]));
                             ow[t] = *reinterpret_cast<uint32_t*>(&b);
                         }
-                        *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
+                        if (SS1_SPAN_IN(yrow + col0 + q * 8 - Y, 8, (int64_t)M * N, kSiteTcY))
+                            *reinterpret_cast<uint4*>(yrow + col0 + q * 8) = o;
                     }
                 }
             }
