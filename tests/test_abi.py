@@ -180,3 +180,20 @@ def test_checked_build_exports_the_same_entry_points():
         assert hasattr(clib, name), name
     record = ctypes.c_uint64(0)
     assert clib.ss1_bounds_check(None, ctypes.byref(record)) == -1
+
+
+def test_binding_switches_library_and_back():
+    """ss1.use_library routes the module's calls through another build; LIB_PATH switches back."""
+    from structured_compressed_linear_b200 import build
+    from structured_compressed_linear_b200 import ss1
+    build.build()
+    build.build(checked=True)
+    try:
+        normal = ss1.use_library(ss1.LIB_PATH)
+        assert ss1.bounds_check() == (False, 0)
+        checked = ss1.use_library(ss1.CHECKED_LIB_PATH)
+        assert checked._name == ss1.CHECKED_LIB_PATH and ss1.lib() is checked
+        assert ss1.lib()._name != normal._name
+    finally:
+        ss1.use_library(ss1.LIB_PATH)
+    assert ss1.lib()._name == ss1.LIB_PATH
