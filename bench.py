@@ -389,7 +389,8 @@ def run_project(args, layers, wid, peaks, peak_src, dev):
         "data": "synthetic (seeded)", "config": {"workload": f"workload {wid} layer shapes", "l2": "flushed before every step"},
         "layers": per,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src, "kernel": "project_rows_kernel",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src,
+                     "kernel": "project_pairs_kernel" if layers[0].dtype == "bf16" else "project_rows_kernel",
                      "algorithmic_bytes": total_bytes},
         "gpu_launches": args.steps * len(objs), "clocks": sampler.summary(),
     }), flush=True)
