@@ -35,7 +35,6 @@ enum CheckSite : int {
     kSiteTc3Tab, kSiteTc3Bias, kSiteTc2Tab, kSiteTc2Wc, kSiteTc2Y,
     kSiteBwdWc, kSiteBwdTab, kSiteBwdSlot, kSiteBwdE,
     kSiteHashH, kSiteHashPerm, kSiteHashSrc, kSiteHashSlot,
-    kSiteTcY,
     kSiteSelftest = 63,
 };
 #if SS1_CHECKED
