@@ -37,7 +37,7 @@ constexpr int kBN = 128;         // N-block size handled (UMMA N)
 constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kSmemBudget = 200 * 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kSiteTcY = kSiteHashSlot + 1;   // checked build: the Y stores of both kernels here
+[[maybe_unused]] constexpr int kSiteTcY = kSiteHashSlot + 1;   // checked build: the Y stores of both kernels here
 
 template <int BK>
 struct Cfg {
