@@ -219,8 +219,9 @@ SS1_API int ss1_chain_fused(const ss1_handle* layers, int n_layers, int* fused);
  *   dtype : SS1_DTYPE_BF16 or SS1_DTYPE_FP32; the c terms are summed in fp32 and rounded once.
  *   stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  * The caller owns W and Wc. Asynchronous; reads the handle only, so calls may run concurrently.
- * Rows and chunks that are multiples of 16 bytes with 16-byte-aligned W and Wc take the fast
- * kernel; any other shape a plain one. Errors: BAD_HANDLE, INVALID_ARG (NULL pointer, dtype),
+ * Rows and K-chunks of W that are multiples of 16 bytes, with W 16-byte aligned, take the fast
+ * kernels (rows streamed through shared memory; bf16 rows in pairs); any other shape a plain
+ * one. Errors: BAD_HANDLE, INVALID_ARG (NULL pointer, dtype),
  * MISALIGNED (W or Wc not aligned to its element size), CUDA (launch failure).
  */
 SS1_API int ss1_project(ss1_handle h, const void* W, void* Wc, int dtype, void* stream);
