@@ -384,7 +384,7 @@ SS1_API int ss1_test_forward_timeout(ss1_handle h, const void* X, const void* Wc
  * launched: which kernel, its grid, cluster and block. For checking that a launch uses the
  * machine as intended (how many CTAs, how K is split); it has no counterpart on the SS1 pages.
  *   kernel : static name: "tc3" (large-M tensor-core kernel, c >= 2), "tc" (c = 1; a grid of
- *            one CTA per SM where N is a multiple of 256), "tc2",
+ *            at most one CTA per SM where N is a multiple of 256 and M is large), "tc2",
  *            "simt", "dec" (tensor-core decode kernel), "dec_fp8", "smallm"; "" before any launch.
  *   grid_x, grid_y : CTAs of the grid (grid_y: K-splits where the kernel splits K).
  *   cluster_y : CTAs per thread-block cluster along y (1: no cluster).

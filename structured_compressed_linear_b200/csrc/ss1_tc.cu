@@ -7,8 +7,9 @@
 // A operand. (c >= 2 runs in ss1_tc3.cu, or in ss1_tc2.cu for the shapes tc3 does not take;
 // launch_tc below chooses.)
 //
-// Two kernels. Where N is a multiple of 256, tcw_kernel (below): persistent CTAs, 128 x 256 output
-// tiles, two TMEM accumulators. Otherwise tc_kernel: one CTA computes a 128-row x 128-column
+// Two kernels. Where N is a multiple of 256 and the layer spans more than one wave of 128 x 128
+// tiles, tcw_kernel (below): persistent CTAs, 128 x 256 output tiles, two TMEM accumulators.
+// Otherwise tc_kernel: one CTA computes a 128-row x 128-column
 // output tile = rows [m0, m0+128) of N-block nb (BN = 128 = the UMMA N). Per K-chunk kc (BK inputs):
 //   * TMA warp      : X[m0:+128, kc*BK:+BK] -> smem (128B-swizzled, 64-column panels) and
 //                     Wc[nb*128:+128, kc*BK:+BK] -> smem (K-major, 128B swizzle).
@@ -489,7 +490,11 @@ cudaError_t launch_tc(const ss1_layer& L, const void* X, const void* Wc, void* Y
     if (tc2_supported(L)) return launch_tc2(L, X, Wc, Y, M, st);
     // c >= 2 shapes that tc_supported accepts are all taken above (tc2_supported covers them)
     if (L.c != 1) return cudaErrorInvalidValue;
-    if (L.N % kWN == 0) return launch_wide(L, X, Wc, Y, M, st);
+    // The wide kernel where the 128 x 128 grid would need more than one wave. Below that, twice
+    // the CTAs of 128 x 128 tiles stream Wc faster (each SM's TMA rate bounds a CTA there): at
+    // M = 64 on 4096 x 4096, 16 wide CTAs took 36 us against 28 us for 32 narrow ones.
+    const int64_t wide_tiles = (M + kBM - 1) / kBM * (L.N / kWN);
+    if (L.N % kWN == 0 && 2 * wide_tiles > (int64_t)L.num_sms) return launch_wide(L, X, Wc, Y, M, st);
     if ((M + kBM - 1) / kBM > 65535) return cudaErrorInvalidValue;
     if (L.BK == 64) return launch_cfg<64>(L, X, Wc, Y, M, st);
     if (L.BK == 128) return launch_cfg<128>(L, X, Wc, Y, M, st);
